@@ -1,0 +1,200 @@
+/*
+ * pagedattn.h -- C ABI of libpagedattn.so: a paged KV cache for single-query
+ * decode attention on NVIDIA B200 (sm_100a).
+ *
+ * The pages this follows:
+ *   [card]   "PagedAttention" (llm-engineer.pages.dev, LLM inference / vLLM path)
+ *   [vllm]   "vLLM KV Cache and PagedAttention Explained" (hrletsgo.me)
+ *   [velog]  "vLLM의 PagedAttention 아키텍처와 GPU 메모리 최적화 원리" (velog.io, @min_tech)
+ *
+ * Cache layout ([velog] section 4): K and V are each one tensor
+ *   [NB, H, S, D] = [num_blocks, num_heads, block_size, head_dim], D fastest,
+ * so the S x D slab of one (block, head) is contiguous. Token t of a request
+ * lives in physical block block_table[t / S] at offset t % S ([card]
+ * "OS paging과 같은 발상"; [vllm] Step 5 "PagedAttention in vLLM"). A slot is
+ * the integer block * S + offset ([vllm] Step 6 "Decode": "slot 6 of block 42").
+ *
+ * Conventions for every call:
+ *   - Errors are return codes; nothing throws across the ABI. Arguments are
+ *     validated on the host before anything is launched; a rejected call
+ *     launches nothing and changes nothing.
+ *   - Device calls take device pointers owned by the caller and enqueue work
+ *     on `stream` (a cudaStream_t; NULL = the legacy default stream). They do
+ *     not synchronise. They allocate no device memory.
+ *   - Device-side range checks are always on: a block id outside [0, NB), a
+ *     seq_len outside [0, MB * S] or a slot at or past NB * S is never
+ *     dereferenced; the kernel skips it and sets a per-device error word that
+ *     pa_get_device_error() reads and clears.
+ *   - The host allocator is not thread-safe: one caller thread per pa_alloc.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = 1,      /* bad argument: null pointer, bad size, misalignment, unknown id */
+  PA_ERR_OOM = 2,          /* the block pool cannot satisfy a grow; state unchanged */
+  PA_ERR_OUT_OF_RANGE = 3, /* an index past an allocated range (or a device range check fired) */
+  PA_ERR_CUDA = 4          /* a CUDA launch or copy failed */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_F32 = 2 } pa_dtype; /* PA_F32 only for decode output */
+
+/* Bits of the device error word (pa_get_device_error). */
+#define PA_DEVERR_BLOCK_ID 0x1u /* a block table entry outside [0, NB) was skipped */
+#define PA_DEVERR_SEQ_LEN 0x2u  /* a seq_len outside [0, MB * S] was clamped */
+#define PA_DEVERR_SLOT 0x4u     /* an append slot at or past NB * S was skipped */
+#define PA_DEVERR_TIMEOUT 0x8u  /* a pipeline wait gave up after about one second */
+
+/* Human-readable name of a status code (static storage). */
+const char* pa_status_string(pa_status s);
+
+/* ABI version of this library (major * 100 + minor). */
+int pa_version(void);
+
+/* ---------------------------------------------------------------------------
+ * KV append: the slot_mapping scatter.
+ * [vllm] Step 6 "Decode" / Step 7 item 5: the new token's K/V is stored in its
+ * slot (slot 6 of block 42); Step 6 "Prefill": K1..K6/V1..V6 written to the cache.
+ *
+ *   k, v          [T, H, D] new tokens' keys and values, dtype `dt`, contiguous
+ *   slot_mapping  [T] int64; token t goes to block slot/S, offset slot%S for
+ *                 every head; a negative slot skips the token (padding). Slots
+ *                 in one call must be distinct (duplicates: one of the writes wins)
+ *   k_cache, v_cache  [NB, H, S, D], dtype `dt`, written in place
+ *   dt            PA_F16 or PA_BF16
+ * Requires D % 8 == 0 and 16-byte aligned k, v, k_cache, v_cache. T == 0 is a
+ * no-op. Bit-exact copy: no arithmetic touches the values.
+ * ------------------------------------------------------------------------- */
+pa_status pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
+                       void* v_cache, int T, int H, int D, int S, int NB, pa_dtype dt,
+                       void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Paged decode attention.
+ * [vllm] "Appendix: The Attention Score Formula": out = softmax(q K^T * scale) V
+ * for one query per (request, head), computed by walking the request's block
+ * table and reading each physical block in place, with a running softmax
+ * ([card] "Kernel은 무엇이 달라지는가": no gather into a contiguous tensor).
+ * Long contexts are split into partitions of `partition` tokens whose partial
+ * results are merged by a log-sum-exp reduce ([card] "헷갈리기 쉬운 구분":
+ * FlashDecoding).
+ *
+ *   out           [B, H, D], dtype out_dt (PA_F32, PA_F16 or PA_BF16). fp16/bf16
+ *                 output is the round-to-nearest-even of the fp32 result
+ *   q             [B, H, D], dtype dt
+ *   k_cache, v_cache [NB, H, S, D], dtype dt
+ *   block_tables  [B, MB] int32; entries past ceil(seq_lens[i] / S) are never read
+ *   seq_lens      [B] int32 on the device; request i attends to exactly its first
+ *                 seq_lens[i] cached tokens; 0 gives an all-zero output row
+ *   scale         multiplies q . k (1/sqrt(D) for the pages' formula)
+ *   dt            PA_F16 or PA_BF16; D in {64, 128, 256}; S in {8, 16, 32}
+ *   partition     0 = choose automatically, -1 = never split, > 0 = split into
+ *                 partitions of this many tokens (a multiple of S)
+ *   max_seq_len   a host-side upper bound on seq_lens (sizes the grid); must be
+ *                 <= MB * S. Requests longer than it are clamped and flagged
+ *   workspace     device scratch of ws_bytes >= pa_decode_workspace_bytes(...)
+ *                 for the same arguments; may be NULL when that size is 0. The
+ *                 library keeps no pointer to it after the call's work ends
+ * Requires 16-byte aligned q, k_cache, v_cache, out and workspace.
+ * ------------------------------------------------------------------------- */
+size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, int partition);
+
+/* The partition length (tokens) and the number of partitions pa_decode will use
+ * for these arguments on the current device; *partition_tokens = 0 and
+ * *num_partitions = 1 mean a single pass with no workspace. */
+pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partition,
+                         int* partition_tokens, int* num_partitions);
+
+pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
+                    const void* v_cache, const int32_t* block_tables, int MB,
+                    const int32_t* seq_lens, float scale, int B, int H, int D, int S, int NB,
+                    pa_dtype dt, int partition, int max_seq_len, void* workspace,
+                    size_t ws_bytes, void* stream);
+
+/* Split-KV workspace layout, for tests that inspect the partition pass
+ * (NP = number of partitions, all fp32, offsets in bytes from `workspace`):
+ *   m   [B, H, NP] at 0                 max of scale * q.k * log2(e) (base-2 units)
+ *   l   [B, H, NP] at B*H*NP*4          sum of 2^(s - m) over the partition
+ *   acc [B, H, NP, D] at align256(B*H*NP*8)   sum of 2^(s - m) * V, unnormalised
+ * Only partitions p < ceil(seq_lens[i] / partition) of requests with more than
+ * one partition are written. */
+
+/* Reads and clears the device error word of the current device after
+ * synchronising `stream`. *flags receives PA_DEVERR_* bits (0 = clean).
+ * Returns PA_OK, or PA_ERR_CUDA if the read failed. */
+pa_status pa_get_device_error(void* stream, uint32_t* flags);
+
+/* ---------------------------------------------------------------------------
+ * Host block allocator ([vllm] 5단계, Step 5-8; [card] "무엇이 좋아지는가").
+ * A pool of NB physical blocks of S tokens. Each sequence owns a block table
+ * that grows on demand (ceil(len / S) blocks; a new block when the length
+ * crosses a block boundary) and returns its blocks to the pool when freed.
+ * The free list is a LIFO stack: growth pops ids one at a time and appends them
+ * in pop order; a freed sequence pushes its ids back in logical order, so they
+ * are the first handed out again. The library owns the state.
+ * ------------------------------------------------------------------------- */
+typedef struct pa_alloc pa_alloc;
+
+/* initial_order: NULL, or a permutation of [0, NB) listing the order in which
+ * ids are first handed out (NULL = 0, 1, 2, ...). Shuffling is the caller's
+ * choice: pass a shuffled order. */
+pa_status pa_alloc_create(int NB, int S, const int32_t* initial_order, pa_alloc** out);
+void pa_alloc_destroy(pa_alloc* a);
+
+/* Creates seq_id if unknown, then grows it to new_len tokens (new_len >= its
+ * current length, else PA_ERR_INVALID). PA_ERR_OOM if the pool is short: the
+ * state is then unchanged (an unknown seq_id is not created). */
+pa_status pa_seq_grow(pa_alloc* a, int64_t seq_id, int new_len);
+
+/* Returns every block of seq_id to the pool and forgets seq_id. */
+pa_status pa_seq_free(pa_alloc* a, int64_t seq_id);
+
+/* Current length (tokens) of seq_id. */
+pa_status pa_seq_len(const pa_alloc* a, int64_t seq_id, int* len);
+
+/* Copies seq_id's block table (logical order) into dst[0..cap); *n receives
+ * its length. PA_ERR_OUT_OF_RANGE if cap is too small (nothing copied). */
+pa_status pa_seq_block_table(const pa_alloc* a, int64_t seq_id, int32_t* dst, int cap, int* n);
+
+/* Host slot mapping: for each sequence k, tokens start_pos[k] .. start_pos[k]
+ * + n_tok[k] - 1 are written to dst in order, as table[pos / S] * S + pos % S.
+ * dst holds sum(n_tok) entries. PA_ERR_OUT_OF_RANGE if a position is not yet
+ * allocated (grow first). */
+pa_status pa_build_slot_mapping(const pa_alloc* a, const int64_t* seq_ids, const int* start_pos,
+                                const int* n_tok, int n_seq, int64_t* dst);
+
+/* Host block tables [n_seq, MB] int32, padded with -1. PA_ERR_OUT_OF_RANGE if
+ * a table has more than MB blocks. */
+pa_status pa_build_block_tables(const pa_alloc* a, const int64_t* seq_ids, int n_seq, int MB,
+                                int32_t* dst);
+
+/* One decode step's host work for n_seq sequences in one call: grows each
+ * sequence by n_new tokens (all-or-nothing: on PA_ERR_OOM nothing changes),
+ * then writes the new tokens' slots (dst_slots [n_seq * n_new], sequence-major),
+ * the padded block tables (dst_tables [n_seq, MB]) and the new lengths
+ * (dst_lens [n_seq]). Any of the three outputs may be NULL to skip it. */
+pa_status pa_prepare_step(pa_alloc* a, const int64_t* seq_ids, int n_seq, int n_new, int MB,
+                          int64_t* dst_slots, int32_t* dst_tables, int32_t* dst_lens);
+
+/* Pool statistics: free blocks, tokens held (sum of lengths) and empty slots in
+ * held blocks (the tail waste of [vllm] Step 5 "Why Waste Stays Below 4%"). */
+pa_status pa_alloc_stats(const pa_alloc* a, int* free_blocks, int64_t* used_slots,
+                         int64_t* wasted_slots);
+
+/* Copies the free list, bottom of the stack first (the last entry is handed out
+ * next), into dst[0..cap); *n receives its length. For bit-exact tests. */
+pa_status pa_alloc_dump(const pa_alloc* a, int32_t* free_list, int cap, int* n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

@@ -1,1 +1,15 @@
-"""B200-native paged KV cache decode path (placeholder; binding added with the boundary)."""
+"""B200-native (sm_100a) paged KV cache: slot_mapping append, block-table-driven
+single-query decode attention with split-KV, and a host block allocator, all
+behind the C ABI of ``libpagedattn.so`` (``include/pagedattn.h``).
+
+The Python layer is marshalling only (``binding``); every step of the path runs
+in the library. Importing this package does not load the library; the first
+call does, and raises if it was never built.
+"""
+
+from .binding import (  # noqa: F401
+    PA_BF16, PA_DEVERR_BLOCK_ID, PA_DEVERR_SEQ_LEN, PA_DEVERR_SLOT, PA_DEVERR_TIMEOUT,
+    PA_ERR_CUDA, PA_ERR_INVALID, PA_ERR_OOM, PA_ERR_OUT_OF_RANGE, PA_F16, PA_F32, PA_OK,
+    BlockAllocator, PagedAttnError, lib, pa_decode, pa_decode_plan, pa_decode_workspace_bytes,
+    pa_get_device_error, pa_kv_append,
+)

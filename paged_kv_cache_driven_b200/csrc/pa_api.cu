@@ -1,0 +1,241 @@
+// The device half of the C ABI (pagedattn.h): argument validation, launch
+// planning and kernel dispatch for pa_kv_append and pa_decode, and the device
+// error word. Every check runs on the host before anything is launched.
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+#include "pa_append.cuh"
+#include "pa_decode.cuh"
+#include "pagedattn.h"
+
+namespace {
+
+constexpr int kDefaultPartition = 512;  // tokens per split-KV partition when splitting
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool cache_dtype_ok(pa_dtype dt) { return dt == PA_F16 || dt == PA_BF16; }
+
+bool out_dtype_ok(pa_dtype dt) { return dt == PA_F16 || dt == PA_BF16 || dt == PA_F32; }
+
+bool decode_shape_ok(int D, int S) {
+  return (D == 64 || D == 128 || D == 256) && (S == 8 || S == 16 || S == 32);
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Chooses the partition length. Returns false on an invalid `partition`.
+//   -1      never split: one partition covering any length up to MB * S
+//   > 0     that many tokens (a multiple of S)
+//   0       automatic: split only when the longest request spans more than
+//           one default partition
+bool plan(int S, int max_seq_len, int partition, int* P_out, int* NP_out) {
+  if (max_seq_len < 0 || S <= 0) return false;
+  int P;
+  if (partition < 0) {
+    if (partition != -1) return false;
+    *P_out = 0;
+    *NP_out = 1;
+    return true;
+  } else if (partition > 0) {
+    if (partition % S != 0) return false;
+    P = partition;
+  } else {
+    P = kDefaultPartition;
+  }
+  const int64_t np = ceil_div(max_seq_len, P);
+  if (np <= 1) {
+    *P_out = 0;
+    *NP_out = 1;
+    return true;
+  }
+  if (np * P > INT_MAX) return false;
+  *P_out = P;
+  *NP_out = static_cast<int>(np);
+  return true;
+}
+
+size_t workspace_for(int B, int H, int D, int NP) {
+  if (NP <= 1) return 0;
+  const size_t n = static_cast<size_t>(B) * H * NP;
+  return align256(n * 2 * sizeof(float)) + n * D * sizeof(float);
+}
+
+pa_status cuda_status() {
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, typename TO, int D, int S>
+pa_status launch_decode(const pa::DecodeParams& prm, cudaStream_t stream) {
+  using Tl = pa::DecodeTiling<D, S>;
+  auto kern = pa::paged_decode_partition_kernel<T, TO, D, S>;
+  // The shared-memory opt-in is a per-device property of the function.
+  static bool configured[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tl::SMEM) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    configured[dev] = true;
+  }
+  const dim3 grid(prm.NP, prm.H, prm.B);
+  kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
+  if (prm.NP > 1) {
+    pa::splitkv_reduce_kernel<TO, D><<<dim3(prm.H, prm.B), 128, 0, stream>>>(prm);
+  }
+  return cuda_status();
+}
+
+template <typename T, typename TO>
+pa_status dispatch_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t st) {
+#define PA_CASE(DD, SS) \
+  if (D == DD && S == SS) return launch_decode<T, TO, DD, SS>(prm, st);
+  PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
+  PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
+  PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
+#undef PA_CASE
+  return PA_ERR_INVALID;
+}
+
+template <typename T>
+pa_status dispatch_out(const pa::DecodeParams& prm, pa_dtype out_dt, int D, int S,
+                       cudaStream_t st) {
+  switch (out_dt) {
+    case PA_F32: return dispatch_shape<T, float>(prm, D, S, st);
+    case PA_F16: return dispatch_shape<T, __half>(prm, D, S, st);
+    case PA_BF16: return dispatch_shape<T, __nv_bfloat16>(prm, D, S, st);
+  }
+  return PA_ERR_INVALID;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID: return "PA_ERR_INVALID";
+    case PA_ERR_OOM: return "PA_ERR_OOM";
+    case PA_ERR_OUT_OF_RANGE: return "PA_ERR_OUT_OF_RANGE";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+  }
+  return "PA_ERR_UNKNOWN";
+}
+
+int pa_version(void) { return 100; }
+
+pa_status pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping, void* k_cache,
+                       void* v_cache, int T, int H, int D, int S, int NB, pa_dtype dt,
+                       void* stream) {
+  if (T < 0 || H <= 0 || D <= 0 || S <= 0 || NB < 0 || !cache_dtype_ok(dt)) return PA_ERR_INVALID;
+  if (D % 8 != 0) return PA_ERR_INVALID;  // rows move as 16-byte vectors
+  if (T == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  const int vpr = D / 8;
+  const int64_t total = static_cast<int64_t>(T) * H * vpr;
+  const int64_t n_slots = static_cast<int64_t>(NB) * S;
+  int64_t blocks = ceil_div(total, 256);
+  const int64_t cap = 148LL * 16;  // grid-stride beyond ~16 CTAs per SM
+  if (blocks > cap) blocks = cap;
+  pa::kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                         static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total, H, vpr, S, n_slots);
+  return cuda_status();
+}
+
+pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partition,
+                         int* partition_tokens, int* num_partitions) {
+  (void)B;
+  (void)H;
+  (void)D;
+  if (!partition_tokens || !num_partitions) return PA_ERR_INVALID;
+  int P, NP;
+  if (!plan(S, max_seq_len, partition, &P, &NP)) return PA_ERR_INVALID;
+  *partition_tokens = P;
+  *num_partitions = NP;
+  return PA_OK;
+}
+
+size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, int partition) {
+  int P, NP;
+  if (B < 0 || H <= 0 || D <= 0 || !plan(S, max_seq_len, partition, &P, &NP)) return 0;
+  return workspace_for(B, H, D, NP);
+}
+
+pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
+                    const void* v_cache, const int32_t* block_tables, int MB,
+                    const int32_t* seq_lens, float scale, int B, int H, int D, int S, int NB,
+                    pa_dtype dt, int partition, int max_seq_len, void* workspace,
+                    size_t ws_bytes, void* stream) {
+  if (B < 0 || H <= 0 || NB < 0 || MB < 0) return PA_ERR_INVALID;
+  if (!cache_dtype_ok(dt) || !out_dtype_ok(out_dt) || !decode_shape_ok(D, S)) return PA_ERR_INVALID;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID;
+  if (B > 65535 || H > 65535) return PA_ERR_INVALID;  // grid y / z limits
+  const int64_t L_max = static_cast<int64_t>(MB) * S;
+  if (L_max > INT_MAX || max_seq_len < 0 || max_seq_len > L_max) return PA_ERR_INVALID;
+  int P, NP;
+  if (!plan(S, max_seq_len, partition, &P, &NP)) return PA_ERR_INVALID;
+  if (B == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || MB == 0)
+    return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  const size_t need = workspace_for(B, H, D, NP);
+  if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace))) return PA_ERR_INVALID;
+
+  pa::DecodeParams prm{};
+  prm.out = out;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.block_tables = block_tables;
+  prm.seq_lens = seq_lens;
+  prm.q_scale = scale * 1.4426950408889634f;  // log2(e)
+  prm.MB = MB;
+  prm.B = B;
+  prm.H = H;
+  prm.NB = NB;
+  if (NP > 1) {
+    const size_t n = static_cast<size_t>(B) * H * NP;
+    prm.ws_m = static_cast<float*>(workspace);
+    prm.ws_l = prm.ws_m + n;
+    prm.ws_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                          align256(n * 2 * sizeof(float)));
+    prm.P = P;
+    prm.NP = NP;
+    prm.L_cap = static_cast<int>(std::min<int64_t>(L_max, static_cast<int64_t>(NP) * P));
+  } else {
+    prm.P = static_cast<int>(L_max > 0 ? L_max : S);  // one partition covers every block
+    prm.NP = 1;
+    prm.L_cap = static_cast<int>(L_max);
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == PA_F16) return dispatch_out<__half>(prm, out_dt, D, S, st);
+  return dispatch_out<__nv_bfloat16>(prm, out_dt, D, S, st);
+}
+
+pa_status pa_get_device_error(void* stream, uint32_t* flags) {
+  if (!flags) return PA_ERR_INVALID;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, pa::g_error_word, sizeof(v)) != cudaSuccess) return PA_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(pa::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return PA_ERR_CUDA;
+  *flags = v;
+  return PA_OK;
+}
+
+}  // extern "C"

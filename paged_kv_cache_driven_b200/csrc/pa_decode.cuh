@@ -1,0 +1,316 @@
+// Paged single-query decode attention for sm_100a: the partition pass and the
+// log-sum-exp reduce.
+//
+// What it computes: "vLLM KV Cache and PagedAttention Explained", "Appendix:
+// The Attention Score Formula" -- out = softmax(q K^T * scale) V, carried out by
+// walking the block table, fetching each block's keys, computing partial
+// scores, updating a running softmax normaliser, weighting the values and
+// accumulating, one block at a time. The blocks are read where they are
+// ("PagedAttention" card, "Kernel은 무엇이 달라지는가"); long contexts are cut into
+// partitions whose partial results a second kernel merges (FlashDecoding, the
+// same card, "헷갈리기 쉬운 구분").
+//
+// Mapping onto the B200 (this is not the pages' shared-memory sketch, which
+// names no hardware):
+//   * one CTA per (partition, head, request); NW warps split the partition's
+//     blocks into contiguous runs; each warp is an independent pipeline.
+//   * a warp's block ids are hoisted 32 at a time with one coalesced load and
+//     prefetched one chunk ahead, so the dependent table load never stalls
+//     the copy stream.
+//   * each physical block's K slab and V slab (S x D contiguous, the
+//     [Block, Head, Block_Size, Head_D] layout) arrive in shared memory by two
+//     1-D bulk async copies (cp.async.bulk, TMA engine, no tensor map needed)
+//     on an mbarrier; NS stages per warp keep several blocks in flight.
+//   * lane l owns D/32 consecutive elements of q, of every K/V row and of the
+//     output accumulator. The S partial dot products of a block are summed
+//     across lanes with a transposing butterfly: S values per lane become one
+//     finished score per lane in S-1+log2(32/S) shuffles.
+//   * the softmax runs in base 2 (q is pre-scaled by scale * log2 e) with an
+//     fp32 running max / sum; masked tokens are removed by selection, never by
+//     multiplying, so NaN in unused slots cannot leak.
+//   * no tensor cores: one query per head is a matrix-vector product.
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+struct DecodeParams {
+  void* out;                   // [B, H, D] final output (dtype TO)
+  const void* q;               // [B, H, D]
+  const void* k_cache;         // [NB, H, S, D]
+  const void* v_cache;         // [NB, H, S, D]
+  const int32_t* block_tables; // [B, MB]
+  const int32_t* seq_lens;     // [B]
+  float* ws_m;                 // [B, H, NP]
+  float* ws_l;                 // [B, H, NP]
+  float* ws_acc;               // [B, H, NP, D]
+  float q_scale;               // scale * log2(e)
+  int MB, B, H, NB;
+  int P;     // tokens per partition (multiple of S)
+  int NP;    // partitions in the grid
+  int L_cap; // lengths are clamped to this (MB*S, or NP*P when split)
+};
+
+// Shared-memory budget of one CTA: NW warps x NS stages x (K + V slabs).
+template <int D, int S>
+struct DecodeTiling {
+  static constexpr int SLAB = S * D * 2;
+  static constexpr int STAGE = 2 * SLAB;
+  static constexpr int NS = STAGE <= 4096 ? 4 : 2;
+  static constexpr int NW_RAW = 65536 / (NS * STAGE);
+  static constexpr int NW = NW_RAW < 1 ? 1 : (NW_RAW > 8 ? 8 : NW_RAW);
+  static constexpr int SMEM_PIPE = NW * NS * STAGE;
+  static constexpr int SMEM_BARS = NW * NS * 8;
+  static constexpr int SMEM_MERGE = NW * (D + 2) * 4;
+  static constexpr int SMEM = SMEM_PIPE + SMEM_BARS + SMEM_MERGE;
+};
+
+// Sums S per-lane partial dot products across the warp. On return v[0] of lane
+// l holds the full dot product of token l / (32 / S) of the block.
+template <int S>
+__device__ __forceinline__ float transpose_reduce(float (&v)[S], int lane) {
+  // Halving steps: exchange half the values with lane ^ off, keep the other half.
+#pragma unroll
+  for (int n = S, off = 16; n > 1; n >>= 1, off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = upper ? v[j] : v[j + n / 2];
+      const float keep = upper ? v[j + n / 2] : v[j];
+      v[j] = keep + __shfl_xor_sync(kFullMask, send, off);
+    }
+  }
+  // Lanes sharing a token still hold disjoint partial sums: finish them.
+  float r = v[0];
+#pragma unroll
+  for (int off = 16 / S; off >= 1; off >>= 1) r += __shfl_xor_sync(kFullMask, r, off);
+  return r;
+}
+
+template <typename T, typename TO, int D, int S>
+__global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
+    paged_decode_partition_kernel(const DecodeParams p) {
+  using Tl = DecodeTiling<D, S>;
+  constexpr int NW = Tl::NW, NS = Tl::NS, SLAB = Tl::SLAB, STAGE = Tl::STAGE;
+  constexpr int DL = D / 32;   // elements per lane
+  constexpr int DUP = 32 / S;  // lanes holding the same token's score
+
+  const int part = blockIdx.x;
+  const int h = blockIdx.y;
+  const int i = blockIdx.z;
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+
+  int L = __ldg(p.seq_lens + i);
+  if (L < 0 || L > p.L_cap) {
+    if (threadIdx.x == 0 && part == 0 && h == 0) raise_error(PA_DEVERR_SEQ_LEN);
+    L = L < 0 ? 0 : p.L_cap;
+  }
+  const int nparts = (L + p.P - 1) / p.P;
+  if (part > 0 && part >= nparts) return;  // nothing here (part 0 writes the L == 0 zeros)
+  const bool direct = nparts <= 1;          // the only partition: write the final output
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tl::SMEM_PIPE);
+  float* merge = reinterpret_cast<float*>(smem + Tl::SMEM_PIPE + Tl::SMEM_BARS);
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int k = 0; k < NW * NS; ++k) mbar_init(&bars[k], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // This partition's blocks, split into NW contiguous runs.
+  const int t_beg = part * p.P;
+  const int t_end = min(t_beg + p.P, L);
+  const int blk_beg = t_beg / S;
+  const int blk_end = t_end > t_beg ? (t_end + S - 1) / S : blk_beg;
+  const int nb = blk_end - blk_beg;
+  const int wb = blk_beg + static_cast<int>((static_cast<int64_t>(nb) * w) / NW);
+  const int we = blk_beg + static_cast<int>((static_cast<int64_t>(nb) * (w + 1)) / NW);
+  const int nbw = we - wb;
+
+  // q, pre-scaled so that scores come out in base-2 units.
+  float qf[DL];
+  {
+    const T* qp = static_cast<const T*>(p.q) + (static_cast<int64_t>(i) * p.H + h) * D + lane * DL;
+    load_row<T, DL>(qp, qf);
+#pragma unroll
+    for (int e = 0; e < DL; ++e) qf[e] *= p.q_scale;
+  }
+
+  uint64_t* bar = bars + w * NS;
+  uint8_t* stage0 = smem + w * NS * STAGE;
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(i) * p.MB;
+  const uint8_t* kbase =
+      static_cast<const uint8_t*>(p.k_cache) + static_cast<int64_t>(h) * SLAB;
+  const uint8_t* vbase =
+      static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(h) * SLAB;
+  const int64_t block_stride = static_cast<int64_t>(p.H) * SLAB;  // bytes per physical block
+  const uint64_t policy = policy_evict_first();
+
+  // Block-id prefetch: ids_a holds the chunk of 32 being issued, ids_b the next.
+  int ids_a = (wb + lane < we) ? __ldg(trow + wb + lane) : -1;
+  int ids_b = (wb + 32 + lane < we) ? __ldg(trow + wb + 32 + lane) : -1;
+  uint32_t bad = 0;  // bit s: stage s holds a block whose id was out of range
+  int issued = 0;
+
+  auto issue_next = [&]() {
+    if (issued >= nbw) return;
+    if ((issued & 31) == 0 && issued > 0) {
+      ids_a = ids_b;
+      const int nx = wb + issued + 32 + lane;
+      ids_b = nx < we ? __ldg(trow + nx) : -1;
+    }
+    const int id = __shfl_sync(kFullMask, ids_a, issued & 31);
+    const int s = issued % NS;
+    const bool ok = static_cast<unsigned>(id) < static_cast<unsigned>(p.NB);
+    if (lane == 0) {
+      if (ok) {
+        mbar_arrive_expect_tx(&bar[s], 2 * SLAB);
+        const int64_t off = static_cast<int64_t>(id) * block_stride;
+        bulk_g2s(stage0 + s * STAGE, kbase + off, SLAB, &bar[s], policy);
+        bulk_g2s(stage0 + s * STAGE + SLAB, vbase + off, SLAB, &bar[s], policy);
+      } else {
+        raise_error(PA_DEVERR_BLOCK_ID);
+        mbar_arrive(&bar[s]);  // completes the phase with no data; the block is skipped
+      }
+    }
+    bad = ok ? (bad & ~(1u << s)) : (bad | (1u << s));
+    ++issued;
+  };
+
+#pragma unroll
+  for (int k = 0; k < NS; ++k) issue_next();
+
+  float m = -INFINITY;  // running max (base-2 units), warp-uniform
+  float lsum = 0.f;     // running sum of 2^(s - m); counted once per token
+  float acc[DL];
+#pragma unroll
+  for (int e = 0; e < DL; ++e) acc[e] = 0.f;
+  const int tok = lane / DUP;
+
+  for (int k = 0; k < nbw; ++k) {
+    const int s = k % NS;
+    if (!mbar_wait_bounded(&bar[s], (k / NS) & 1)) {
+      if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+      // drain what this warp still has in flight (bounded), then stop
+      for (int r = k; r < issued; ++r) mbar_wait_bounded(&bar[r % NS], (r / NS) & 1);
+      break;
+    }
+    if (!((bad >> s) & 1u)) {
+      const int j = wb + k;
+      const int nvalid = min(S, L - j * S);
+      const uint8_t* ks = stage0 + s * STAGE;
+      const uint8_t* vs = ks + SLAB;
+
+      float part_dot[S];
+#pragma unroll
+      for (int t = 0; t < S; ++t) {
+        float kf[DL];
+        load_row<T, DL>(ks + (t * D + lane * DL) * 2, kf);
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) a = fmaf(qf[e], kf[e], a);
+        part_dot[t] = a;
+      }
+      const float score = transpose_reduce<S>(part_dot, lane);
+      const bool valid = tok < nvalid;
+      const float sc = valid ? score : -INFINITY;
+      float mb = sc;
+#pragma unroll
+      for (int off = DUP; off < 32; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(kFullMask, mb, off));
+      const float m_new = fmaxf(m, mb);
+      const float alpha = exp2f(m - m_new);
+      const float pr = valid ? exp2f(sc - m_new) : 0.f;
+      lsum = lsum * alpha + ((lane % DUP) == 0 ? pr : 0.f);
+#pragma unroll
+      for (int e = 0; e < DL; ++e) acc[e] *= alpha;
+#pragma unroll
+      for (int t = 0; t < S; ++t) {
+        if (t < nvalid) {  // warp-uniform
+          const float pt = __shfl_sync(kFullMask, pr, t * DUP);
+          float vf[DL];
+          load_row<T, DL>(vs + (t * D + lane * DL) * 2, vf);
+#pragma unroll
+          for (int e = 0; e < DL; ++e) acc[e] = fmaf(pt, vf[e], acc[e]);
+        }
+      }
+      m = m_new;
+    }
+    __syncwarp();
+    issue_next();
+  }
+
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, off);
+
+  // Merge the NW warps' (m, l, acc) in shared memory.
+  float* m_s = merge;
+  float* l_s = merge + NW;
+  float* acc_s = merge + 2 * NW;
+#pragma unroll
+  for (int e = 0; e < DL; ++e) acc_s[w * D + lane * DL + e] = acc[e];
+  if (lane == 0) {
+    m_s[w] = m;
+    l_s[w] = lsum;
+  }
+  __syncthreads();
+
+  float M = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < NW; ++u) M = fmaxf(M, m_s[u]);
+  float wgt[NW];
+  float Ltot = 0.f;
+#pragma unroll
+  for (int u = 0; u < NW; ++u) {
+    wgt[u] = m_s[u] == -INFINITY ? 0.f : exp2f(m_s[u] - M);
+    Ltot = fmaf(wgt[u], l_s[u], Ltot);
+  }
+  const int64_t ih = static_cast<int64_t>(i) * p.H + h;
+  for (int d = threadIdx.x; d < D; d += NW * 32) {
+    float a = 0.f;
+#pragma unroll
+    for (int u = 0; u < NW; ++u) a = fmaf(wgt[u], acc_s[u * D + d], a);
+    if (direct) {
+      const float o = Ltot > 0.f ? a / Ltot : 0.f;
+      static_cast<TO*>(p.out)[ih * D + d] = to_out<TO>(o);
+    } else {
+      p.ws_acc[(ih * p.NP + part) * D + d] = a;
+    }
+  }
+  if (!direct && threadIdx.x == 0) {
+    p.ws_m[ih * p.NP + part] = M;
+    p.ws_l[ih * p.NP + part] = Ltot;
+  }
+}
+
+// Merges the partitions of every (request, head) that has more than one:
+//   M = max_p m_p;  out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.
+template <typename TO, int D>
+__global__ void __launch_bounds__(128) splitkv_reduce_kernel(const DecodeParams p) {
+  const int h = blockIdx.x;
+  const int i = blockIdx.y;
+  int L = __ldg(p.seq_lens + i);
+  L = L < 0 ? 0 : (L > p.L_cap ? p.L_cap : L);
+  const int nparts = (L + p.P - 1) / p.P;
+  if (nparts <= 1) return;  // written by the partition pass
+  const int64_t ih = static_cast<int64_t>(i) * p.H + h;
+  const float* m = p.ws_m + ih * p.NP;
+  const float* l = p.ws_l + ih * p.NP;
+  const float* acc = p.ws_acc + ih * p.NP * D;
+
+  float M = -INFINITY;
+  for (int q = 0; q < nparts; ++q) M = fmaxf(M, m[q]);
+  float Ltot = 0.f;
+  for (int q = 0; q < nparts; ++q) Ltot = fmaf(exp2f(m[q] - M), l[q], Ltot);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float a = 0.f;
+    for (int q = 0; q < nparts; ++q) a = fmaf(exp2f(m[q] - M), acc[static_cast<int64_t>(q) * D + d], a);
+    static_cast<TO*>(p.out)[ih * D + d] = to_out<TO>(Ltot > 0.f ? a / Ltot : 0.f);
+  }
+}
+
+}  // namespace pa

@@ -1,0 +1,165 @@
+// Device-side building blocks shared by the append and decode kernels:
+// the per-device error word, mbarrier / bulk-copy wrappers (inline PTX for
+// sm_100a), and 16-bit <-> fp32 conversions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "pagedattn.h"
+
+namespace pa {
+
+// One word per device; kernels OR PA_DEVERR_* bits into it, the host reads and
+// clears it through pa_get_device_error(). All device code is compiled as one
+// translation unit (pa_api.cu), which is the only includer of this header.
+__device__ unsigned int g_error_word = 0;
+
+__device__ __forceinline__ void raise_error(unsigned int bits) { atomicOr(&g_error_word, bits); }
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+// About one second at B200 clocks: the bound on every wait for a bulk copy.
+constexpr long long kWaitLimitCycles = 2000000000LL;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+// Makes mbarrier initialisation visible to the async proxy (bulk copies).
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Waits for the phase with the given parity to complete; gives up after about
+// a second and returns false (the caller flags PA_DEVERR_TIMEOUT).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+  }
+  return true;
+}
+
+// L2 policy for data read exactly once per step (the KV slabs).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// One-dimensional bulk copy global -> this CTA's shared memory, completing on
+// `bar` with `bytes` of transaction count. Both addresses 16-byte aligned,
+// bytes a multiple of 16. No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// ---- 16-bit element conversions -------------------------------------------------
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<__half> {
+  __device__ __forceinline__ static float2 pair(uint32_t x) {
+    __half2 h;
+    *reinterpret_cast<uint32_t*>(&h) = x;
+    return __half22float2(h);
+  }
+  __device__ __forceinline__ static float one(uint16_t x) {
+    return __half2float(__ushort_as_half(x));
+  }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+  // bf16 is the top half of an fp32: widening is a shift / mask, exact.
+  __device__ __forceinline__ static float2 pair(uint32_t x) {
+    return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+  }
+  __device__ __forceinline__ static float one(uint16_t x) {
+    return __uint_as_float(static_cast<uint32_t>(x) << 16);
+  }
+};
+
+// DL consecutive 16-bit elements (DL in {2, 4, 8}) from shared or global memory
+// into fp32 registers, with one 4/8/16-byte load.
+template <typename T, int DL>
+__device__ __forceinline__ void load_row(const void* p, float (&f)[DL]) {
+  if constexpr (DL == 2) {
+    const uint32_t x = *reinterpret_cast<const uint32_t*>(p);
+    const float2 a = Elem<T>::pair(x);
+    f[0] = a.x;
+    f[1] = a.y;
+  } else if constexpr (DL == 4) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    const float2 a = Elem<T>::pair(x.x), b = Elem<T>::pair(x.y);
+    f[0] = a.x;
+    f[1] = a.y;
+    f[2] = b.x;
+    f[3] = b.y;
+  } else {
+    static_assert(DL == 8, "DL must be 2, 4 or 8");
+    const uint4 x = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 a = Elem<T>::pair(w[k]);
+      f[2 * k] = a.x;
+      f[2 * k + 1] = a.y;
+    }
+  }
+}
+
+// fp32 -> output element, round to nearest even.
+template <typename TO>
+__device__ __forceinline__ TO to_out(float x);
+template <>
+__device__ __forceinline__ float to_out<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ __half to_out<__half>(float x) {
+  return __float2half_rn(x);
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+}  // namespace pa

@@ -1,0 +1,104 @@
+"""The C-ABI library loads without a GPU, exports every symbol the header
+declares, and rejects bad arguments on the host before launching anything."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_driven_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(binding._SIGNATURES) >= set(names)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.pa_version() == 100
+    assert lib.pa_status_string(0) == b"PA_OK"
+    assert lib.pa_status_string(2) == b"PA_ERR_OOM"
+
+
+NULL = None
+P = ctypes.c_void_p(16 * 1024)  # an aligned address the host checks never dereference
+
+
+def decode_args(**kw):
+    a = dict(out=P, out_dt=binding.PA_F32, q=P, k=P, v=P, bt=P, MB=8, sl=P, scale=0.1, B=2, H=4,
+             D=128, S=16, NB=16, dt=binding.PA_BF16, partition=0, max_seq_len=100, ws=NULL,
+             ws_bytes=0, stream=NULL)
+    a.update(kw)
+    return [a[k] for k in ("out", "out_dt", "q", "k", "v", "bt", "MB", "sl", "scale", "B", "H", "D",
+                           "S", "NB", "dt", "partition", "max_seq_len", "ws", "ws_bytes", "stream")]
+
+
+@pytest.mark.parametrize("bad", [
+    dict(D=96), dict(D=512), dict(S=4), dict(S=64), dict(dt=binding.PA_F32), dict(out_dt=7),
+    dict(q=NULL), dict(k=NULL), dict(out=NULL), dict(bt=NULL), dict(sl=NULL),
+    dict(q=ctypes.c_void_p(16 * 1024 + 8)), dict(H=0), dict(B=-1), dict(MB=0),
+    dict(partition=24), dict(partition=-2), dict(max_seq_len=8 * 16 + 1), dict(max_seq_len=-1),
+    dict(scale=float("nan")), dict(scale=float("inf")), dict(B=70000),
+    dict(max_seq_len=100, partition=16),  # needs a workspace, none given
+])
+def test_decode_rejects_bad_arguments_on_host(lib, bad):
+    assert lib.pa_decode(*decode_args(**bad)) == binding.PA_ERR_INVALID
+
+
+def test_decode_zero_batch_is_noop(lib):
+    assert lib.pa_decode(*decode_args(B=0, q=NULL, out=NULL)) == binding.PA_OK
+
+
+def test_workspace_and_plan(lib):
+    assert binding.pa_decode_workspace_bytes(64, 40, 128, 16, 512) == 0
+    assert binding.pa_decode_plan(64, 40, 128, 16, 512) == (0, 1)
+    assert binding.pa_decode_plan(64, 40, 128, 16, 2048) == (512, 4)
+    assert binding.pa_decode_plan(64, 40, 128, 16, 2048, partition=-1) == (0, 1)
+    assert binding.pa_decode_plan(64, 40, 128, 16, 2048, partition=256) == (256, 8)
+    n = 64 * 40 * 4
+    want = ((n * 8 + 255) // 256) * 256 + n * 128 * 4
+    assert binding.pa_decode_workspace_bytes(64, 40, 128, 16, 2048) == want
+    with pytest.raises(binding.PagedAttnError):
+        binding.pa_decode_plan(1, 1, 128, 16, 100, partition=20)
+
+
+def append_args(**kw):
+    a = dict(k=P, v=P, slots=P, kc=P, vc=P, T=4, H=2, D=64, S=16, NB=8, dt=binding.PA_F16,
+             stream=NULL)
+    a.update(kw)
+    return [a[k] for k in ("k", "v", "slots", "kc", "vc", "T", "H", "D", "S", "NB", "dt", "stream")]
+
+
+@pytest.mark.parametrize("bad", [
+    dict(D=60), dict(T=-1), dict(H=0), dict(S=0), dict(dt=binding.PA_F32), dict(k=NULL),
+    dict(slots=NULL), dict(kc=ctypes.c_void_p(16 * 1024 + 2)),
+])
+def test_append_rejects_bad_arguments_on_host(lib, bad):
+    assert lib.pa_kv_append(*append_args(**bad)) == binding.PA_ERR_INVALID
+
+
+def test_append_zero_tokens_is_noop(lib):
+    assert lib.pa_kv_append(*append_args(T=0, k=NULL, v=NULL)) == binding.PA_OK
