@@ -38,6 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from paged_kv_cache_driven_b200 import binding, workloads  # noqa: E402
+from paged_kv_cache_driven_b200.batching import StagingRing  # noqa: E402
 
 H, D, S, BATCH, MAX_LEN = 40, 128, 16, 64, 2048
 DTYPE = torch.bfloat16
@@ -59,55 +60,94 @@ def append_bytes(T):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """SM clock and throttle-reason samples taken while the timed region runs.
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Polls NVML (read-only queries) from a background thread about every
+    millisecond, so even a timed region of a few milliseconds gets samples;
+    ``mark_start`` / ``mark_end`` bracket the region and only samples inside it
+    are summarised. Falls back to an nvidia-smi poll if NVML is unavailable."""
 
-    def __init__(self, device_index):
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, local_index):
+        import threading
         visible = os.environ.get("CUDA_VISIBLE_DEVICES")
         ids = [x.strip() for x in visible.split(",")] if visible else []
-        self.idx = ids[device_index] if device_index < len(ids) else str(device_index)
-        self.proc = None
+        self.dev_id = ids[local_index] if local_index < len(ids) else str(local_index)
+        self.samples = []
+        self.window = [None, None]
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self.max_mhz = None
+        self.source = None
+
+    def _handle(self, nv):
+        if self.dev_id.isdigit():
+            return nv.nvmlDeviceGetHandleByIndex(int(self.dev_id))
+        return nv.nvmlDeviceGetHandleByUUID(self.dev_id)
+
+    def _run(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.source = "nvml"
+            while not self._stop.is_set():
+                t = time.perf_counter()
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((t, float(mhz), int(reasons)))
+                time.sleep(0.001)
+            nv.nvmlShutdown()
+        except Exception:
+            self._run_smi()
+
+    def _run_smi(self):
+        q = "clocks.sm,clocks.max.sm,clocks_event_reasons.active"
+        try:
+            proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev_id}", f"--query-gpu={q}",
+                                     "--format=csv,noheader,nounits", "-lms", "100"],
+                                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+        self.source = "nvidia-smi"
+        while not self._stop.is_set():
+            line = proc.stdout.readline()
+            if not line:
+                break
+            f = [x.strip() for x in line.split(",")]
+            try:
+                self.max_mhz = float(f[1])
+                self.samples.append((time.perf_counter(), float(f[0]), int(f[2], 16)))
+            except (ValueError, IndexError):
+                continue
+        proc.terminate()
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        self._thread.start()
+        time.sleep(0.05)
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        self._stop.set()
+        self._thread.join(timeout=10)
+
+    def mark_start(self):
+        self.window[0] = time.perf_counter()
+
+    def mark_end(self):
+        self.window[1] = time.perf_counter()
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        t0, t1 = self.window
+        inside = [s for s in self.samples if t0 is not None and t1 is not None and t0 <= s[0] <= t1]
+        reasons = sorted({n for _, _, r in inside for n, bit in self.REASONS if r & bit})
+        mhz = [m for _, m, _ in inside]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz), "source": self.source}
 
 
 def measured_peak():
@@ -178,13 +218,16 @@ class Workload:
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
         self.plan = binding.pa_decode_plan(BATCH, H, D, S, self.max_seq, 0)
         self.scale = 1.0 / math.sqrt(D)
-        # pinned host buffers of the end-to-end step
+        self.e2e_ready = False
+
+    def prepare_e2e(self):
+        """Pinned host buffers and device landing buffers of the end-to-end step."""
+        device = self.device
+        self.e2e_ready = True
         self.h_q = self.q.cpu().pin_memory()
         self.h_k = self.k_new.cpu().pin_memory()
         self.h_v = self.v_new.cpu().pin_memory()
-        self.h_slots = torch.empty(BATCH, dtype=torch.int64).pin_memory()
-        self.h_tables = torch.empty((BATCH, self.MB), dtype=torch.int32).pin_memory()
-        self.h_lens = torch.empty(BATCH, dtype=torch.int32).pin_memory()
+        self.staging = StagingRing(BATCH, self.MB)
         self.h_out = torch.empty((BATCH, H, D), dtype=DTYPE).pin_memory()
         self.d_q = torch.empty_like(self.q)
         self.d_k = torch.empty_like(self.k_new)
@@ -208,20 +251,23 @@ class Workload:
     def e2e_step(self):
         """One decode step through the public API from host memory. Returns the
         sequence lengths it decoded."""
-        self.alloc.pa_prepare_step(self.seq_ids, 1, self.MB, self.h_slots, self.h_tables,
-                                   self.h_lens)
+        if not self.e2e_ready:
+            self.prepare_e2e()
+        h = self.staging.acquire()
+        self.alloc.pa_prepare_step(self.seq_ids, 1, self.MB, h["slots"], h["tables"], h["lens"])
         self.d_q.copy_(self.h_q, non_blocking=True)
         self.d_k.copy_(self.h_k, non_blocking=True)
         self.d_v.copy_(self.h_v, non_blocking=True)
-        self.d_slots.copy_(self.h_slots, non_blocking=True)
-        self.d_tables.copy_(self.h_tables, non_blocking=True)
-        self.d_lens.copy_(self.h_lens, non_blocking=True)
+        self.d_slots.copy_(h["slots"], non_blocking=True)
+        self.d_tables.copy_(h["tables"], non_blocking=True)
+        self.d_lens.copy_(h["lens"], non_blocking=True)
+        self.staging.release()
+        lens = h["lens"].tolist()
         binding.pa_kv_append(self.d_k, self.d_v, self.d_slots, self.k_cache, self.v_cache)
         binding.pa_decode(self.out, self.d_q, self.k_cache, self.v_cache, self.d_tables,
-                          self.d_lens, self.scale, int(self.h_lens.max()), partition=0,
-                          workspace=self.ws)
+                          self.d_lens, self.scale, max(lens), partition=0, workspace=self.ws)
         self.h_out.copy_(self.out, non_blocking=True)
-        return self.h_lens.tolist()
+        return lens
 
     def h2d_bytes(self):
         return (3 * BATCH * H * D * ELEM + 8 * BATCH + 4 * BATCH * self.MB + 4 * BATCH)
@@ -265,14 +311,33 @@ def sum_over_ranks(x, world, device):
     return float(t.item())
 
 
-def cpu_oracle_sample(wl, target_seconds, cores):
-    """Times the fp64 CPU oracle on a bounded sample of this workload's
-    (request, head) pairs; returns (GB/s of KV, description)."""
-    from oracle import decode as oracle_decode  # test infrastructure: the CPU baseline leg only
+class CpuOracleSample:
+    """A bounded sample of this workload's (request, head) pairs for the fp64 CPU
+    oracle, sized so that one pass takes about ``pass_seconds`` (or the whole
+    workload, if that is quicker)."""
 
-    tables = wl.tables_d.cpu()
+    def __init__(self, wl, pass_seconds, cores):
+        from oracle import decode as oracle_decode  # test infrastructure: CPU-baseline legs only
 
-    def sub_problem(pairs):
+        self._decode = oracle_decode.paged_decode
+        self.wl, self.cores = wl, cores
+        g = torch.Generator().manual_seed(123)
+        all_pairs = [(i, h) for i in range(BATCH) for h in range(H)]
+        perm = torch.randperm(len(all_pairs), generator=g).tolist()
+        n = min(len(all_pairs), 2 * cores)
+        while True:
+            self.pairs = [all_pairs[k] for k in perm[:n]]
+            self.prob = self._sub_problem(self.pairs)
+            dt = self.run()
+            if dt >= pass_seconds * 0.5 or n >= len(all_pairs):
+                break
+            n = min(len(all_pairs), max(2 * n, int(n * pass_seconds / max(dt, 1e-3))))
+        self.tokens = sum(wl.lens[i] for i, _ in self.pairs)
+        self.nbytes = sum(2 * wl.lens[i] * D * ELEM for i, _ in self.pairs)
+
+    def _sub_problem(self, pairs):
+        wl = self.wl
+        tables = wl.tables_d.cpu()
         ks, vs, qs, rows, lens = [], [], [], [], []
         off = 0
         for i, h in pairs:
@@ -291,48 +356,48 @@ def cpu_oracle_sample(wl, target_seconds, cores):
         return (torch.cat(qs), torch.cat(ks), torch.cat(vs), bt,
                 torch.tensor(lens, dtype=torch.int32))
 
-    g = torch.Generator().manual_seed(123)
-    all_pairs = [(i, h) for i in range(BATCH) for h in range(H)]
-    perm = torch.randperm(len(all_pairs), generator=g).tolist()
-    # calibrate on a few pairs, then size the sample for ~target_seconds
-    n = 2 * cores
-    while True:
-        pairs = [all_pairs[k] for k in perm[:n]]
-        prob = sub_problem(pairs)
+    def run(self):
         t0 = time.perf_counter()
-        oracle_decode.paged_decode(*prob, wl.scale, threads=cores)
-        dt = time.perf_counter() - t0
-        if dt >= target_seconds * 0.5 or n >= len(all_pairs):
-            break
-        n = min(len(all_pairs), max(n * 2, int(n * target_seconds / max(dt, 1e-3))))
-    nbytes = sum(2 * wl.lens[i] * D * ELEM for i, _ in pairs)
-    desc = (f"{len(pairs)} of {BATCH * H} (request, head) pairs of the workload, "
-            f"{sum(wl.lens[i] for i, _ in pairs)} tokens, {dt:.1f} s on {cores} threads")
-    return nbytes / dt / 1e9, desc, dt
+        self._decode(*self.prob, self.wl.scale, threads=self.cores)
+        return time.perf_counter() - t0
+
+    def describe(self, passes, seconds):
+        return (f"{len(self.pairs)} of {BATCH * H} (request, head) pairs of the workload "
+                f"({self.tokens} tokens) x {passes} passes, {seconds:.1f} s on {self.cores} threads")
+
+
+def cpu_baseline(wl, target_seconds, cores):
+    """The oracle as it stands, timed on this host: (GB/s of KV, description)."""
+    smp = CpuOracleSample(wl, min(target_seconds, 10.0), cores)
+    passes, total = 0, 0.0
+    while total < target_seconds * 0.7 or passes == 0:
+        total += smp.run()
+        passes += 1
+    return passes * smp.nbytes / total / 1e9, smp.describe(passes, total)
 
 
 def run_reference(args):
-    """The reference arm: the fp64 CPU oracle on the host cores, rank 0 only."""
+    """The reference arm: the fp64 CPU oracle on the host cores, rank 0 only. Each
+    step is one pass over a bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     device = "cuda" if torch.cuda.is_available() else "cpu"
-    wl = Workload(seed=0, device=device, extra_tokens=0)
+    wl = Workload(seed=args.seed, device=device, extra_tokens=0)
     cores = os.cpu_count() or 1
-    vals = []
+    per_step = min(5.0, max(0.05, 150.0 / (args.steps + args.warmup)))
+    smp = CpuOracleSample(wl, per_step, cores)
     for _ in range(args.warmup):
-        cpu_oracle_sample(wl, 1.0, cores)
-    desc = ""
-    for _ in range(args.steps):
-        v, desc, _ = cpu_oracle_sample(wl, 5.0, cores)
-        vals.append(v)
-    value = statistics.mean(vals)
+        smp.run()
+    total = sum(smp.run() for _ in range(args.steps))
+    value = args.steps * smp.nbytes / total / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": WORKLOAD, "l2": "inputs larger than L2"},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
-                             "kind": "oracle", "sample": desc},
+                             "kind": "oracle", "sample": smp.describe(args.steps, total)},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -341,7 +406,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
@@ -371,12 +436,14 @@ def main():
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
-    with ClockSampler(device.index if device.index is not None else 0) as clk:
+    with ClockSampler(local) as clk:
+        clk.mark_start()
         start.record(stream)
         for k in range(args.steps):
             wl.device_step(dec_events[k])
         end.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
     barrier(world)
     torch.cuda.synchronize()
     ms_total = max_over_ranks(start.elapsed_time(end), world, device)
@@ -416,7 +483,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
-        v, desc, _ = cpu_oracle_sample(wl, 15.0, cores)
+        v, desc = cpu_baseline(wl, 12.0, cores)
         cpu = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": desc}
 

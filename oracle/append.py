@@ -17,6 +17,19 @@ def _bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
+def scatter_into(k_bits, v_bits, slots, kc_bits, vc_bits):
+    """In-place form on uint16 bit arrays: k_bits, v_bits [T, H, D]; caches [NB, H, S, D]."""
+    slots = np.asarray(slots, dtype=np.int64)
+    S = kc_bits.shape[2]
+    for t in range(slots.shape[0]):
+        s = int(slots[t])
+        if s < 0:
+            continue
+        block, offset = divmod(s, S)
+        kc_bits[block, :, offset, :] = k_bits[t]
+        vc_bits[block, :, offset, :] = v_bits[t]
+
+
 def kv_append(k, v, slot_mapping, k_cache, v_cache):
     """Returns (k_cache', v_cache') as uint16 bit arrays after the scatter.
 
@@ -26,14 +39,6 @@ def kv_append(k, v, slot_mapping, k_cache, v_cache):
     keep their values.
     """
     kc, vc = _bits(k_cache).copy(), _bits(v_cache).copy()
-    kb, vb = _bits(k), _bits(v)
     slots = np.asarray(torch.as_tensor(slot_mapping).to("cpu").numpy(), dtype=np.int64)
-    S = kc.shape[2]
-    for t in range(slots.shape[0]):
-        s = int(slots[t])
-        if s < 0:
-            continue
-        block, offset = divmod(s, S)
-        kc[block, :, offset, :] = kb[t]
-        vc[block, :, offset, :] = vb[t]
+    scatter_into(_bits(k), _bits(v), slots, kc, vc)
     return kc, vc

@@ -45,8 +45,11 @@ def _load():
     return _lib
 
 
-def _bits(t: torch.Tensor) -> np.ndarray:
-    """The raw 16-bit patterns of a CPU fp16/bf16 tensor, as a contiguous uint16 array."""
+def _bits(t) -> np.ndarray:
+    """The raw 16-bit patterns of an fp16/bf16 tensor (or a uint16 array of them),
+    as a contiguous uint16 array."""
+    if isinstance(t, np.ndarray):
+        return np.ascontiguousarray(t, dtype=np.uint16)
     t = t.detach().to("cpu").contiguous()
     return t.view(torch.int16).numpy().view(np.uint16)
 
@@ -68,20 +71,24 @@ def decode16(bits: int, dtype: torch.dtype) -> float:
     return _load().oracle_decode16(bits, _DTYPE_CODE[dtype])
 
 
-def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs=None, threads=0):
+def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs=None, threads=0,
+                 dtype=None):
     """fp64 attention output.
 
     q [B, H, D]; k_cache, v_cache [NB, H, S, D] (fp16 or bf16, same dtype as q);
     block_tables [B, MB] int32; seq_lens [B] int32. ``pairs`` is an optional
     sequence of (request, head) pairs; the result is then [len(pairs), D],
-    otherwise [B, H, D]. ``threads`` = 0 uses every host core.
+    otherwise [B, H, D]. ``threads`` = 0 uses every host core. The 16-bit inputs
+    may also be uint16 numpy arrays of bit patterns, with ``dtype`` naming them.
     """
     B, H, D = q.shape
     NB, H2, S, D2 = k_cache.shape
     if (H2, D2) != (H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise OracleError("shape mismatch")
-    if q.dtype != k_cache.dtype or q.dtype != v_cache.dtype:
-        raise OracleError("dtype mismatch")
+    if dtype is None:
+        if q.dtype != k_cache.dtype or q.dtype != v_cache.dtype:
+            raise OracleError("dtype mismatch")
+        dtype = q.dtype
     qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
     bt = _i32(block_tables).reshape(B, -1)
     sl = _i32(seq_lens).reshape(B)
@@ -93,7 +100,7 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs=None,
         n, out = pa.shape[0], np.zeros((pa.shape[0], D), np.float64)
     rc = _load().oracle_paged_decode(
         _ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), _ptr(sl), B, H, D, S, NB, MB, float(scale),
-        _DTYPE_CODE[q.dtype], None if pa is None else _ptr(pa), n, int(threads), _ptr(out))
+        _DTYPE_CODE[dtype], None if pa is None else _ptr(pa), n, int(threads), _ptr(out))
     if rc:
         raise OracleError(f"oracle_paged_decode returned {rc}")
     return out

@@ -1,0 +1,127 @@
+"""Continuous-batching decode loop over the paged KV cache.
+
+"vLLM KV Cache and PagedAttention Explained", Step 8 "Continuous Batching in
+vLLM": as soon as a request finishes, its batch slot is refilled with a new
+request, and because each request's KV lives in its own physical blocks only
+the finished request's blocks are freed and handed on (Step 7 item 7). Each
+step is the decode loop of 7단계 "전체 흐름 요약": the new token's K/V is appended
+to the cache, then attention reads the cached K/V.
+
+One step, in this order (the order is part of the contract the tests check):
+  1. host: every active request grows by one token (pa_prepare_step: new blocks
+     at block boundaries, the new tokens' slots, padded block tables, lengths);
+  2. host -> device copies of slots, tables and lengths;
+  3. pa_kv_append of the step's new K/V, then pa_decode over every request's
+     cached tokens including the new one;
+  4. host: each request's token budget drops by one; for batch slots in index
+     order, a finished request is freed (pa_seq_free) and its slot immediately
+     refilled by the next arrival: grow to its prompt length and append its
+     prompt K/V through slot_mapping (the prefill write of Step 6 "Prefill").
+
+Random draws (lengths, budgets, token values, the shuffled free list) come from
+``workloads.BatchingLoop``; everything else runs in the library.
+"""
+
+import math
+
+import torch
+
+from . import binding
+
+
+class StagingRing:
+    """Pinned host buffers for each step's slots, block tables and lengths, ``depth``
+    sets deep. The host fills set k while the copies of earlier sets may still be
+    in flight; before a set is refilled, the event recorded after its copies is
+    waited on, so the host never rewrites memory a pending copy still reads."""
+
+    def __init__(self, n_seq, max_blocks, n_new=1, depth=2):
+        self.sets = [dict(slots=torch.empty(n_seq * n_new, dtype=torch.int64).pin_memory(),
+                          tables=torch.empty((n_seq, max_blocks), dtype=torch.int32).pin_memory(),
+                          lens=torch.empty(n_seq, dtype=torch.int32).pin_memory())
+                     for _ in range(depth)]
+        self.events = [None] * depth
+        self.k = 0
+
+    def acquire(self):
+        i = self.k % len(self.sets)
+        if self.events[i] is not None:
+            self.events[i].synchronize()
+        return self.sets[i]
+
+    def release(self, stream=None):
+        ev = torch.cuda.Event()
+        ev.record(stream if stream is not None else torch.cuda.current_stream())
+        self.events[self.k % len(self.sets)] = ev
+        self.k += 1
+
+
+class ContinuousBatching:
+    def __init__(self, loop, device, max_steps=64, poison=True):
+        self.loop = loop
+        self.device = device
+        B, H, D, S = loop.batch, loop.H, loop.D, loop.S
+        self.B, self.H, self.D, self.S = B, H, D, S
+        self.max_len = 4096 + max_steps
+        self.MB = -(-self.max_len // S)
+        NB = loop.num_blocks
+        fill = float("nan") if poison else 0.0
+        self.k_cache = torch.full((NB, H, S, D), fill, dtype=loop.dtype, device=device)
+        self.v_cache = torch.full((NB, H, S, D), fill, dtype=loop.dtype, device=device)
+        self.alloc = binding.BlockAllocator(NB, S, initial_order=loop.block_order)
+        self.scale = 1.0 / math.sqrt(D)
+        self.serial = 0
+        self.slots = []  # per batch slot: [seq_id, remaining budget]
+        self.staging = StagingRing(B, self.MB)
+        self.d_slots = torch.empty(B, dtype=torch.int64, device=device)
+        self.d_tables = torch.empty((B, self.MB), dtype=torch.int32, device=device)
+        self.d_lens = torch.empty(B, dtype=torch.int32, device=device)
+        self.out = torch.empty((B, H, D), dtype=torch.float32, device=device)
+        ws = binding.pa_decode_workspace_bytes(B, H, D, S, self.max_len, 0)
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        self.events = []  # (kind, seq_id, serial, prompt_len) for admissions / retirements
+        for b in range(B):
+            self.slots.append(self._admit(loop.initial_lens[b], loop.budgets[b]))
+
+    def _admit(self, prompt_len, budget):
+        """Creates a request, allocates its prompt blocks and appends its prompt K/V."""
+        sid = self.serial
+        self.serial += 1
+        self.alloc.pa_seq_grow(sid, prompt_len)
+        k, v = self.loop.prompt_kv(sid, prompt_len, self.device)
+        slots = self.alloc.pa_build_slot_mapping([sid], [0], [prompt_len]).to(self.device)
+        binding.pa_kv_append(k, v, slots, self.k_cache, self.v_cache)
+        self.events.append(("admit", sid, prompt_len))
+        return [sid, max(1, int(budget))]
+
+    def seq_ids(self):
+        return [s[0] for s in self.slots]
+
+    def step(self, step_idx):
+        """One decode step; returns a record of what it did (for checking)."""
+        ids = self.seq_ids()
+        h = self.staging.acquire()
+        self.alloc.pa_prepare_step(ids, 1, self.MB, h["slots"], h["tables"], h["lens"])
+        self.d_slots.copy_(h["slots"], non_blocking=True)
+        self.d_tables.copy_(h["tables"], non_blocking=True)
+        self.d_lens.copy_(h["lens"], non_blocking=True)
+        self.staging.release()
+        q, k, v = self.loop.token_kv(step_idx, self.B, self.device)
+        binding.pa_kv_append(k, v, self.d_slots, self.k_cache, self.v_cache)
+        max_len = int(h["lens"].max())
+        binding.pa_decode(self.out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
+                          self.scale, max_len, partition=0, workspace=self.ws)
+        record = dict(ids=ids, slots=h["slots"].clone(), lens=h["lens"].clone(),
+                      tables=h["tables"].clone(), q=q, k=k, v=v, out=self.out, retired=[],
+                      admitted=[])
+        for b in range(self.B):
+            self.slots[b][1] -= 1
+            if self.slots[b][1] <= 0:
+                old = self.slots[b][0]
+                self.alloc.pa_seq_free(old)
+                self.events.append(("retire", old, 0))
+                L, budget = self.loop.arrival()
+                self.slots[b] = self._admit(L, budget)
+                record["retired"].append(old)
+                record["admitted"].append((self.slots[b][0], L, self.slots[b][1]))
+        return record
