@@ -127,6 +127,34 @@ pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cac
  * Only partitions p < ceil(seq_lens[i] / partition) of requests with more than
  * one partition are written. */
 
+/* ---------------------------------------------------------------------------
+ * Decode without any caller-provided scratch. This entry point has no
+ * counterpart on the pages: it exists for callers that cannot allocate device
+ * memory themselves, such as a plugin whose host framework owns every device
+ * allocation and offers it no allocator, or a serving process that fixes its
+ * device-memory budget at start-up and must not call cudaMalloc afterwards
+ * (an allocation at run time can synchronise the device and stall other
+ * streams). It behaves exactly like pa_decode, with the same arguments minus
+ * the workspace: the split-KV partials go to a static device array of
+ * PA_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads it,
+ * until the process exits. The call allocates nothing.
+ *   - The first call on a device looks up that array's device address
+ *     (cudaGetSymbolAddress) with the device current; make that first call
+ *     before any stream capture on the device.
+ *   - A call whose split needs more scratch than the array holds (see
+ *     pa_decode_workspace_bytes) returns PA_ERR_OOM and launches nothing.
+ *   - Every call shares the one array and leaves its partials there; nothing
+ *     in it needs to start at zero (each call writes every partial it reads).
+ *     Calls whose work overlaps on the GPU (other streams, other threads)
+ *     race on the array: order them on one stream or serialise them.
+ * ------------------------------------------------------------------------- */
+#define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+pa_status pa_decode_noalloc(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables, int MB,
+                            const int32_t* seq_lens, float scale, int B, int H, int D, int S,
+                            int NB, pa_dtype dt, int partition, int max_seq_len, void* stream);
+
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`. *flags receives PA_DEVERR_* bits (0 = clean).
  * Returns PA_OK, or PA_ERR_CUDA if the read failed. */

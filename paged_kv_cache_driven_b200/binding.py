@@ -32,6 +32,8 @@ _SIGNATURES = {
     "pa_decode": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32, _i32,
                    _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_get_device_error": ([_vp, _vp], _i32),
+    "pa_decode_noalloc": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32,
+                           _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "pa_alloc_create": ([_i32, _i32, _vp, _vp], _i32),
     "pa_alloc_destroy": ([_vp], None),
     "pa_seq_grow": ([_vp, _i64, _i32], _i32),
@@ -146,6 +148,28 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_l
                            _ptr(block_tables), MB, _ptr(seq_lens), float(scale), B, H, D, S, NB,
                            _DT[q.dtype], int(partition), int(max_seq_len), _ptr(workspace),
                            ws_bytes, _stream(stream)), "pa_decode")
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,
+                      partition=0, stream=None):
+    """pa_decode without a workspace argument: for callers that cannot allocate
+    device memory. The split-KV partials go to the library's static device array
+    (PA_NOALLOC_SCRATCH_BYTES); a split that needs more raises PA_ERR_OOM."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                 ("block_tables", block_tables), ("seq_lens", seq_lens)):
+        _cuda(t, n)
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    B, H, D = q.shape
+    NB, _, S, _ = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    _check(lib().pa_decode_noalloc(_ptr(out), _DT[out.dtype], _ptr(q), _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(block_tables), MB, _ptr(seq_lens),
+                                   float(scale), B, H, D, S, NB, _DT[q.dtype], int(partition),
+                                   int(max_seq_len), _stream(stream)), "pa_decode_noalloc")
+
+
+PA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def pa_get_device_error(stream=None):

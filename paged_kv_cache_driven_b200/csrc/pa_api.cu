@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -239,3 +240,43 @@ pa_status pa_get_device_error(void* stream, uint32_t* flags) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// pa_decode_noalloc: decode whose split-KV partials live in a static device
+// array instead of a caller-provided workspace, for callers that cannot
+// allocate device memory (see pagedattn.h). It reuses pa_decode unchanged.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch per device, looked up on the first call
+// made with that device current. The host-side name of the array is only a
+// stand-in for the symbol, never a usable device address.
+std::atomic<void*> g_noalloc_scratch_addr[kMaxDevices];
+
+}  // namespace
+
+extern "C" pa_status pa_decode_noalloc(void* out, pa_dtype out_dt, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, int MB,
+                                       const int32_t* seq_lens, float scale, int B, int H, int D,
+                                       int S, int NB, pa_dtype dt, int partition, int max_seq_len,
+                                       void* stream) {
+  int P, NP;
+  if (B < 0 || H <= 0 || !decode_shape_ok(D, S) || !plan(S, max_seq_len, partition, &P, &NP))
+    return PA_ERR_INVALID;
+  const size_t need = workspace_for(B, H, D, NP);
+  if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_OOM;  // larger than the static array
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  void* scratch = g_noalloc_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!scratch) {
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch)
+      return PA_ERR_CUDA;
+    g_noalloc_scratch_addr[dev].store(scratch, std::memory_order_release);
+  }
+  return pa_decode(out, out_dt, q, k_cache, v_cache, block_tables, MB, seq_lens, scale, B, H, D, S,
+                   NB, dt, partition, max_seq_len, scratch, PA_NOALLOC_SCRATCH_BYTES, stream);
+}
