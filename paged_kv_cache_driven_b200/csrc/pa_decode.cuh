@@ -2,10 +2,11 @@
 // log-sum-exp reduce.
 //
 // What it computes: "vLLM KV Cache and PagedAttention Explained", "Appendix:
-// The Attention Score Formula" -- out = softmax(q K^T * scale) V, carried out by
-// walking the block table, fetching each block's keys, computing partial
-// scores, updating a running softmax normaliser, weighting the values and
-// accumulating, one block at a time. The blocks are read where they are
+// The Attention Score Formula" -- out = softmax(q K^T * scale) V. The paged form
+// described there visits the request's physical blocks in table order; for
+// each block it scores the block's keys against the query, rescales the
+// running max and sum, and adds the block's weighted values into the
+// accumulator. The blocks are read where they are
 // ("PagedAttention" card, "Kernel은 무엇이 달라지는가"); long contexts are cut into
 // partitions whose partial results a second kernel merges (FlashDecoding, the
 // same card, "헷갈리기 쉬운 구분").

@@ -58,7 +58,7 @@ def test_worked_example_identity_order_matches_5단계():
     """5단계: request A gets block 0 and request B starts at blocks 1, 2, 3.
 
     The page lists only three blocks for B's 50 tokens, against its own 6단계
-    ("4블록") and ceil(50/16) = 4; the model gives B a fourth block.
+    (four blocks) and ceil(50/16) = 4; the model gives B a fourth block.
     """
     pool = BlockPoolModel(64, 16)
     pool.grow("A", 6)
@@ -156,7 +156,7 @@ def test_page_request_b_blocks():
 
 
 def test_free_then_reuse_lifo():
-    """Step 7 item 7: a freed block is immediately available to the next request."""
+    """Step 7 item 7: a released block can be handed to the very next request."""
     pool = BlockPoolModel(16, 16)
     pool.grow("a", 40)  # blocks 0, 1, 2
     pool.grow("b", 5)   # block 3
