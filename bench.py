@@ -38,7 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from paged_kv_cache_driven_b200 import binding, workloads  # noqa: E402
-from paged_kv_cache_driven_b200.batching import StagingRing  # noqa: E402
+from paged_kv_cache_driven_b200.pipeline import HostFedDecoder  # noqa: E402
 
 H, D, S, BATCH, MAX_LEN = 40, 128, 16, 64, 2048
 DTYPE = torch.bfloat16
@@ -55,8 +55,10 @@ def decode_bytes(lens):
     return kv + sum(4 * (-(-L // S)) for L in lens) + 4 * len(lens)
 
 
-def append_bytes(T):
-    return T * H * D * ELEM * 4 + 8 * T
+def append_bytes(T, slots=True):
+    """New tokens' K and V read and written; plus the int64 slots when the
+    append goes through slot_mapping (the fused step derives them on device)."""
+    return T * H * D * ELEM * 4 + (8 * T if slots else 0)
 
 
 class ClockSampler:
@@ -159,10 +161,15 @@ def measured_peak():
 
 
 def kernel_source_hash():
+    """Hash of the decode kernels' source with comments and blank lines removed,
+    so a profile stays attached to the code it measured and nothing else."""
+    import re
     h = hashlib.sha256()
     for f in ("pa_decode.cuh", "pa_device.cuh", "pa_api.cu"):
-        with open(os.path.join(ROOT, "paged_kv_cache_driven_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "paged_kv_cache_driven_b200", "csrc", f)) as fh:
+            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        lines = [re.sub(r"//.*", "", l).rstrip() for l in text.splitlines()]
+        h.update("\n".join(l for l in lines if l.strip()).encode())
     return h.hexdigest()[:16]
 
 
@@ -221,59 +228,51 @@ class Workload:
         self.e2e_ready = False
 
     def prepare_e2e(self):
-        """Pinned host buffers and device landing buffers of the end-to-end step."""
-        device = self.device
+        """Pinned host inputs and the host-fed step pipeline of the end-to-end step."""
         self.e2e_ready = True
-        self.h_q = self.q.cpu().pin_memory()
-        self.h_k = self.k_new.cpu().pin_memory()
-        self.h_v = self.v_new.cpu().pin_memory()
-        self.staging = StagingRing(BATCH, self.MB)
-        self.h_out = torch.empty((BATCH, H, D), dtype=DTYPE).pin_memory()
-        self.d_q = torch.empty_like(self.q)
-        self.d_k = torch.empty_like(self.k_new)
-        self.d_v = torch.empty_like(self.v_new)
-        self.d_slots = torch.empty(BATCH, dtype=torch.int64, device=device)
-        self.d_tables = torch.empty((BATCH, self.MB), dtype=torch.int32, device=device)
-        self.d_lens = torch.empty(BATCH, dtype=torch.int32, device=device)
+        self.h_qkv = torch.stack([self.q, self.k_new, self.v_new]).cpu().pin_memory()
+        self.fed = HostFedDecoder(self.alloc, self.k_cache, self.v_cache, BATCH, self.MB,
+                                  self.max_len, out_dtype=DTYPE, fused=True)
 
-    def launches_per_step(self):
-        return 2 + (1 if self.plan[1] > 1 else 0)
+    def launches_per_step(self, fused=True):
+        return (1 if fused else 2) + (1 if self.plan[1] > 1 else 0)
 
-    def device_step(self, ev_decode=None):
-        binding.pa_kv_append(self.k_new, self.v_new, self.slots_d, self.k_cache, self.v_cache)
+    def device_step(self, ev_decode=None, fused=True):
+        """One step on device-resident inputs. Fused: pa_decode_append (the new
+        tokens' K/V written at their last positions inside the decode launch);
+        unfused: pa_kv_append through slot_mapping, then pa_decode."""
+        if not fused:
+            binding.pa_kv_append(self.k_new, self.v_new, self.slots_d, self.k_cache, self.v_cache)
         if ev_decode is not None:
             ev_decode[0].record()
-        binding.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.tables_d, self.lens_d,
-                          self.scale, self.max_seq, partition=0, workspace=self.ws)
+        if fused:
+            binding.pa_decode_append(self.out, self.q, self.k_new, self.v_new, self.k_cache,
+                                     self.v_cache, self.tables_d, self.lens_d, self.scale,
+                                     self.max_seq, partition=0, workspace=self.ws)
+        else:
+            binding.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.tables_d,
+                              self.lens_d, self.scale, self.max_seq, partition=0,
+                              workspace=self.ws)
         if ev_decode is not None:
             ev_decode[1].record()
 
     def e2e_step(self):
-        """One decode step through the public API from host memory. Returns the
-        sequence lengths it decoded."""
+        """One decode step through the public API from host memory: the host
+        allocator grows every request by one token, q/k/v, tables and lengths are
+        copied from pinned host memory, the decode (with the append) runs, the
+        output is copied back."""
         if not self.e2e_ready:
             self.prepare_e2e()
-        h = self.staging.acquire()
-        self.alloc.pa_prepare_step(self.seq_ids, 1, self.MB, h["slots"], h["tables"], h["lens"])
-        self.d_q.copy_(self.h_q, non_blocking=True)
-        self.d_k.copy_(self.h_k, non_blocking=True)
-        self.d_v.copy_(self.h_v, non_blocking=True)
-        self.d_slots.copy_(h["slots"], non_blocking=True)
-        self.d_tables.copy_(h["tables"], non_blocking=True)
-        self.d_lens.copy_(h["lens"], non_blocking=True)
-        self.staging.release()
-        lens = h["lens"].tolist()
-        binding.pa_kv_append(self.d_k, self.d_v, self.d_slots, self.k_cache, self.v_cache)
-        binding.pa_decode(self.out, self.d_q, self.k_cache, self.v_cache, self.d_tables,
-                          self.d_lens, self.scale, max(lens), partition=0, workspace=self.ws)
-        self.h_out.copy_(self.out, non_blocking=True)
-        return lens
+        self.fed.step(self.seq_ids, self.h_qkv)
+
+    def e2e_drain(self):
+        self.fed.drain()
 
     def h2d_bytes(self):
-        return (3 * BATCH * H * D * ELEM + 8 * BATCH + 4 * BATCH * self.MB + 4 * BATCH)
+        return self.fed.h2d_bytes()
 
     def d2h_bytes(self):
-        return BATCH * H * D * ELEM
+        return self.fed.d2h_bytes()
 
 
 def dist_setup(n_gpus):
@@ -428,34 +427,49 @@ def main():
     stream = torch.cuda.current_stream()
 
     # ---- device-resident steps -------------------------------------------------
-    for _ in range(args.warmup):
-        wl.device_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
-        clk.mark_start()
+    def timed_steps(fused, sampler=None):
+        for _ in range(args.warmup):
+            wl.device_step(fused=fused)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        calls = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        if sampler is not None:
+            sampler.mark_start()
         start.record(stream)
         for k in range(args.steps):
-            wl.device_step(dec_events[k])
+            wl.device_step(calls[k], fused=fused)
         end.record(stream)
         torch.cuda.synchronize()
-        clk.mark_end()
-    barrier(world)
-    torch.cuda.synchronize()
-    ms_total = max_over_ranks(start.elapsed_time(end), world, device)
-    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_events)
-    flags = binding.pa_get_device_error()
-    if flags:
-        raise SystemExit(f"device error word set: {flags:#x}")
-    step_bytes = decode_bytes(wl.lens) + append_bytes(BATCH)
+        if sampler is not None:
+            sampler.mark_end()
+        barrier(world)
+        torch.cuda.synchronize()
+        total = max_over_ranks(start.elapsed_time(end), world, device)
+        call_ms = statistics.mean(a.elapsed_time(b) for a, b in calls)
+        flags = binding.pa_get_device_error()
+        if flags:
+            raise SystemExit(f"device error word set: {flags:#x}")
+        return total, call_ms
+
+    # the two-call step (pa_kv_append through slot_mapping, then pa_decode), for reference
+    unfused_ms, unfused_dec_ms = timed_steps(fused=False)
+    # the fused step, timed for the headline with clocks sampled inside the region
+    with ClockSampler(local) as clk:
+        ms_total, dec_ms = timed_steps(fused=True, sampler=clk)
+    step_bytes = decode_bytes(wl.lens) + append_bytes(BATCH, slots=False)
     total_bytes = sum_over_ranks(step_bytes * args.steps, world, device)
     value = total_bytes / (ms_total / 1e3) / 1e9
     ms_per_step = ms_total / args.steps
-    dec_gbs = decode_bytes(wl.lens) / (dec_ms / 1e3) / 1e9
+    dec_gbs = step_bytes / (dec_ms / 1e3) / 1e9
+    unfused_bytes = decode_bytes(wl.lens) + append_bytes(BATCH)
+    unfused = {"ms_per_step": round(unfused_ms / args.steps, 4),
+               "gb_s": round(sum_over_ranks(unfused_bytes * args.steps, world, device)
+                             / (unfused_ms / 1e3) / 1e9, 2),
+               "pa_decode_ms": round(unfused_dec_ms, 4),
+               "pa_decode_gb_s": round(decode_bytes(wl.lens) / (unfused_dec_ms / 1e3) / 1e9, 2)}
     peak, peak_kind = measured_peak()
 
     # ---- end-to-end steps through the C ABI from host buffers ------------------
@@ -465,13 +479,17 @@ def main():
     barrier(world)
     torch.cuda.synchronize()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_bytes = 0
     e_start.record(stream)
     for _ in range(args.steps):
-        lens = wl.e2e_step()
-        e2e_bytes += decode_bytes(lens) + append_bytes(BATCH)
+        wl.e2e_step()
+    wl.e2e_drain()  # the last result copies are inside the timed region
     e_end.record(stream)
     torch.cuda.synchronize()
+    # every e2e step grew each request by one token: timed step j decoded L + W + j + 1
+    e2e_bytes = sum(decode_bytes([L + args.warmup + j + 1 for L in wl.lens])
+                    + append_bytes(BATCH, slots=False) for j in range(args.steps))
+    assert [wl.alloc.pa_seq_len(i) for i in wl.seq_ids] == \
+        [L + args.warmup + args.steps for L in wl.lens]
     barrier(world)
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device)
     e2e_total = sum_over_ranks(e2e_bytes, world, device)
@@ -500,17 +518,19 @@ def main():
                        "l2": "inputs larger than L2 (1.3 GB of KV per step vs 126 MB L2)",
                        "parallelism": f"dp{world} (independent batches, no collective)"},
             "decode_tok_s_layer": round(tok_s_layer, 1),
-            "decode_only": {"ms": round(dec_ms, 4), "gb_s": round(dec_gbs, 2),
-                            "tok_s_layer": round(BATCH / (dec_ms / 1e3), 1)},
+            "step": "pa_decode_append: the 64 new tokens' K/V appended inside the decode launch",
+            "unfused_step": unfused,
             "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(dec_gbs / peak, 4),
                          "peak_kind": peak_kind, "traffic": profiled_traffic(),
-                         "kernel": "pa_decode (paged_decode_partition_kernel + splitkv_reduce_kernel)",
-                         "algorithmic_bytes_per_launch": decode_bytes(wl.lens)},
+                         "kernel": "pa_decode_append call: paged_decode_partition_kernel<APPEND> "
+                                   "+ splitkv_reduce_kernel",
+                         "call_ms": round(dec_ms, 4),
+                         "algorithmic_bytes_per_launch": step_bytes},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": wl.h2d_bytes(), "d2h_bytes_per_step": wl.d2h_bytes(),
                     "ms_per_step": round(e2e_ms / args.steps, 4)},
-            "gpu_launches": wl.launches_per_step() * args.steps,
+            "gpu_launches": wl.launches_per_step(fused=True) * args.steps,
             "clocks": clk.summary(),
         }
         if cpu is not None:

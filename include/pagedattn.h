@@ -119,6 +119,25 @@ pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cac
                     pa_dtype dt, int partition, int max_seq_len, void* workspace,
                     size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * One decode step in one launch: append, then attend.
+ * [vllm] 7단계 "전체 흐름 요약" and Step 6 "Decode": in every decode step the new
+ * token's K/V is added to the cache and attention reads the cached K/V. For each
+ * request i with L = seq_lens[i] >= 1, k_new[i] and v_new[i] ([B, H, D], dtype
+ * dt) are written to the cache at token position L - 1 (physical block
+ * block_tables[i][(L-1)/S], offset (L-1)%S), and out[i] is the attention over
+ * the first L tokens, the new one included. The result, cache and output, is
+ * bit for bit that of pa_kv_append with those slots followed by pa_decode with
+ * the same arguments, with one launch fewer. Arguments are pa_decode's plus
+ * k_new and v_new (16-byte aligned); the cache is written.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_append(void* out, pa_dtype out_dt, const void* q, const void* k_new,
+                           const void* v_new, void* k_cache, void* v_cache,
+                           const int32_t* block_tables, int MB, const int32_t* seq_lens,
+                           float scale, int B, int H, int D, int S, int NB, pa_dtype dt,
+                           int partition, int max_seq_len, void* workspace, size_t ws_bytes,
+                           void* stream);
+
 /* Split-KV workspace layout, for tests that inspect the partition pass
  * (NP = number of partitions, all fp32, offsets in bytes from `workspace`):
  *   m   [B, H, NP] at 0                 max of scale * q.k * log2(e) (base-2 units)

@@ -12,7 +12,7 @@ One step, in this order (the order is part of the contract the tests check):
      at block boundaries, the new tokens' slots, padded block tables, lengths);
   2. host -> device copies of slots, tables and lengths;
   3. pa_kv_append of the step's new K/V, then pa_decode over every request's
-     cached tokens including the new one;
+     cached tokens including the new one (or both in one pa_decode_append);
   4. host: each request's token budget drops by one; for batch slots in index
      order, a finished request is freed (pa_seq_free) and its slot immediately
      refilled by the next arrival: grow to its prompt length and append its
@@ -57,8 +57,9 @@ class StagingRing:
 
 
 class ContinuousBatching:
-    def __init__(self, loop, device, max_steps=64, poison=True):
+    def __init__(self, loop, device, max_steps=64, poison=True, fused=False):
         self.loop = loop
+        self.fused = fused  # pa_decode_append instead of pa_kv_append + pa_decode
         self.device = device
         B, H, D, S = loop.batch, loop.H, loop.D, loop.S
         self.B, self.H, self.D, self.S = B, H, D, S
@@ -107,10 +108,15 @@ class ContinuousBatching:
         self.d_lens.copy_(h["lens"], non_blocking=True)
         self.staging.release()
         q, k, v = self.loop.token_kv(step_idx, self.B, self.device)
-        binding.pa_kv_append(k, v, self.d_slots, self.k_cache, self.v_cache)
         max_len = int(h["lens"].max())
-        binding.pa_decode(self.out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
-                          self.scale, max_len, partition=0, workspace=self.ws)
+        if self.fused:
+            binding.pa_decode_append(self.out, q, k, v, self.k_cache, self.v_cache,
+                                     self.d_tables, self.d_lens, self.scale, max_len,
+                                     partition=0, workspace=self.ws)
+        else:
+            binding.pa_kv_append(k, v, self.d_slots, self.k_cache, self.v_cache)
+            binding.pa_decode(self.out, q, self.k_cache, self.v_cache, self.d_tables,
+                              self.d_lens, self.scale, max_len, partition=0, workspace=self.ws)
         record = dict(ids=ids, slots=h["slots"].clone(), lens=h["lens"].clone(),
                       tables=h["tables"].clone(), q=q, k=k, v=v, out=self.out, retired=[],
                       admitted=[])

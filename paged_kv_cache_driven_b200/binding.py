@@ -32,6 +32,8 @@ _SIGNATURES = {
     "pa_decode": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32, _i32,
                    _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_get_device_error": ([_vp, _vp], _i32),
+    "pa_decode_append": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32,
+                          _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_decode_noalloc": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32,
                            _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "pa_alloc_create": ([_i32, _i32, _vp, _vp], _i32),
@@ -148,6 +150,28 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_l
                            _ptr(block_tables), MB, _ptr(seq_lens), float(scale), B, H, D, S, NB,
                            _DT[q.dtype], int(partition), int(max_seq_len), _ptr(workspace),
                            ws_bytes, _stream(stream)), "pa_decode")
+
+
+def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, scale,
+                     max_seq_len, partition=0, workspace=None, stream=None):
+    """One decode step in one launch: writes k_new, v_new [B, H, D] at each
+    request's last position (seq_lens[i] - 1), then decodes as pa_decode."""
+    for n, t in (("out", out), ("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                 ("v_cache", v_cache), ("block_tables", block_tables), ("seq_lens", seq_lens)):
+        _cuda(t, n)
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    if k_new.shape != q.shape or v_new.shape != q.shape or k_new.dtype != q.dtype:
+        raise ValueError("k_new, v_new must match q")
+    B, H, D = q.shape
+    NB, _, S, _ = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_decode_append(_ptr(out), _DT[out.dtype], _ptr(q), _ptr(k_new), _ptr(v_new),
+                                  _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), MB,
+                                  _ptr(seq_lens), float(scale), B, H, D, S, NB, _DT[q.dtype],
+                                  int(partition), int(max_seq_len), _ptr(workspace), ws_bytes,
+                                  _stream(stream)), "pa_decode_append")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

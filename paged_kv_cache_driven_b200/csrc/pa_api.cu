@@ -74,10 +74,10 @@ pa_status cuda_status() {
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <typename T, typename TO, int D, int S>
+template <typename T, typename TO, int D, int S, bool APPEND>
 pa_status launch_decode(const pa::DecodeParams& prm, cudaStream_t stream) {
   using Tl = pa::DecodeTiling<D, S>;
-  auto kern = pa::paged_decode_partition_kernel<T, TO, D, S>;
+  auto kern = pa::paged_decode_partition_kernel<T, TO, D, S, APPEND>;
   // The shared-memory opt-in is a per-device property of the function.
   static bool configured[kMaxDevices] = {};
   int dev = 0;
@@ -91,15 +91,17 @@ pa_status launch_decode(const pa::DecodeParams& prm, cudaStream_t stream) {
   const dim3 grid(prm.NP, prm.H, prm.B);
   kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
   if (prm.NP > 1) {
-    pa::splitkv_reduce_kernel<TO, D><<<dim3(prm.H, prm.B), 128, 0, stream>>>(prm);
+    const int64_t pairs = static_cast<int64_t>(prm.B) * prm.H;
+    pa::splitkv_reduce_kernel<TO, D>
+        <<<static_cast<unsigned>((pairs + 3) / 4), 128, 0, stream>>>(prm);
   }
   return cuda_status();
 }
 
-template <typename T, typename TO>
+template <typename T, typename TO, bool APPEND>
 pa_status dispatch_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t st) {
 #define PA_CASE(DD, SS) \
-  if (D == DD && S == SS) return launch_decode<T, TO, DD, SS>(prm, st);
+  if (D == DD && S == SS) return launch_decode<T, TO, DD, SS, APPEND>(prm, st);
   PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
   PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
   PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
@@ -107,13 +109,13 @@ pa_status dispatch_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t
   return PA_ERR_INVALID;
 }
 
-template <typename T>
+template <typename T, bool APPEND>
 pa_status dispatch_out(const pa::DecodeParams& prm, pa_dtype out_dt, int D, int S,
                        cudaStream_t st) {
   switch (out_dt) {
-    case PA_F32: return dispatch_shape<T, float>(prm, D, S, st);
-    case PA_F16: return dispatch_shape<T, __half>(prm, D, S, st);
-    case PA_BF16: return dispatch_shape<T, __nv_bfloat16>(prm, D, S, st);
+    case PA_F32: return dispatch_shape<T, float, APPEND>(prm, D, S, st);
+    case PA_F16: return dispatch_shape<T, __half, APPEND>(prm, D, S, st);
+    case PA_BF16: return dispatch_shape<T, __nv_bfloat16, APPEND>(prm, D, S, st);
   }
   return PA_ERR_INVALID;
 }
@@ -176,11 +178,16 @@ size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, in
   return workspace_for(B, H, D, NP);
 }
 
-pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
-                    const void* v_cache, const int32_t* block_tables, int MB,
-                    const int32_t* seq_lens, float scale, int B, int H, int D, int S, int NB,
-                    pa_dtype dt, int partition, int max_seq_len, void* workspace,
-                    size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// pa_decode and pa_decode_append: k_new / v_new null = plain decode.
+pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_new,
+                      const void* v_new, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
+                      int B, int H, int D, int S, int NB, pa_dtype dt, int partition,
+                      int max_seq_len, void* workspace, size_t ws_bytes, void* stream) {
   if (B < 0 || H <= 0 || NB < 0 || MB < 0) return PA_ERR_INVALID;
   if (!cache_dtype_ok(dt) || !out_dtype_ok(out_dt) || !decode_shape_ok(D, S)) return PA_ERR_INVALID;
   if (!std::isfinite(scale)) return PA_ERR_INVALID;
@@ -224,8 +231,41 @@ pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cac
     prm.L_cap = static_cast<int>(L_max);
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dt == PA_F16) return dispatch_out<__half>(prm, out_dt, D, S, st);
-  return dispatch_out<__nv_bfloat16>(prm, out_dt, D, S, st);
+  prm.k_new = k_new;
+  prm.v_new = v_new;
+  if (k_new) {
+    if (dt == PA_F16) return dispatch_out<__half, true>(prm, out_dt, D, S, st);
+    return dispatch_out<__nv_bfloat16, true>(prm, out_dt, D, S, st);
+  }
+  if (dt == PA_F16) return dispatch_out<__half, false>(prm, out_dt, D, S, st);
+  return dispatch_out<__nv_bfloat16, false>(prm, out_dt, D, S, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
+                    const void* v_cache, const int32_t* block_tables, int MB,
+                    const int32_t* seq_lens, float scale, int B, int H, int D, int S, int NB,
+                    pa_dtype dt, int partition, int max_seq_len, void* workspace,
+                    size_t ws_bytes, void* stream) {
+  return decode_impl(out, out_dt, q, nullptr, nullptr, k_cache, v_cache, block_tables, MB,
+                     seq_lens, scale, B, H, D, S, NB, dt, partition, max_seq_len, workspace,
+                     ws_bytes, stream);
+}
+
+pa_status pa_decode_append(void* out, pa_dtype out_dt, const void* q, const void* k_new,
+                           const void* v_new, void* k_cache, void* v_cache,
+                           const int32_t* block_tables, int MB, const int32_t* seq_lens,
+                           float scale, int B, int H, int D, int S, int NB, pa_dtype dt,
+                           int partition, int max_seq_len, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  if (B > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)))
+    return PA_ERR_INVALID;
+  return decode_impl(out, out_dt, q, B > 0 ? k_new : nullptr, v_new, k_cache, v_cache,
+                     block_tables, MB, seq_lens, scale, B, H, D, S, NB, dt, partition,
+                     max_seq_len, workspace, ws_bytes, stream);
 }
 
 pa_status pa_get_device_error(void* stream, uint32_t* flags) {

@@ -46,6 +46,8 @@ struct DecodeParams {
   float* ws_m;                 // [B, H, NP]
   float* ws_l;                 // [B, H, NP]
   float* ws_acc;               // [B, H, NP, D]
+  const void* k_new;           // [B, H, D] fused append: the new token's K (or null)
+  const void* v_new;           // [B, H, D] fused append: the new token's V (or null)
   float q_scale;               // scale * log2(e)
   int MB, B, H, NB;
   int P;     // tokens per partition (multiple of S)
@@ -89,7 +91,27 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[S], int lane) {
   return r;
 }
 
-template <typename T, typename TO, int D, int S>
+// Raw 16-bit row fragment of DL elements (4, 8 or 16 bytes) for copying K/V
+// rows bit for bit.
+template <int DL>
+struct RawRow {
+  uint32_t w[DL / 2];
+  __device__ __forceinline__ void load(const void* src) {
+#pragma unroll
+    for (int k = 0; k < DL / 2; ++k) w[k] = reinterpret_cast<const uint32_t*>(src)[k];
+  }
+  __device__ __forceinline__ void store(void* dst) const {
+#pragma unroll
+    for (int k = 0; k < DL / 2; ++k) reinterpret_cast<uint32_t*>(dst)[k] = w[k];
+  }
+};
+
+// APPEND = true fuses the decode step's append: for request i with L >= 1, the
+// new token (position L - 1) takes its K/V from k_new / v_new. The warp whose
+// run holds that token's block copies the rows into its shared-memory slabs
+// once the bulk copy has landed (so the scores see them) and stores them to
+// the cache, as pa_kv_append would have before the decode.
+template <typename T, typename TO, int D, int S, bool APPEND>
 __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
     paged_decode_partition_kernel(const DecodeParams p) {
   using Tl = DecodeTiling<D, S>;
@@ -104,7 +126,8 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
   const int w = threadIdx.x >> 5;
 
   int L = __ldg(p.seq_lens + i);
-  if (L < 0 || L > p.L_cap) {
+  const bool len_ok = L >= 0 && L <= p.L_cap;
+  if (!len_ok) {
     if (threadIdx.x == 0 && part == 0 && h == 0) raise_error(PA_DEVERR_SEQ_LEN);
     L = L < 0 ? 0 : p.L_cap;
   }
@@ -151,6 +174,19 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
       static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(h) * SLAB;
   const int64_t block_stride = static_cast<int64_t>(p.H) * SLAB;  // bytes per physical block
   const uint64_t policy = policy_evict_first();
+
+  // Fused append: does this warp own the new token's block?
+  const int t_new = L - 1;
+  // (a clamped, out-of-range length appends nothing: its position is unknown)
+  const bool appender = APPEND && len_ok && L >= 1 && t_new / S >= wb && t_new / S < we;
+  RawRow<DL> k_row, v_row;
+  int id_new = -1;
+  if (appender) {
+    const int64_t off = ((static_cast<int64_t>(i) * p.H + h) * D + lane * DL) * 2;
+    k_row.load(static_cast<const uint8_t*>(p.k_new) + off);
+    v_row.load(static_cast<const uint8_t*>(p.v_new) + off);
+    id_new = __ldg(trow + t_new / S);
+  }
 
   // Block-id prefetch: ids_a holds the chunk of 32 being issued, ids_b the next.
   int ids_a = (wb + lane < we) ? __ldg(trow + wb + lane) : -1;
@@ -206,6 +242,20 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
       const int nvalid = min(S, L - j * S);
       const uint8_t* ks = stage0 + s * STAGE;
       const uint8_t* vs = ks + SLAB;
+      if (APPEND && appender && j == t_new / S) {
+        // the bulk copy brought the block's old bytes; put the new token's row
+        // in both the staged slabs and the cache
+        const int64_t row_off = (static_cast<int64_t>(t_new % S) * D + lane * DL) * 2;
+        k_row.store(stage0 + s * STAGE + row_off);
+        v_row.store(stage0 + s * STAGE + SLAB + row_off);
+        const int64_t goff = static_cast<int64_t>(id_new) * block_stride + row_off;
+        k_row.store(const_cast<uint8_t*>(kbase) + goff);
+        v_row.store(const_cast<uint8_t*>(vbase) + goff);
+        // these generic-proxy writes must be ordered before the next bulk copy
+        // (async proxy) that reuses this stage
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+      }
 
       float part_dot[S];
 #pragma unroll
@@ -290,28 +340,55 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
 
 // Merges the partitions of every (request, head) that has more than one:
 //   M = max_p m_p;  out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.
+// One warp per (request, head): lanes load the partitions' m and l in parallel
+// (32 at a time), then every lane accumulates its D/32 output elements over
+// the partitions with the weights broadcast by shuffle.
 template <typename TO, int D>
 __global__ void __launch_bounds__(128) splitkv_reduce_kernel(const DecodeParams p) {
-  const int h = blockIdx.x;
-  const int i = blockIdx.y;
+  constexpr int DL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t ih = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (ih >= static_cast<int64_t>(p.B) * p.H) return;
+  const int i = static_cast<int>(ih / p.H);
   int L = __ldg(p.seq_lens + i);
   L = L < 0 ? 0 : (L > p.L_cap ? p.L_cap : L);
   const int nparts = (L + p.P - 1) / p.P;
   if (nparts <= 1) return;  // written by the partition pass
-  const int64_t ih = static_cast<int64_t>(i) * p.H + h;
   const float* m = p.ws_m + ih * p.NP;
   const float* l = p.ws_l + ih * p.NP;
-  const float* acc = p.ws_acc + ih * p.NP * D;
+  const float* acc = p.ws_acc + ih * p.NP * D + lane * DL;
 
   float M = -INFINITY;
-  for (int q = 0; q < nparts; ++q) M = fmaxf(M, m[q]);
-  float Ltot = 0.f;
-  for (int q = 0; q < nparts; ++q) Ltot = fmaf(exp2f(m[q] - M), l[q], Ltot);
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float a = 0.f;
-    for (int q = 0; q < nparts; ++q) a = fmaf(exp2f(m[q] - M), acc[static_cast<int64_t>(q) * D + d], a);
-    static_cast<TO*>(p.out)[ih * D + d] = to_out<TO>(Ltot > 0.f ? a / Ltot : 0.f);
+  for (int q = lane; q < nparts; q += 32) M = fmaxf(M, m[q]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
+
+  float lsum = 0.f;
+  float a[DL];
+#pragma unroll
+  for (int e = 0; e < DL; ++e) a[e] = 0.f;
+  for (int c = 0; c < nparts; c += 32) {
+    const int q = c + lane;
+    const float wq = q < nparts ? exp2f(m[q] - M) : 0.f;
+    if (q < nparts) lsum = fmaf(wq, l[q], lsum);
+    const int n = min(32, nparts - c);
+#pragma unroll 4
+    for (int r = 0; r < n; ++r) {
+      const float w = __shfl_sync(kFullMask, wq, r);
+      const float* row = acc + static_cast<int64_t>(c + r) * D;
+#pragma unroll
+      for (int e = 0; e < DL; e += 2) {
+        const float2 v = *reinterpret_cast<const float2*>(row + e);
+        a[e] = fmaf(w, v.x, a[e]);
+        a[e + 1] = fmaf(w, v.y, a[e + 1]);
+      }
+    }
   }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, off);
+  TO* o = static_cast<TO*>(p.out) + ih * D + lane * DL;
+#pragma unroll
+  for (int e = 0; e < DL; ++e) o[e] = to_out<TO>(lsum > 0.f ? a[e] / lsum : 0.f);
 }
 
 }  // namespace pa

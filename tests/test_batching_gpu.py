@@ -81,9 +81,9 @@ class OracleMirror:
         return want
 
 
-def run_loop(batch, H, steps, check_steps, heads, seed):
+def run_loop(batch, H, steps, check_steps, heads, seed, fused=False):
     loop = workloads.batching_loop(seed=seed, batch=batch, H=H)
-    drv = ContinuousBatching(loop, DEV, max_steps=steps)
+    drv = ContinuousBatching(loop, DEV, max_steps=steps, fused=fused)
     mirror = OracleMirror(loop, heads, drv.MB)
     assert drv.alloc.pa_alloc_dump() == mirror.model.dump()
     n_retired = 0
@@ -103,14 +103,18 @@ def run_loop(batch, H, steps, check_steps, heads, seed):
     return n_retired
 
 
-def test_batching_loop_reduced_every_step():
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "fused"])
+def test_batching_loop_reduced_every_step(fused):
     """Batch 16, 4 heads, 64 steps: every output, every cache byte, every step."""
-    n = run_loop(batch=16, H=4, steps=64, check_steps=set(range(64)), heads=[0, 1, 2, 3], seed=1)
+    n = run_loop(batch=16, H=4, steps=64, check_steps=set(range(64)), heads=[0, 1, 2, 3], seed=1,
+                 fused=fused)
     assert n > 0  # some requests retired and were replaced
 
 
-def test_batching_loop_full_size():
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "fused"])
+def test_batching_loop_full_size(fused):
     """Batch 256, 40 heads, a 66,560-block shuffled pool, 64 steps: allocator state
     every step; cache and decode on two mirrored heads at three steps."""
-    n = run_loop(batch=256, H=40, steps=64, check_steps={0, 31, 63}, heads=[0, 39], seed=0)
+    n = run_loop(batch=256, H=40, steps=64, check_steps={0, 31, 63}, heads=[0, 39], seed=0,
+                 fused=fused)
     assert n > 50  # mean budget 128: about 40% of 256 requests stop within 64 steps
