@@ -81,6 +81,7 @@ class ClockSampler:
         self.samples = []
         self.window = [None, None]
         self._stop = threading.Event()
+        self._ready = threading.Event()  # set once the first sample (or a failure) is in
         self._thread = threading.Thread(target=self._run, daemon=True)
         self.max_mhz = None
         self.source = None
@@ -102,10 +103,13 @@ class ClockSampler:
                 mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
                 reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
                 self.samples.append((t, float(mhz), int(reasons)))
+                self._ready.set()
                 time.sleep(0.001)
             nv.nvmlShutdown()
         except Exception:
             self._run_smi()
+        finally:
+            self._ready.set()
 
     def _run_smi(self):
         q = "clocks.sm,clocks.max.sm,clocks_event_reasons.active"
@@ -124,13 +128,14 @@ class ClockSampler:
             try:
                 self.max_mhz = float(f[1])
                 self.samples.append((time.perf_counter(), float(f[0]), int(f[2], 16)))
+                self._ready.set()
             except (ValueError, IndexError):
                 continue
         proc.terminate()
 
     def __enter__(self):
         self._thread.start()
-        time.sleep(0.05)
+        self._ready.wait(timeout=10.0)  # the timed region starts only once sampling runs
         return self
 
     def __exit__(self, *exc):
@@ -528,6 +533,8 @@ def main():
                          "call_ms": round(dec_ms, 4),
                          "algorithmic_bytes_per_launch": step_bytes},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                    "api": "pa_stepper_step (host allocator step, uploads, pa_decode_append, "
+                           "download; every request grows by one token per step)",
                     "h2d_bytes_per_step": wl.h2d_bytes(), "d2h_bytes_per_step": wl.d2h_bytes(),
                     "ms_per_step": round(e2e_ms / args.steps, 4)},
             "gpu_launches": wl.launches_per_step(fused=True) * args.steps,

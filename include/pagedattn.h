@@ -240,6 +240,51 @@ pa_status pa_alloc_stats(const pa_alloc* a, int* free_blocks, int64_t* used_slot
  * next), into dst[0..cap); *n receives its length. For bit-exact tests. */
 pa_status pa_alloc_dump(const pa_alloc* a, int32_t* free_list, int cap, int* n);
 
+/* ---------------------------------------------------------------------------
+ * Host-fed decode step executor ([vllm] 7단계 "전체 흐름 요약", Step 8; [card]
+ * "vLLM에서의 위치": the worker turns the scheduler's block tables into device
+ * tensors each step). For a fixed batch of B running sequences whose per-step
+ * q, k, v arrive in host memory, one pa_stepper_step call grows every sequence
+ * by one token on the allocator (pa_prepare_step), uploads q|k|v and the
+ * tables and lengths, runs the decode with the append, and downloads the
+ * output. Transfers go on the executor's own copy stream and every staging
+ * buffer is `depth` sets deep, so a step's transfers overlap its neighbours'
+ * kernels. Unlike the calls above, the executor allocates: at creation it
+ * takes pinned host memory and device memory for its staging (depth sets of
+ * q|k|v, tables, lengths, output, plus the split-KV workspace) and a CUDA
+ * stream; pa_stepper_destroy releases them. Not thread-safe.
+ * ------------------------------------------------------------------------- */
+typedef struct pa_stepper pa_stepper;
+
+/* k_cache, v_cache [NB, H, S, D] (dtype dt) and the allocator `alloc` stay
+ * owned by the caller and must outlive the executor. max_len bounds every
+ * sequence length the executor will decode (sizes the workspace; <= MB * S).
+ * fused != 0 uses pa_decode_append, 0 uses pa_kv_append + pa_decode. depth in
+ * [1, 8]. compute_stream: the stream the kernels run on (NULL = legacy). */
+pa_status pa_stepper_create(pa_alloc* alloc, void* k_cache, void* v_cache, int B, int H, int D,
+                            int S, int NB, int MB, pa_dtype dt, pa_dtype out_dt, float scale,
+                            int max_len, int partition, int fused, int depth,
+                            void* compute_stream, pa_stepper** out);
+void pa_stepper_destroy(pa_stepper* s);
+
+/* Enqueues one step for seq_ids[0..B) (each must exist in the allocator and
+ * grows by one token). h_qkv: host memory (pinned, for the copy to overlap)
+ * holding q, k, v as [3, B, H, D], read by the upload; it must stay unchanged
+ * until the step's upload has run, i.e. until the next call that reuses the
+ * step's staging set (depth steps later) returns, or pa_stepper_output.
+ * *step_out receives the step's number, *max_len_out its longest sequence.
+ * PA_ERR_OUT_OF_RANGE (nothing changed) if a sequence would exceed max_len. */
+pa_status pa_stepper_step(pa_stepper* s, const int64_t* seq_ids, const void* h_qkv,
+                          int64_t* step_out, int* max_len_out);
+
+/* Waits for step `step`'s download and returns the host address of its output
+ * [B, H, D] (dtype out_dt), valid until the call that reuses its staging set.
+ * PA_ERR_OUT_OF_RANGE if that step is not among the last `depth` steps. */
+pa_status pa_stepper_output(pa_stepper* s, int64_t step, const void** host_out);
+
+/* Makes the compute stream wait for every outstanding download. */
+pa_status pa_stepper_drain(pa_stepper* s);
+
 #ifdef __cplusplus
 }
 #endif

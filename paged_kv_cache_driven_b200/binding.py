@@ -36,6 +36,12 @@ _SIGNATURES = {
                           _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_decode_noalloc": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32,
                            _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "pa_stepper_create": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                           ctypes.c_float, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
+    "pa_stepper_destroy": ([_vp], None),
+    "pa_stepper_step": ([_vp, _vp, _vp, _vp, _vp], _i32),
+    "pa_stepper_output": ([_vp, _i64, _vp], _i32),
+    "pa_stepper_drain": ([_vp], _i32),
     "pa_alloc_create": ([_i32, _i32, _vp, _vp], _i32),
     "pa_alloc_destroy": ([_vp], None),
     "pa_seq_grow": ([_vp, _i64, _i32], _i32),

@@ -1,28 +1,15 @@
-"""Decode steps fed from host memory, with transfers overlapped with kernels.
+"""Decode steps fed from host memory: a thin wrapper of the library's native
+step executor (pa_stepper_* in include/pagedattn.h).
 
-Each step of the decode loop ("vLLM KV Cache and PagedAttention Explained",
-7단계 "전체 흐름 요약": the new token's K/V goes into the cache, then attention
-reads the cached K/V) needs the step's q and new K/V, the block tables and the
-lengths on the device, and its output back on the host. ``HostFedDecoder`` runs
-those steps through the C ABI with the copies on a second CUDA stream and every
-device and pinned host buffer ``depth`` sets deep, so the copies of step n+1
-and the result copy of step n-1 run while the kernels of step n do:
-
-  host          : pa_prepare_step(n) -> staging set n % depth
-                  (after that set's upload of step n - depth has landed)
-  copy stream   : wait compute(n - depth) ; upload q|k|v and tables|lengths ; record up(n)
-  compute stream: wait up(n) ; pa_decode_append (or pa_kv_append + pa_decode) ; record compute(n)
-  copy stream   : wait compute(n) ; download out(n) ; record down(n)
-
-The KV cache is only touched on the compute stream, so steps stay in order.
-Per step the host does one allocator call, two uploads, one decode call and
-one download; the C calls go through ctypes with their arguments converted
-once, so the host stays ahead of a ~200 us decode.
+One ``step`` call runs, in C++, the host allocator's step for the batch, the
+uploads of q|k|v and of the block tables and lengths on the executor's copy
+stream, the decode with the append on the compute stream, and the download of
+the output, with the transfers of neighbouring steps overlapped with the
+kernels (see csrc/pa_stepper.cpp). This module only converts arguments.
 """
 
 import ctypes
 
-import numpy as np
 import torch
 
 from . import binding
@@ -30,124 +17,65 @@ from . import binding
 
 class HostFedDecoder:
     def __init__(self, alloc, k_cache, v_cache, batch, max_blocks, max_len, out_dtype=None,
-                 depth=2, partition=0, fused=True):
+                 depth=2, partition=0, fused=True, stream=None):
         NB, H, S, D = k_cache.shape
-        self.alloc, self.k_cache, self.v_cache = alloc, k_cache, v_cache
         self.B, self.H, self.S, self.D, self.MB = batch, H, S, D, max_blocks
-        self.partition = partition
-        self.fused = fused  # pa_decode_append (slots derived on the device) or two calls
-        self.device = k_cache.device
+        self.fused = fused
         self.dtype = k_cache.dtype
         self.out_dtype = out_dtype or k_cache.dtype
-        self.scale = D ** -0.5
-        self.compute = torch.cuda.current_stream(self.device)
-        self.copy = torch.cuda.Stream(self.device)
-        ws = binding.pa_decode_workspace_bytes(batch, H, D, S, max_len, partition)
-        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
-        dev, pin = dict(device=self.device), dict(pin_memory=True)
-        meta_n = batch * max_blocks + batch
-        self.sets = []
-        for _ in range(depth):
-            s = dict(
-                h_slots=torch.empty(batch, dtype=torch.int64, **pin),
-                h_meta=torch.empty(meta_n, dtype=torch.int32, **pin),  # tables | lengths
-                h_out=torch.empty((batch, H, D), dtype=self.out_dtype, **pin),
-                d_qkv=torch.empty((3, batch, H, D), dtype=self.dtype, **dev),
-                d_slots=torch.empty(batch, dtype=torch.int64, **dev),
-                d_meta=torch.empty(meta_n, dtype=torch.int32, **dev),
-                d_out=torch.empty((batch, H, D), dtype=self.out_dtype, **dev),
-                ev_up=torch.cuda.Event(), ev_compute=torch.cuda.Event(),
-                ev_d2h=torch.cuda.Event(), used=False)
-            s["h_tables"] = s["h_meta"][:batch * max_blocks].view(batch, max_blocks)
-            s["h_lens"] = s["h_meta"][batch * max_blocks:]
-            s["h_lens_np"] = s["h_lens"].numpy()
-            s["d_tables"] = s["d_meta"][:batch * max_blocks].view(batch, max_blocks)
-            s["d_lens"] = s["d_meta"][batch * max_blocks:]
-            s["args"] = self._decode_args(s)
-            self.sets.append(s)
+        self.stream = stream or torch.cuda.current_stream(k_cache.device)
+        self._keep = (alloc, k_cache, v_cache)  # the executor borrows these
+        handle = ctypes.c_void_p()
+        binding._check(binding.lib().pa_stepper_create(
+            alloc._h, ctypes.c_void_p(k_cache.data_ptr()), ctypes.c_void_p(v_cache.data_ptr()),
+            batch, H, D, S, NB, max_blocks, binding._DT[self.dtype], binding._DT[self.out_dtype],
+            D ** -0.5, max_len, partition, int(fused), depth,
+            ctypes.c_void_p(self.stream.cuda_stream), ctypes.byref(handle)), "pa_stepper_create")
+        self._h = handle
         self._ids_key, self._ids = None, None
-        self.n = 0
+        self._step_no, self._max_len = ctypes.c_int64(), ctypes.c_int()
 
-    def _decode_args(self, s):
-        """pa_decode_append / pa_decode arguments of one buffer set, as ctypes values;
-        the entry 'max_seq_len' is filled in per step."""
-        p = lambda t: ctypes.c_void_p(t.data_ptr())
-        dt = binding._DT[self.dtype]
-        q, k, v = s["d_qkv"][0], s["d_qkv"][1], s["d_qkv"][2]
-        NB = self.k_cache.shape[0]
-        common = dict(out=p(s["d_out"]), out_dt=binding._DT[self.out_dtype], q=p(q), k=p(k),
-                      v=p(v), kc=p(self.k_cache), vc=p(self.v_cache), bt=p(s["d_tables"]),
-                      lens=p(s["d_lens"]), ws=p(self.ws),
-                      ws_bytes=self.ws.numel(), dt=dt, NB=NB)
-        return common
+    def close(self):
+        if self._h:
+            binding.lib().pa_stepper_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
     def h2d_bytes(self):
         slots = 0 if self.fused else 8
-        return 3 * self.B * self.H * self.D * self.k_cache.element_size() + \
+        return 3 * self.B * self.H * self.D * torch.empty((), dtype=self.dtype).element_size() + \
             self.B * (slots + 4 * self.MB + 4)
 
     def d2h_bytes(self):
         return self.B * self.H * self.D * torch.empty((), dtype=self.out_dtype).element_size()
 
-    def _seq_ids(self, seq_ids):
+    def step(self, seq_ids, h_qkv):
+        """Enqueues one decode step: every sequence in ``seq_ids`` grows by one
+        token. ``h_qkv`` [3, batch, H, D] (q, k, v) in pinned host memory must stay
+        unchanged until the step's upload has run. Returns (step number, longest
+        sequence decoded)."""
         key = tuple(seq_ids)
         if key != self._ids_key:
             self._ids_key, self._ids = key, (ctypes.c_int64 * len(key))(*key)
-        return self._ids
+        binding._check(binding.lib().pa_stepper_step(
+            self._h, self._ids, ctypes.c_void_p(h_qkv.data_ptr()), ctypes.byref(self._step_no),
+            ctypes.byref(self._max_len)), "pa_stepper_step")
+        return self._step_no.value, self._max_len.value
 
-    def step(self, seq_ids, h_qkv):
-        """Enqueues one decode step for ``seq_ids`` (each grows by one token).
-        ``h_qkv`` [3, batch, H, D] holds q, k, v in pinned host memory and must stay
-        unchanged until the step's upload has run. Returns (max length decoded,
-        buffer set); the output is ``set["h_out"]`` once ``set["ev_d2h"]`` completes."""
-        s = self.sets[self.n % len(self.sets)]
-        lib = binding.lib()
-        if s["used"]:
-            s["ev_up"].synchronize()  # this set's previous upload has landed
-        ids = self._seq_ids(seq_ids)
-        rc = lib.pa_prepare_step(self.alloc._h, ids, len(ids), 1, self.MB,
-                                 ctypes.c_void_p(s["h_slots"].data_ptr()),
-                                 ctypes.c_void_p(s["h_tables"].data_ptr()),
-                                 ctypes.c_void_p(s["h_lens"].data_ptr()))
-        binding._check(rc, "pa_prepare_step")
-        max_len = int(s["h_lens_np"].max())
-        with torch.cuda.stream(self.copy):
-            if s["used"]:
-                self.copy.wait_event(s["ev_compute"])  # kernels of step n - depth read these
-            s["d_qkv"].copy_(h_qkv, non_blocking=True)
-            s["d_meta"].copy_(s["h_meta"], non_blocking=True)
-            if not self.fused:
-                s["d_slots"].copy_(s["h_slots"], non_blocking=True)
-            s["ev_up"].record(self.copy)
-        self.compute.wait_event(s["ev_up"])
-        a = s["args"]
-        st = ctypes.c_void_p(self.compute.cuda_stream)
-        if self.fused:
-            rc = lib.pa_decode_append(a["out"], a["out_dt"], a["q"], a["k"], a["v"], a["kc"],
-                                      a["vc"], a["bt"], self.MB, a["lens"], self.scale, self.B,
-                                      self.H, self.D, self.S, a["NB"], a["dt"], self.partition,
-                                      max_len, a["ws"], a["ws_bytes"], st)
-            binding._check(rc, "pa_decode_append")
-        else:
-            rc = lib.pa_kv_append(a["k"], a["v"], ctypes.c_void_p(s["d_slots"].data_ptr()),
-                                  a["kc"], a["vc"], self.B, self.H, self.D, self.S, a["NB"],
-                                  a["dt"], st)
-            binding._check(rc, "pa_kv_append")
-            rc = lib.pa_decode(a["out"], a["out_dt"], a["q"], a["kc"], a["vc"], a["bt"], self.MB,
-                               a["lens"], self.scale, self.B, self.H, self.D, self.S, a["NB"],
-                               a["dt"], self.partition, max_len, a["ws"], a["ws_bytes"], st)
-            binding._check(rc, "pa_decode")
-        s["ev_compute"].record(self.compute)
-        with torch.cuda.stream(self.copy):
-            self.copy.wait_event(s["ev_compute"])
-            s["h_out"].copy_(s["d_out"], non_blocking=True)
-            s["ev_d2h"].record(self.copy)
-        s["used"] = True
-        self.n += 1
-        return max_len, s
+    def output(self, step_no):
+        """The output [batch, H, D] of a recent step (waits for its download)."""
+        ptr = ctypes.c_void_p()
+        binding._check(binding.lib().pa_stepper_output(self._h, step_no, ctypes.byref(ptr)),
+                       "pa_stepper_output")
+        n = self.d2h_bytes()
+        buf = (ctypes.c_uint8 * n).from_address(ptr.value)
+        return torch.frombuffer(bytearray(buf), dtype=self.out_dtype).view(self.B, self.H, self.D)
 
     def drain(self):
-        """Makes the compute stream wait for every outstanding result copy."""
-        for s in self.sets:
-            if s["used"]:
-                self.compute.wait_event(s["ev_d2h"])
+        """Makes the compute stream wait for every outstanding download."""
+        binding._check(binding.lib().pa_stepper_drain(self._h), "pa_stepper_drain")

@@ -102,3 +102,17 @@ def test_append_rejects_bad_arguments_on_host(lib, bad):
 
 def test_append_zero_tokens_is_noop(lib):
     assert lib.pa_kv_append(*append_args(T=0, k=NULL, v=NULL)) == binding.PA_OK
+
+
+def test_stepper_rejects_bad_arguments_on_host(lib):
+    h = ctypes.c_void_p()
+    a = binding.BlockAllocator(8, 16)
+    base = [a._h, P, P, 4, 2, 64, 16, 8, 8, binding.PA_BF16, binding.PA_F32, 0.1, 100, 0, 1, 2,
+            NULL, ctypes.byref(h)]
+    for idx, bad in [(0, NULL), (1, NULL), (3, 0), (9, binding.PA_F32), (10, 9), (12, 8 * 16 + 1),
+                     (15, 0), (15, 9), (13, 24)]:
+        args = list(base)
+        args[idx] = bad
+        assert lib.pa_stepper_create(*args) == binding.PA_ERR_INVALID, idx
+    assert lib.pa_stepper_step(NULL, P, P, NULL, NULL) == binding.PA_ERR_INVALID
+    assert lib.pa_stepper_output(NULL, 0, ctypes.byref(h)) == binding.PA_ERR_INVALID

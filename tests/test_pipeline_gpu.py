@@ -1,5 +1,5 @@
-"""HostFedDecoder (decode steps fed from pinned host memory, copies overlapped
-with kernels on a second stream) against the same steps run one call at a time,
+"""HostFedDecoder / pa_stepper_* (decode steps fed from pinned host memory,
+copies overlapped with kernels on a second stream) against the same steps run one call at a time,
 and its last step against the oracle."""
 
 import math
@@ -48,14 +48,17 @@ def test_pipelined_steps_equal_sequential_steps(fused):
     fed = HostFedDecoder(alloc, kc, vc, B, MB, max_len, out_dtype=torch.float32, fused=fused)
     got, prev = [], None
     for n in range(steps):
-        _, s = fed.step(ids, inputs[n])
+        step_no, _ = fed.step(ids, inputs[n])
+        assert step_no == n
         if prev is not None:  # read step n-1 while step n is in flight
-            prev["ev_d2h"].synchronize()
-            got.append(prev["h_out"].clone())
-        prev = s
+            got.append(fed.output(prev))
+        prev = step_no
     fed.drain()
     torch.cuda.synchronize()
-    got.append(prev["h_out"].clone())
+    got.append(fed.output(prev))
+    with pytest.raises(binding.PagedAttnError):
+        fed.output(0)  # its staging set has been reused
+    fed.close()
 
     ws = torch.empty(binding.pa_decode_workspace_bytes(B, H, D, S, max_len, 0) + 16,
                      dtype=torch.uint8, device=DEV)
