@@ -407,6 +407,80 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def decode_bytes_case(case):
+    """Algorithmic bytes of one pa_decode call on a workloads.DecodeCase."""
+    B, Hc, Dc = case.q.shape
+    Sc = case.k_cache.shape[2]
+    e = case.q.element_size()
+    return sum(Hc * (2 * L * Dc * e + 2 * Dc * e) + 4 * (-(-L // Sc)) for L in case.seq_lens_host) \
+        + 4 * B
+
+
+def time_decode_case(case, iters, warmup, partition=0):
+    """Median event-timed pa_decode call with L2 flushed (a 256 MB write) before each."""
+    B, Hc, Dc = case.q.shape
+    Sc = case.k_cache.shape[2]
+    maxlen = max(case.seq_lens_host)
+    out = torch.empty((B, Hc, Dc), dtype=case.q.dtype, device=case.q.device)
+    wsb = binding.pa_decode_workspace_bytes(B, Hc, Dc, Sc, maxlen, partition)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=case.q.device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=case.q.device)
+    times = []
+    for k in range(warmup + iters):
+        flush.fill_(k & 0xff)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        binding.pa_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables,
+                          case.seq_lens, case.scale, maxlen, partition=partition, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        if k >= warmup:
+            times.append(a.elapsed_time(b))
+    if binding.pa_get_device_error():
+        raise SystemExit("device error word set")
+    return statistics.median(times), binding.pa_decode_plan(B, Hc, Dc, Sc, maxlen, partition)
+
+
+def run_shape_workloads(args):
+    """--workload long_context | sweep: decode-only KV GB/s of the other
+    configurations, one JSON line per case (L2 flushed before every call)."""
+    device = torch.device("cuda", 0)
+    peak, peak_kind = measured_peak()
+    if args.workload == "long_context":
+        cases = [("long_context", lambda: workloads.long_context_decode(seed=args.seed,
+                                                                        device=device))]
+    else:
+        cases = []
+        for Sx in (8, 16, 32):
+            for Dx in (64, 128, 256):
+                for Bx in (1, 32, 256):
+                    for dt in (torch.float16, torch.bfloat16):
+                        name = f"S{Sx}_D{Dx}_B{Bx}_{'fp16' if dt == torch.float16 else 'bf16'}"
+                        cases.append((name, (lambda Sx=Sx, Dx=Dx, Bx=Bx, dt=dt: workloads.sweep_case(
+                            Sx, Dx, Bx, dt, seed=args.seed, device=device))))
+    rows = []
+    for name, make in cases:
+        case = make()
+        ms, plan = time_decode_case(case, args.steps, args.warmup)
+        nbytes = decode_bytes_case(case)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        row = {"workload": name, "ms": round(ms, 4), "gb_s": round(gbs, 1),
+               "frac_of_peak": round(gbs / peak, 3), "kv_bytes": nbytes,
+               "tok_s_layer": round(case.q.shape[0] / (ms / 1e3), 1),
+               "partition": {"tokens": plan[0], "num": plan[1]}}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+        del case
+        torch.cuda.empty_cache()
+    big = [r for r in rows if r["kv_bytes"] > 1 << 30]
+    summary = {"metric": METRIC + " (decode only)", "workload": args.workload,
+               "peak": peak, "peak_kind": peak_kind, "cases": len(rows),
+               "min_frac_over_1GB": min((r["frac_of_peak"] for r in big), default=None),
+               "median_frac_over_1GB": statistics.median([r["frac_of_peak"] for r in big])
+               if big else None}
+    print(json.dumps(summary), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,11 +489,18 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="llama13b", choices=["llama13b", "long_context", "sweep"],
+                    help="llama13b: the headline step (default); the others time decode-only "
+                         "calls of the long-context and shape-sweep configurations")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.workload != "llama13b":
+        binding.lib()
+        run_shape_workloads(args)
         return
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
