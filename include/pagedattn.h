@@ -109,7 +109,9 @@ size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, in
 
 /* The partition length (tokens) and the number of partitions pa_decode will use
  * for these arguments on the current device; *partition_tokens = 0 and
- * *num_partitions = 1 mean a single pass with no workspace. */
+ * *num_partitions = 1 mean a single pass with no workspace. The automatic choice
+ * (partition = 0) depends on B * H and the device's SM count: call this and
+ * pa_decode_workspace_bytes with the device current that pa_decode will run on. */
 pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partition,
                          int* partition_tokens, int* num_partitions);
 

@@ -33,12 +33,25 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// SMs of the current device (148 on B200; also the answer without a device).
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();  // clear the error state of the failed query
+    return 148;
+  }
+  return n;
+}
+
 // Chooses the partition length. Returns false on an invalid `partition`.
 //   -1      never split: one partition covering any length up to MB * S
 //   > 0     that many tokens (a multiple of S)
-//   0       automatic: split only when the longest request spans more than
-//           one default partition
-bool plan(int S, int max_seq_len, int partition, int* P_out, int* NP_out) {
+//   0       automatic: 512-token partitions, halved (down to 64 tokens, staying a
+//           multiple of S) while the grid would hold fewer than about four
+//           waves of CTAs (three CTAs per SM), so that small batches still
+//           spread over every SM; no split if one partition covers every request
+bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* NP_out) {
   if (max_seq_len < 0 || S <= 0) return false;
   int P;
   if (partition < 0) {
@@ -51,6 +64,9 @@ bool plan(int S, int max_seq_len, int partition, int* P_out, int* NP_out) {
     P = partition;
   } else {
     P = kDefaultPartition;
+    const int64_t target = 4LL * 3 * sm_count();
+    const int64_t pairs = static_cast<int64_t>(B > 0 ? B : 1) * (H > 0 ? H : 1);
+    while (P > 64 && (P / 2) % S == 0 && pairs * ceil_div(max_seq_len, P) < target) P /= 2;
   }
   const int64_t np = ceil_div(max_seq_len, P);
   if (np <= 1) {
@@ -166,7 +182,7 @@ pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partit
   (void)D;
   if (!partition_tokens || !num_partitions) return PA_ERR_INVALID;
   int P, NP;
-  if (!plan(S, max_seq_len, partition, &P, &NP)) return PA_ERR_INVALID;
+  if (!plan(B, H, S, max_seq_len, partition, &P, &NP)) return PA_ERR_INVALID;
   *partition_tokens = P;
   *num_partitions = NP;
   return PA_OK;
@@ -174,7 +190,7 @@ pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partit
 
 size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, int partition) {
   int P, NP;
-  if (B < 0 || H <= 0 || D <= 0 || !plan(S, max_seq_len, partition, &P, &NP)) return 0;
+  if (B < 0 || H <= 0 || D <= 0 || !plan(B, H, S, max_seq_len, partition, &P, &NP)) return 0;
   return workspace_for(B, H, D, NP);
 }
 
@@ -195,7 +211,7 @@ pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_n
   const int64_t L_max = static_cast<int64_t>(MB) * S;
   if (L_max > INT_MAX || max_seq_len < 0 || max_seq_len > L_max) return PA_ERR_INVALID;
   int P, NP;
-  if (!plan(S, max_seq_len, partition, &P, &NP)) return PA_ERR_INVALID;
+  if (!plan(B, H, S, max_seq_len, partition, &P, &NP)) return PA_ERR_INVALID;
   if (B == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || MB == 0)
     return PA_ERR_INVALID;
@@ -305,7 +321,7 @@ extern "C" pa_status pa_decode_noalloc(void* out, pa_dtype out_dt, const void* q
                                        int S, int NB, pa_dtype dt, int partition, int max_seq_len,
                                        void* stream) {
   int P, NP;
-  if (B < 0 || H <= 0 || !decode_shape_ok(D, S) || !plan(S, max_seq_len, partition, &P, &NP))
+  if (B < 0 || H <= 0 || !decode_shape_ok(D, S) || !plan(B, H, S, max_seq_len, partition, &P, &NP))
     return PA_ERR_INVALID;
   const size_t need = workspace_for(B, H, D, NP);
   if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_OOM;  // larger than the static array

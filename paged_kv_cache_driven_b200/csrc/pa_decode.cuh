@@ -55,11 +55,24 @@ struct DecodeParams {
   int L_cap; // lengths are clamped to this (MB*S, or NP*P when split)
 };
 
-// Shared-memory budget of one CTA: NW warps x NS stages x (K + V slabs).
+// Shapes of the partition pass for head_dim D and block_size S.
+//   EPL = 8  elements per lane per row fragment (one 16-byte shared load)
+//   LPR      lanes per row (D / 8: 8, 16 or 32); RPW = 32 / LPR rows per warp-wide load
+//   CR       rows per pipeline unit: CR x D of K and of V (about 4 KB each) is one
+//            stage, so the stage size no longer grows with S; a block of S rows
+//            is S / CR units
+//   NS, NW   stages per warp and warps per CTA: about 64 KB of stages per CTA
 template <int D, int S>
 struct DecodeTiling {
-  static constexpr int SLAB = S * D * 2;
-  static constexpr int STAGE = 2 * SLAB;
+  static constexpr int EPL = 8;
+  static constexpr int LPR = D / EPL;
+  static constexpr int RPW = 32 / LPR;
+  static constexpr int CR_RAW = 2048 / D;
+  static constexpr int CR = CR_RAW < S ? CR_RAW : S;
+  static constexpr int NV = CR / RPW;  // rows per lane per unit
+  static constexpr int SLAB = S * D * 2;     // one (block, head) slab of K or of V
+  static constexpr int UNIT = CR * D * 2;    // one unit of K or of V
+  static constexpr int STAGE = 2 * UNIT;
   static constexpr int NS = STAGE <= 4096 ? 4 : 2;
   static constexpr int NW_RAW = 65536 / (NS * STAGE);
   static constexpr int NW = NW_RAW < 1 ? 1 : (NW_RAW > 8 ? 8 : NW_RAW);
@@ -67,15 +80,20 @@ struct DecodeTiling {
   static constexpr int SMEM_BARS = NW * NS * 8;
   static constexpr int SMEM_MERGE = NW * (D + 2) * 4;
   static constexpr int SMEM = SMEM_PIPE + SMEM_BARS + SMEM_MERGE;
+  static_assert(S % CR == 0 && CR % RPW == 0 && NV >= 1 && NV <= LPR, "bad tiling");
+  static_assert(UNIT % 16 == 0, "bulk copies move multiples of 16 bytes");
 };
 
-// Sums S per-lane partial dot products across the warp. On return v[0] of lane
-// l holds the full dot product of token l / (32 / S) of the block.
-template <int S>
-__device__ __forceinline__ float transpose_reduce(float (&v)[S], int lane) {
-  // Halving steps: exchange half the values with lane ^ off, keep the other half.
+// Finishes NV per-lane partial dot products. Lane l of row group g = l / LPR
+// holds, in v[k], its fragment's partial dot of row k * RPW + g. The lanes of a
+// group exchange halves of their values (a transposing butterfly) so that each
+// value is summed over the group in NV - 1 + log2(LPR / NV) shuffles. On return
+// lane l holds the full dot of row (pl / DUP) * RPW + g, pl = l % LPR,
+// DUP = LPR / NV; the DUP lanes pl = k * DUP .. k * DUP + DUP - 1 hold row k's.
+template <int NV, int LPR>
+__device__ __forceinline__ float transpose_reduce(float (&v)[NV], int lane) {
 #pragma unroll
-  for (int n = S, off = 16; n > 1; n >>= 1, off >>= 1) {
+  for (int n = NV, off = LPR / 2; n > 1; n >>= 1, off >>= 1) {
     const bool upper = (lane & off) != 0;
 #pragma unroll
     for (int j = 0; j < n / 2; ++j) {
@@ -84,46 +102,43 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[S], int lane) {
       v[j] = keep + __shfl_xor_sync(kFullMask, send, off);
     }
   }
-  // Lanes sharing a token still hold disjoint partial sums: finish them.
   float r = v[0];
 #pragma unroll
-  for (int off = 16 / S; off >= 1; off >>= 1) r += __shfl_xor_sync(kFullMask, r, off);
+  for (int off = LPR / NV / 2; off >= 1; off >>= 1) r += __shfl_xor_sync(kFullMask, r, off);
   return r;
 }
 
-// Raw 16-bit row fragment of DL elements (4, 8 or 16 bytes) for copying K/V
-// rows bit for bit.
-template <int DL>
-struct RawRow {
-  uint32_t w[DL / 2];
-  __device__ __forceinline__ void load(const void* src) {
-#pragma unroll
-    for (int k = 0; k < DL / 2; ++k) w[k] = reinterpret_cast<const uint32_t*>(src)[k];
-  }
-  __device__ __forceinline__ void store(void* dst) const {
-#pragma unroll
-    for (int k = 0; k < DL / 2; ++k) reinterpret_cast<uint32_t*>(dst)[k] = w[k];
-  }
+// Raw 16-bit row fragment of 8 elements (16 bytes) for copying K/V rows bit for bit.
+struct RawFrag {
+  uint4 w;
+  __device__ __forceinline__ void load(const void* src) { w = *reinterpret_cast<const uint4*>(src); }
+  __device__ __forceinline__ void store(void* dst) const { *reinterpret_cast<uint4*>(dst) = w; }
 };
 
+// One CTA per (partition, head, request); NW warps, each an independent
+// pipeline over the tokens of a contiguous run of the partition's blocks,
+// taken CR rows (one unit) at a time.
+//
 // APPEND = true fuses the decode step's append: for request i with L >= 1, the
 // new token (position L - 1) takes its K/V from k_new / v_new. The warp whose
-// run holds that token's block copies the rows into its shared-memory slabs
-// once the bulk copy has landed (so the scores see them) and stores them to
-// the cache, as pa_kv_append would have before the decode.
+// run holds that token copies the row into its staged unit once the bulk copy
+// has landed (so the scores see it) and stores it to the cache, as
+// pa_kv_append would have before the decode.
 template <typename T, typename TO, int D, int S, bool APPEND>
 __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
     paged_decode_partition_kernel(const DecodeParams p) {
   using Tl = DecodeTiling<D, S>;
-  constexpr int NW = Tl::NW, NS = Tl::NS, SLAB = Tl::SLAB, STAGE = Tl::STAGE;
-  constexpr int DL = D / 32;   // elements per lane
-  constexpr int DUP = 32 / S;  // lanes holding the same token's score
+  constexpr int NW = Tl::NW, NS = Tl::NS, SLAB = Tl::SLAB, UNIT = Tl::UNIT, STAGE = Tl::STAGE;
+  constexpr int EPL = Tl::EPL, LPR = Tl::LPR, RPW = Tl::RPW, CR = Tl::CR, NV = Tl::NV;
+  constexpr int DUP = LPR / NV;  // lanes of a group holding the same row's score
 
   const int part = blockIdx.x;
   const int h = blockIdx.y;
   const int i = blockIdx.z;
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
+  const int g = lane / LPR;   // row group
+  const int pl = lane % LPR;  // position in the row: elements pl * 8 .. pl * 8 + 7
 
   int L = __ldg(p.seq_lens + i);
   const bool len_ok = L >= 0 && L <= p.L_cap;
@@ -146,7 +161,8 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
   }
   __syncthreads();
 
-  // This partition's blocks, split into NW contiguous runs.
+  // This partition's blocks, split into NW contiguous runs; a warp's tokens are
+  // [wb * S, min(we * S, L)), taken CR at a time (units; none is wholly past L).
   const int t_beg = part * p.P;
   const int t_end = min(t_beg + p.P, L);
   const int blk_beg = t_beg / S;
@@ -154,65 +170,71 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
   const int nb = blk_end - blk_beg;
   const int wb = blk_beg + static_cast<int>((static_cast<int64_t>(nb) * w) / NW);
   const int we = blk_beg + static_cast<int>((static_cast<int64_t>(nb) * (w + 1)) / NW);
-  const int nbw = we - wb;
+  const int wt0 = wb * S;
+  const int wt1 = min(we * S, L);
+  const int nunits = wt1 > wt0 ? (wt1 - wt0 + CR - 1) / CR : 0;
 
-  // q, pre-scaled so that scores come out in base-2 units.
-  float qf[DL];
+  // q fragment, pre-scaled so that scores come out in base-2 units.
+  float qf[EPL];
   {
-    const T* qp = static_cast<const T*>(p.q) + (static_cast<int64_t>(i) * p.H + h) * D + lane * DL;
-    load_row<T, DL>(qp, qf);
+    const T* qp = static_cast<const T*>(p.q) + (static_cast<int64_t>(i) * p.H + h) * D + pl * EPL;
+    load_row<T, EPL>(qp, qf);
 #pragma unroll
-    for (int e = 0; e < DL; ++e) qf[e] *= p.q_scale;
+    for (int e = 0; e < EPL; ++e) qf[e] *= p.q_scale;
   }
 
   uint64_t* bar = bars + w * NS;
   uint8_t* stage0 = smem + w * NS * STAGE;
   const int32_t* trow = p.block_tables + static_cast<int64_t>(i) * p.MB;
-  const uint8_t* kbase =
-      static_cast<const uint8_t*>(p.k_cache) + static_cast<int64_t>(h) * SLAB;
-  const uint8_t* vbase =
-      static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(h) * SLAB;
+  const uint8_t* kbase = static_cast<const uint8_t*>(p.k_cache) + static_cast<int64_t>(h) * SLAB;
+  const uint8_t* vbase = static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(h) * SLAB;
   const int64_t block_stride = static_cast<int64_t>(p.H) * SLAB;  // bytes per physical block
   const uint64_t policy = policy_evict_first();
 
-  // Fused append: does this warp own the new token's block?
+  // Fused append: does this warp own the new token?
   const int t_new = L - 1;
   // (a clamped, out-of-range length appends nothing: its position is unknown)
-  const bool appender = APPEND && len_ok && L >= 1 && t_new / S >= wb && t_new / S < we;
-  RawRow<DL> k_row, v_row;
+  const bool appender = APPEND && len_ok && L >= 1 && t_new >= wt0 && t_new < wt1;
+  RawFrag k_row, v_row;
   int id_new = -1;
-  if (appender) {
-    const int64_t off = ((static_cast<int64_t>(i) * p.H + h) * D + lane * DL) * 2;
+  if (appender && g == 0) {
+    const int64_t off = ((static_cast<int64_t>(i) * p.H + h) * D + pl * EPL) * 2;
     k_row.load(static_cast<const uint8_t*>(p.k_new) + off);
     v_row.load(static_cast<const uint8_t*>(p.v_new) + off);
     id_new = __ldg(trow + t_new / S);
   }
 
-  // Block-id prefetch: ids_a holds the chunk of 32 being issued, ids_b the next.
+  // Block-id prefetch: ids_a holds the table entries of blocks wb + base .. +31,
+  // ids_b the next 32.
+  int base = 0;
   int ids_a = (wb + lane < we) ? __ldg(trow + wb + lane) : -1;
   int ids_b = (wb + 32 + lane < we) ? __ldg(trow + wb + 32 + lane) : -1;
-  uint32_t bad = 0;  // bit s: stage s holds a block whose id was out of range
+  uint32_t bad = 0;  // bit s: stage s holds a unit whose block id was out of range
   int issued = 0;
 
   auto issue_next = [&]() {
-    if (issued >= nbw) return;
-    if ((issued & 31) == 0 && issued > 0) {
+    if (issued >= nunits) return;
+    const int t0 = wt0 + issued * CR;       // first token of the unit
+    const int rb = t0 / S - wb;             // block, relative to the warp's run
+    if (rb >= base + 32) {
+      base += 32;
       ids_a = ids_b;
-      const int nx = wb + issued + 32 + lane;
+      const int nx = wb + base + 32 + lane;
       ids_b = nx < we ? __ldg(trow + nx) : -1;
     }
-    const int id = __shfl_sync(kFullMask, ids_a, issued & 31);
+    const int id = __shfl_sync(kFullMask, ids_a, rb - base);
     const int s = issued % NS;
     const bool ok = static_cast<unsigned>(id) < static_cast<unsigned>(p.NB);
     if (lane == 0) {
       if (ok) {
-        mbar_arrive_expect_tx(&bar[s], 2 * SLAB);
-        const int64_t off = static_cast<int64_t>(id) * block_stride;
-        bulk_g2s(stage0 + s * STAGE, kbase + off, SLAB, &bar[s], policy);
-        bulk_g2s(stage0 + s * STAGE + SLAB, vbase + off, SLAB, &bar[s], policy);
+        mbar_arrive_expect_tx(&bar[s], 2 * UNIT);
+        const int64_t off = static_cast<int64_t>(id) * block_stride +
+                            static_cast<int64_t>(t0 % S) * D * 2;
+        bulk_g2s(stage0 + s * STAGE, kbase + off, UNIT, &bar[s], policy);
+        bulk_g2s(stage0 + s * STAGE + UNIT, vbase + off, UNIT, &bar[s], policy);
       } else {
         raise_error(PA_DEVERR_BLOCK_ID);
-        mbar_arrive(&bar[s]);  // completes the phase with no data; the block is skipped
+        mbar_arrive(&bar[s]);  // completes the phase with no data; the unit is skipped
       }
     }
     bad = ok ? (bad & ~(1u << s)) : (bad | (1u << s));
@@ -223,13 +245,13 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
   for (int k = 0; k < NS; ++k) issue_next();
 
   float m = -INFINITY;  // running max (base-2 units), warp-uniform
-  float lsum = 0.f;     // running sum of 2^(s - m); counted once per token
-  float acc[DL];
+  float lsum = 0.f;     // running sum of 2^(s - m); one lane per row counts it
+  float acc[EPL];       // this lane's fragment, over the rows of its group
 #pragma unroll
-  for (int e = 0; e < DL; ++e) acc[e] = 0.f;
-  const int tok = lane / DUP;
+  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+  const int my_row = (pl / DUP) * RPW + g;  // the row whose score this lane ends with
 
-  for (int k = 0; k < nbw; ++k) {
+  for (int k = 0; k < nunits; ++k) {
     const int s = k % NS;
     if (!mbar_wait_bounded(&bar[s], (k / NS) & 1)) {
       if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
@@ -238,37 +260,40 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
       break;
     }
     if (!((bad >> s) & 1u)) {
-      const int j = wb + k;
-      const int nvalid = min(S, L - j * S);
-      const uint8_t* ks = stage0 + s * STAGE;
-      const uint8_t* vs = ks + SLAB;
-      if (APPEND && appender && j == t_new / S) {
-        // the bulk copy brought the block's old bytes; put the new token's row
-        // in both the staged slabs and the cache
-        const int64_t row_off = (static_cast<int64_t>(t_new % S) * D + lane * DL) * 2;
-        k_row.store(stage0 + s * STAGE + row_off);
-        v_row.store(stage0 + s * STAGE + SLAB + row_off);
-        const int64_t goff = static_cast<int64_t>(id_new) * block_stride + row_off;
-        k_row.store(const_cast<uint8_t*>(kbase) + goff);
-        v_row.store(const_cast<uint8_t*>(vbase) + goff);
-        // these generic-proxy writes must be ordered before the next bulk copy
-        // (async proxy) that reuses this stage
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const int t0 = wt0 + k * CR;
+      const int nvalid = min(CR, L - t0);
+      uint8_t* ks = stage0 + s * STAGE;
+      uint8_t* vs = ks + UNIT;
+      if (APPEND && appender && t_new >= t0 && t_new < t0 + CR) {
+        // the bulk copy brought the old bytes; put the new token's row in both
+        // the staged unit and the cache
+        if (g == 0) {
+          const int64_t row_off = (static_cast<int64_t>(t_new - t0) * D + pl * EPL) * 2;
+          k_row.store(ks + row_off);
+          v_row.store(vs + row_off);
+          const int64_t goff = static_cast<int64_t>(id_new) * block_stride +
+                               (static_cast<int64_t>(t_new % S) * D + pl * EPL) * 2;
+          k_row.store(const_cast<uint8_t*>(kbase) + goff);
+          v_row.store(const_cast<uint8_t*>(vbase) + goff);
+          // these generic-proxy writes must be ordered before the next bulk
+          // copy (async proxy) that reuses this stage
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
         __syncwarp();
       }
 
-      float part_dot[S];
+      float dot[NV];
 #pragma unroll
-      for (int t = 0; t < S; ++t) {
-        float kf[DL];
-        load_row<T, DL>(ks + (t * D + lane * DL) * 2, kf);
+      for (int v = 0; v < NV; ++v) {
+        float kf[EPL];
+        load_row<T, EPL>(ks + ((v * RPW + g) * D + pl * EPL) * 2, kf);
         float a = 0.f;
 #pragma unroll
-        for (int e = 0; e < DL; ++e) a = fmaf(qf[e], kf[e], a);
-        part_dot[t] = a;
+        for (int e = 0; e < EPL; ++e) a = fmaf(qf[e], kf[e], a);
+        dot[v] = a;
       }
-      const float score = transpose_reduce<S>(part_dot, lane);
-      const bool valid = tok < nvalid;
+      const float score = transpose_reduce<NV, LPR>(dot, lane);
+      const bool valid = my_row < nvalid;
       const float sc = valid ? score : -INFINITY;
       float mb = sc;
 #pragma unroll
@@ -276,17 +301,31 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
       const float m_new = fmaxf(m, mb);
       const float alpha = exp2f(m - m_new);
       const float pr = valid ? exp2f(sc - m_new) : 0.f;
-      lsum = lsum * alpha + ((lane % DUP) == 0 ? pr : 0.f);
+      lsum = lsum * alpha + ((pl % DUP) == 0 ? pr : 0.f);
 #pragma unroll
-      for (int e = 0; e < DL; ++e) acc[e] *= alpha;
+      for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
+      if (nvalid == CR) {
 #pragma unroll
-      for (int t = 0; t < S; ++t) {
-        if (t < nvalid) {  // warp-uniform
-          const float pt = __shfl_sync(kFullMask, pr, t * DUP);
-          float vf[DL];
-          load_row<T, DL>(vs + (t * D + lane * DL) * 2, vf);
+        for (int v = 0; v < NV; ++v) {
+          const float pv = __shfl_sync(kFullMask, pr, g * LPR + v * DUP);
+          float vf[EPL];
+          load_row<T, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * 2, vf);
 #pragma unroll
-          for (int e = 0; e < DL; ++e) acc[e] = fmaf(pt, vf[e], acc[e]);
+          for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pv, vf[e], acc[e]);
+        }
+      } else {
+        // the request's last unit: rows past nvalid may hold anything (NaN);
+        // they are left out by selection, never multiplied by zero
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          if (v * RPW < nvalid) {  // warp-uniform
+            const float pv = __shfl_sync(kFullMask, pr, g * LPR + v * DUP);
+            const bool row_ok = v * RPW + g < nvalid;
+            float vf[EPL];
+            load_row<T, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * 2, vf);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] = row_ok ? fmaf(pv, vf[e], acc[e]) : acc[e];
+          }
         }
       }
       m = m_new;
@@ -297,13 +336,21 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
 
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, off);
+  // the row groups accumulated disjoint rows of the same fragment: add them up
+#pragma unroll
+  for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] += __shfl_xor_sync(kFullMask, acc[e], off);
+  }
 
   // Merge the NW warps' (m, l, acc) in shared memory.
   float* m_s = merge;
   float* l_s = merge + NW;
   float* acc_s = merge + 2 * NW;
+  if (g == 0) {
 #pragma unroll
-  for (int e = 0; e < DL; ++e) acc_s[w * D + lane * DL + e] = acc[e];
+    for (int e = 0; e < EPL; ++e) acc_s[w * D + pl * EPL + e] = acc[e];
+  }
   if (lane == 0) {
     m_s[w] = m;
     l_s[w] = lsum;

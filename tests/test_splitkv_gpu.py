@@ -64,7 +64,8 @@ def test_long_context_reduced():
     """Long-context shape (32 heads, head_dim 128, bf16) at lengths 32K-40K, 2 requests."""
     case = workloads.long_context_decode(seed=1, device=DEV, batch=2, lo=32768, hi=40000, H=4)
     out, _ = run_decode(case)
-    assert binding.pa_decode_plan(2, 4, 128, 16, max(case.seq_lens_host))[0] == 512
+    P, NP = binding.pa_decode_plan(2, 4, 128, 16, max(case.seq_lens_host))
+    assert NP > 1 and P % 16 == 0  # split (a small grid gets partitions below 512 tokens)
     assert_parity(out.cpu().numpy(), oracle_full(case), "long context reduced")
 
 
