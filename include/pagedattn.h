@@ -213,6 +213,34 @@ pa_status pa_seq_len(const pa_alloc* a, int64_t seq_id, int* len);
  * its length. PA_ERR_OUT_OF_RANGE if cap is too small (nothing copied). */
 pa_status pa_seq_block_table(const pa_alloc* a, int64_t seq_id, int32_t* dst, int cap, int* n);
 
+/* Prefix sharing ([vllm] Step 9 "Safe Sharing with Copy-on-Write"): child
+ * starts as parent's copy (same length, same physical blocks, every block's
+ * reference count + 1). Blocks return to the pool when their count reaches 0.
+ * When a sequence grows past its length while its last block is partly filled
+ * and named by another table too, pa_seq_grow / pa_prepare_step first give it
+ * a private block: a free block is taken, the (shared, private) pair is queued,
+ * the sequence's table entry is repointed; the other tables keep the original.
+ * The caller must copy the queued pairs on the device (pa_copy_blocks) before
+ * the append that writes the new token. PA_ERR_INVALID if parent is unknown or
+ * child exists. */
+pa_status pa_seq_fork(pa_alloc* a, int64_t parent, int64_t child);
+
+/* Moves the queued copy-on-write pairs, oldest first, into src_dst [cap, 2]
+ * (int32: source block, destination block) and clears the queue; *n receives
+ * the count. PA_ERR_OUT_OF_RANGE (nothing taken) if cap is too small. */
+pa_status pa_alloc_take_copies(pa_alloc* a, int32_t* src_dst, int cap, int* n);
+
+/* Copies the reference count of every block into dst[0..NB) (0 = free). */
+pa_status pa_alloc_refcounts(const pa_alloc* a, int32_t* dst, int cap);
+
+/* Device half of copy-on-write: for each of the n pairs in src_dst (device
+ * int32 [n, 2]), copies physical block src to block dst in both caches, every
+ * head, bit for bit. Destinations must be distinct and not sources of other
+ * pairs. Ids outside [0, NB) are skipped and flagged (PA_DEVERR_BLOCK_ID).
+ * Requires D % 8 == 0 and 16-byte aligned caches. */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst, int n, int H,
+                         int S, int D, int NB, pa_dtype dt, void* stream);
+
 /* Host slot mapping: for each sequence k, tokens start_pos[k] .. start_pos[k]
  * + n_tok[k] - 1 are written to dst in order, as table[pos / S] * S + pos % S.
  * dst holds sum(n_tok) entries. PA_ERR_OUT_OF_RANGE if a position is not yet
@@ -234,7 +262,8 @@ pa_status pa_prepare_step(pa_alloc* a, const int64_t* seq_ids, int n_seq, int n_
                           int64_t* dst_slots, int32_t* dst_tables, int32_t* dst_lens);
 
 /* Pool statistics: free blocks, tokens held (sum of lengths) and empty slots in
- * held blocks (the tail waste of [vllm] Step 5 "Why Waste Stays Below 4%"). */
+ * held blocks (the tail waste of [vllm] Step 5 "Why Waste Stays Below 4%"),
+ * counted per sequence (a shared block counts once per table naming it). */
 pa_status pa_alloc_stats(const pa_alloc* a, int* free_blocks, int64_t* used_slots,
                          int64_t* wasted_slots);
 

@@ -14,6 +14,13 @@ follows the pages' account of on-demand allocation:
 * on completion the request's blocks go back to the pool, immediately reusable
   (Step 7, item 7; Step 8 "Continuous Batching in vLLM").
 
+* prefix sharing ("vLLM KV Cache and PagedAttention Explained", Step 9 "Safe
+  Sharing with Copy-on-Write"): a block may be named by several requests' tables
+  and keeps a reference count; it returns to the pool when the count drops to
+  zero; a request that is about to write into a block others also name first
+  gets its own copy of that block (the copy is queued for the device) and its
+  table entry is repointed, the others keep the original.
+
 Readings where the pages are silent (listed in the design notes): the free list
 is a LIFO stack; ``initial_order`` lists the ids in the order they are first
 handed out (identity when omitted); growth pops ids one at a time and appends
@@ -42,9 +49,19 @@ class BlockPoolModel:
         self.free = order[::-1]  # top of the stack = end of the list = next id handed out
         self.tables = {}
         self.lens = {}
+        self.refs = [0] * num_blocks   # how many tables name each block
+        self.copies = []               # pending (src, dst) block copies from copy-on-write
 
     def blocks_needed(self, n_tokens):
         return -(-n_tokens // self.block_size)
+
+    def _cow_needed(self, seq_id, new_len):
+        """Growing past the current length writes into the last block if it is
+        partly filled; if other tables also name it, it must be copied first."""
+        table = self.tables.get(seq_id, [])
+        cur = self.lens.get(seq_id, 0)
+        return (new_len > cur and cur % self.block_size != 0 and table
+                and self.refs[table[-1]] > 1)
 
     def grow(self, seq_id, new_len):
         if new_len < 0:
@@ -53,19 +70,45 @@ class BlockPoolModel:
         cur = self.lens.get(seq_id, 0)
         if new_len < cur:
             raise PoolError(INVALID, "a sequence cannot shrink")
-        need = self.blocks_needed(new_len) - len(table)
+        cow = self._cow_needed(seq_id, new_len)
+        need = self.blocks_needed(new_len) - len(table) + (1 if cow else 0)
         if need > len(self.free):
             raise PoolError(OOM, "pool exhausted")
         table = list(table)
-        for _ in range(need):
-            table.append(self.free.pop())
+        if cow:
+            src = table[-1]
+            dst = self.free.pop()
+            self.refs[src] -= 1
+            self.refs[dst] = 1
+            table[-1] = dst
+            self.copies.append((src, dst))
+        for _ in range(self.blocks_needed(new_len) - len(table)):
+            b = self.free.pop()
+            self.refs[b] = 1
+            table.append(b)
         self.tables[seq_id] = table
         self.lens[seq_id] = new_len
+
+    def fork(self, parent, child):
+        """child starts as a copy of parent's table and length; every block is shared."""
+        if parent not in self.tables or child in self.tables:
+            raise PoolError(INVALID, "unknown parent or existing child")
+        self.tables[child] = list(self.tables[parent])
+        self.lens[child] = self.lens[parent]
+        for b in self.tables[child]:
+            self.refs[b] += 1
+
+    def take_copies(self):
+        out, self.copies = self.copies, []
+        return out
 
     def release(self, seq_id):
         if seq_id not in self.tables:
             raise PoolError(INVALID, "unknown sequence")
-        self.free.extend(self.tables.pop(seq_id))
+        for b in self.tables.pop(seq_id):
+            self.refs[b] -= 1
+            if self.refs[b] == 0:
+                self.free.append(b)
         del self.lens[seq_id]
 
     def block_table(self, seq_id):

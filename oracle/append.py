@@ -42,3 +42,12 @@ def kv_append(k, v, slot_mapping, k_cache, v_cache):
     slots = np.asarray(torch.as_tensor(slot_mapping).to("cpu").numpy(), dtype=np.int64)
     scatter_into(_bits(k), _bits(v), slots, kc, vc)
     return kc, vc
+
+
+def copy_blocks_into(kc_bits, vc_bits, pairs):
+    """Copy-on-write, device half ("vLLM KV Cache and PagedAttention Explained",
+    Step 9): physical block dst becomes a bit copy of block src, every head, in
+    both caches, for each (src, dst) pair in order. In place on uint16 arrays."""
+    for src, dst in pairs:
+        kc_bits[dst] = kc_bits[src]
+        vc_bits[dst] = vc_bits[src]

@@ -52,6 +52,10 @@ _SIGNATURES = {
     "pa_build_block_tables": ([_vp, _vp, _i32, _i32, _vp], _i32),
     "pa_prepare_step": ([_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp], _i32),
     "pa_alloc_stats": ([_vp, _vp, _vp, _vp], _i32),
+    "pa_seq_fork": ([_vp, _i64, _i64], _i32),
+    "pa_alloc_take_copies": ([_vp, _vp, _i32, _vp], _i32),
+    "pa_alloc_refcounts": ([_vp, _vp, _i32], _i32),
+    "pa_copy_blocks": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "pa_alloc_dump": ([_vp, _vp, _i32, _vp], _i32),
 }
 
@@ -202,6 +206,18 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, m
 PA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
+def pa_copy_blocks(k_cache, v_cache, src_dst, stream=None):
+    """Copies physical blocks src -> dst (device int32 [n, 2]) in both caches."""
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache), ("src_dst", src_dst)):
+        _cuda(t, n)
+    if src_dst.dtype != torch.int32:
+        raise ValueError("src_dst must be int32")
+    NB, H, S, D = k_cache.shape
+    n = src_dst.shape[0] if src_dst.numel() else 0
+    _check(lib().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(src_dst), n, H, S, D, NB,
+                                _DT[k_cache.dtype], _stream(stream)), "pa_copy_blocks")
+
+
 def pa_get_device_error(stream=None):
     """Synchronises the stream, then reads and clears the device error word."""
     flags = ctypes.c_uint32()
@@ -292,6 +308,23 @@ class BlockAllocator:
         _check(lib().pa_alloc_stats(self._h, ctypes.byref(f), ctypes.byref(u), ctypes.byref(w)),
                "pa_alloc_stats")
         return f.value, u.value, w.value
+
+    def pa_seq_fork(self, parent, child):
+        _check(lib().pa_seq_fork(self._h, int(parent), int(child)), "pa_seq_fork")
+
+    def pa_alloc_take_copies(self):
+        """The queued copy-on-write pairs as a CPU int32 tensor [n, 2] (queue cleared)."""
+        n = ctypes.c_int()
+        cap = self.num_blocks
+        out = torch.empty((max(cap, 1), 2), dtype=torch.int32)
+        _check(lib().pa_alloc_take_copies(self._h, _ptr(out), cap, ctypes.byref(n)),
+               "pa_alloc_take_copies")
+        return out[:n.value].clone()
+
+    def pa_alloc_refcounts(self):
+        out = torch.empty(max(self.num_blocks, 1), dtype=torch.int32)
+        _check(lib().pa_alloc_refcounts(self._h, _ptr(out), self.num_blocks), "pa_alloc_refcounts")
+        return out[:self.num_blocks].tolist()
 
     def pa_alloc_dump(self):
         n = ctypes.c_int()

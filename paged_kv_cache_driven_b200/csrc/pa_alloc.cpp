@@ -9,9 +9,18 @@
 // "무엇이 좋아지는가": on-demand allocation, waste bounded by each request's
 // last block.
 //
+// Step 9 "Safe Sharing with Copy-on-Write": a block can be named by several
+// tables (a shared prompt prefix, or the prompt of parallel samples forked from
+// one request); each block keeps a reference count and goes back to the pool
+// when it drops to zero. A sequence about to write into a partly filled block
+// that other tables also name first gets a private copy: a new block is taken,
+// the (old, new) pair is queued for pa_copy_blocks, and only this sequence's
+// table entry changes.
+//
 // State: a LIFO free list (std::vector used as a stack; back() is handed out
-// next) and a hash map from sequence id to {length, block table}. Every call is
-// O(work it reports) and validates its arguments before changing anything.
+// next), a reference count per block, a hash map from sequence id to {length,
+// block table}, and the queue of pending copies. Every call is O(work it
+// reports) and validates its arguments before changing anything.
 
 #include <algorithm>
 #include <cstdint>
@@ -30,9 +39,34 @@ struct pa_alloc {
   int num_blocks = 0;
   int block_size = 0;
   std::vector<int32_t> free_list;
+  std::vector<int32_t> refs;                       // tables naming each block
+  std::vector<std::pair<int32_t, int32_t>> copies;  // pending copy-on-write (src, dst)
   std::unordered_map<int64_t, Seq> seqs;
 
   int64_t blocks_for(int64_t len) const { return (len + block_size - 1) / block_size; }
+
+  // Growing seq s past its length writes into its last block when that block
+  // is partly filled; a block other tables also name must be copied first.
+  bool cow_needed(const Seq& s, int64_t new_len) const {
+    return new_len > s.len && s.len % block_size != 0 && !s.blocks.empty() &&
+           refs[static_cast<size_t>(s.blocks.back())] > 1;
+  }
+
+  int32_t pop_block() {
+    const int32_t b = free_list.back();
+    free_list.pop_back();
+    refs[static_cast<size_t>(b)] = 1;
+    return b;
+  }
+
+  // Gives s a private copy of its last block (free list known to be non-empty).
+  void copy_on_write(Seq& s) {
+    const int32_t src = s.blocks.back();
+    const int32_t dst = pop_block();
+    --refs[static_cast<size_t>(src)];
+    s.blocks.back() = dst;
+    copies.emplace_back(src, dst);
+  }
 };
 
 namespace {
@@ -54,6 +88,8 @@ pa_status pa_alloc_create(int NB, int S, const int32_t* initial_order, pa_alloc*
   a->num_blocks = NB;
   a->block_size = S;
   try {
+    a->refs.assign(static_cast<size_t>(NB), 0);
+    a->copies.reserve(64);
     a->free_list.resize(static_cast<size_t>(NB));
     if (initial_order) {
       std::vector<uint8_t> seen(static_cast<size_t>(NB), 0);
@@ -85,15 +121,15 @@ pa_status pa_seq_grow(pa_alloc* a, int64_t seq_id, int new_len) {
   const int cur_len = it == a->seqs.end() ? 0 : it->second.len;
   const size_t cur_blocks = it == a->seqs.end() ? 0 : it->second.blocks.size();
   if (new_len < cur_len) return PA_ERR_INVALID;
-  const int64_t need = a->blocks_for(new_len) - static_cast<int64_t>(cur_blocks);
-  if (need > static_cast<int64_t>(a->free_list.size())) return PA_ERR_OOM;
+  const bool cow = it != a->seqs.end() && a->cow_needed(it->second, new_len);
+  const int64_t grow = a->blocks_for(new_len) - static_cast<int64_t>(cur_blocks);
+  if (grow + (cow ? 1 : 0) > static_cast<int64_t>(a->free_list.size())) return PA_ERR_OOM;
   try {
     pa_alloc::Seq& s = a->seqs[seq_id];  // may create
-    s.blocks.reserve(s.blocks.size() + static_cast<size_t>(need));
-    for (int64_t k = 0; k < need; ++k) {
-      s.blocks.push_back(a->free_list.back());
-      a->free_list.pop_back();
-    }
+    s.blocks.reserve(s.blocks.size() + static_cast<size_t>(grow));
+    a->copies.reserve(a->copies.size() + 1);
+    if (cow) a->copy_on_write(s);
+    for (int64_t k = 0; k < grow; ++k) s.blocks.push_back(a->pop_block());
     s.len = new_len;
   } catch (...) {
     return PA_ERR_OOM;  // only reachable on host allocation failure before any pop
@@ -106,8 +142,41 @@ pa_status pa_seq_free(pa_alloc* a, int64_t seq_id) {
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PA_ERR_INVALID;
   // capacity was reserved for the whole pool at creation, so this cannot throw
-  for (int32_t b : it->second.blocks) a->free_list.push_back(b);
+  for (int32_t b : it->second.blocks)
+    if (--a->refs[static_cast<size_t>(b)] == 0) a->free_list.push_back(b);
   a->seqs.erase(it);
+  return PA_OK;
+}
+
+pa_status pa_seq_fork(pa_alloc* a, int64_t parent, int64_t child) {
+  if (!a) return PA_ERR_INVALID;
+  auto it = a->seqs.find(parent);
+  if (it == a->seqs.end() || a->seqs.count(child)) return PA_ERR_INVALID;
+  try {
+    pa_alloc::Seq copy = it->second;
+    for (int32_t b : copy.blocks) ++a->refs[static_cast<size_t>(b)];
+    a->seqs.emplace(child, std::move(copy));
+  } catch (...) {
+    return PA_ERR_OOM;
+  }
+  return PA_OK;
+}
+
+pa_status pa_alloc_take_copies(pa_alloc* a, int32_t* src_dst, int cap, int* n) {
+  if (!a || !n || cap < 0 || (cap > 0 && !src_dst)) return PA_ERR_INVALID;
+  *n = static_cast<int>(a->copies.size());
+  if (*n > cap) return PA_ERR_OUT_OF_RANGE;  // nothing taken
+  for (int k = 0; k < *n; ++k) {
+    src_dst[2 * k] = a->copies[static_cast<size_t>(k)].first;
+    src_dst[2 * k + 1] = a->copies[static_cast<size_t>(k)].second;
+  }
+  a->copies.clear();
+  return PA_OK;
+}
+
+pa_status pa_alloc_refcounts(const pa_alloc* a, int32_t* dst, int cap) {
+  if (!a || !dst || cap < a->num_blocks) return PA_ERR_INVALID;
+  if (a->num_blocks) std::memcpy(dst, a->refs.data(), sizeof(int32_t) * a->refs.size());
   return PA_OK;
 }
 
@@ -187,18 +256,21 @@ pa_status pa_prepare_step(pa_alloc* a, const int64_t* seq_ids, int n_seq, int n_
     if (new_len > INT32_MAX) return PA_ERR_INVALID;
     const int64_t nb = a->blocks_for(new_len);
     if (dst_tables && nb > MB) return PA_ERR_OUT_OF_RANGE;
-    need += nb - static_cast<int64_t>(s->blocks.size());
+    need += nb - static_cast<int64_t>(s->blocks.size()) + (a->cow_needed(*s, new_len) ? 1 : 0);
   }
   if (need > static_cast<int64_t>(a->free_list.size())) return PA_ERR_OOM;
+  try {
+    a->copies.reserve(a->copies.size() + static_cast<size_t>(n_seq));
+  } catch (...) {
+    return PA_ERR_OOM;
+  }
   for (int k = 0; k < n_seq; ++k) {
     pa_alloc::Seq& s = a->seqs.find(seq_ids[k])->second;
     const int old_len = s.len;
     const int new_len = old_len + n_new;
+    if (a->cow_needed(s, new_len)) a->copy_on_write(s);
     const int64_t add = a->blocks_for(new_len) - static_cast<int64_t>(s.blocks.size());
-    for (int64_t j = 0; j < add; ++j) {
-      s.blocks.push_back(a->free_list.back());
-      a->free_list.pop_back();
-    }
+    for (int64_t j = 0; j < add; ++j) s.blocks.push_back(a->pop_block());
     s.len = new_len;
     const int64_t S = a->block_size;
     if (dst_slots)

@@ -175,6 +175,23 @@ pa_status pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping
   return cuda_status();
 }
 
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst, int n, int H,
+                         int S, int D, int NB, pa_dtype dt, void* stream) {
+  if (n < 0 || H <= 0 || S <= 0 || D <= 0 || NB < 0 || !cache_dtype_ok(dt) || D % 8 != 0)
+    return PA_ERR_INVALID;
+  if (n == 0) return PA_OK;
+  if (!k_cache || !v_cache || !src_dst || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  const int64_t vpb = static_cast<int64_t>(H) * S * D / 8;  // 16-byte vectors per block
+  const int64_t total = vpb * n;
+  int64_t blocks = ceil_div(total, 256);
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  pa::copy_blocks_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                           static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), src_dst, total, vpb, NB);
+  return cuda_status();
+}
+
 pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partition,
                          int* partition_tokens, int* num_partitions) {
   (void)B;

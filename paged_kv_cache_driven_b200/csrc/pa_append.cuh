@@ -44,4 +44,30 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Copy-on-write, device half ("vLLM KV Cache and PagedAttention Explained",
+// Step 9): copies whole physical blocks, every head, of K and V from src to
+// dst for each (src, dst) pair. One thread per 16-byte vector; the pairs come
+// from the allocator's queue and name distinct destinations.
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                       const int32_t* __restrict__ src_dst, int64_t total, int64_t vec_per_block,
+                       int NB) {
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t pair = idx / vec_per_block;
+    const int64_t c = idx - pair * vec_per_block;
+    const int32_t src = __ldg(src_dst + 2 * pair);
+    const int32_t dst = __ldg(src_dst + 2 * pair + 1);
+    if (static_cast<unsigned>(src) >= static_cast<unsigned>(NB) ||
+        static_cast<unsigned>(dst) >= static_cast<unsigned>(NB)) {
+      if (c == 0) raise_error(PA_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const uint4 kv = k_cache[src * vec_per_block + c];
+    const uint4 vv = v_cache[src * vec_per_block + c];
+    k_cache[dst * vec_per_block + c] = kv;
+    v_cache[dst * vec_per_block + c] = vv;
+  }
+}
+
 }  // namespace pa

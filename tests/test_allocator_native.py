@@ -142,3 +142,116 @@ def test_random_walk_bit_exact(seed):
                 ns = [rng.randint(0, live[s] - p) for s, p in zip(ids, starts)]
                 assert a.pa_build_slot_mapping(ids, starts, ns).tolist() == \
                     m.slot_mapping(ids, starts, ns)
+
+
+def same_sharing_state(native, model):
+    assert native.pa_alloc_refcounts() == model.refs
+    got = native.pa_alloc_take_copies().tolist()
+    assert [tuple(x) for x in got] == model.take_copies()
+
+
+def test_copy_on_write_page_example_native():
+    order = [5, 40, 41] + [b for b in range(100) if b not in (5, 40, 41)]
+    a = BlockAllocator(100, 16, initial_order=order)
+    m = BlockPoolModel(100, 16, initial_order=order)
+    for x in (a, m):
+        (x.pa_seq_grow if x is a else x.grow)(0, 8)
+    for r in (1, 2, 3):
+        a.pa_seq_fork(0, r)
+        m.fork(0, r)
+    a.pa_seq_free(0)
+    m.release(0)
+    assert a.pa_alloc_refcounts()[5] == 3
+    a.pa_seq_grow(1, 9)
+    m.grow(1, 9)
+    assert a.pa_seq_block_table(1) == [40] and a.pa_seq_block_table(2) == [5]
+    same_sharing_state(a, m)
+    same_state(a, m, [1, 2, 3])
+    with pytest.raises(PagedAttnError) as e:
+        a.pa_seq_fork(99, 7)
+    assert e.value.code == binding.PA_ERR_INVALID
+    with pytest.raises(PagedAttnError) as e:
+        a.pa_seq_fork(1, 2)
+    assert e.value.code == binding.PA_ERR_INVALID
+
+
+@pytest.mark.parametrize("seed", [3, 4, 5])
+def test_random_walk_with_forks_bit_exact(seed):
+    rng = random.Random(seed)
+    S = rng.choice([8, 16, 32])
+    NB = 400
+    order = list(range(NB))
+    rng.shuffle(order)
+    a = BlockAllocator(NB, S, initial_order=order)
+    m = BlockPoolModel(NB, S, initial_order=order)
+    live = {}
+    next_id = 0
+    for step in range(1500):
+        op = rng.random()
+        if op < 0.15 and live:  # fork
+            parent = rng.choice(sorted(live))
+            child = next_id
+            next_id += 1
+            a.pa_seq_fork(parent, child)
+            m.fork(parent, child)
+            live[child] = live[parent]
+        elif op < 0.5 and live:  # grow (may copy on write)
+            sid = rng.choice(sorted(live))
+            new = live[sid] + rng.randint(1, S + 2)
+            try:
+                m.grow(sid, new)
+            except PoolError as e:
+                with pytest.raises(PagedAttnError) as ee:
+                    a.pa_seq_grow(sid, new)
+                assert ee.value.code == e.code
+            else:
+                a.pa_seq_grow(sid, new)
+                live[sid] = new
+        elif op < 0.65 and live:  # one decode step for a few sequences
+            ids = rng.sample(sorted(live), min(len(live), rng.randint(1, 5)))
+            MB = max(-(-(live[s] + 1) // S) for s in ids) + 1
+            slots = torch.empty(len(ids), dtype=torch.int64)
+            tables = torch.empty((len(ids), MB), dtype=torch.int32)
+            lens = torch.empty(len(ids), dtype=torch.int32)
+            need = sum(-(-(live[s] + 1) // S) - len(m.tables[s]) + (1 if m._cow_needed(s, live[s] + 1) else 0)
+                       for s in ids)
+            if need > len(m.free):
+                with pytest.raises(PagedAttnError):
+                    a.pa_prepare_step(ids, 1, MB, slots, tables, lens)
+            else:
+                a.pa_prepare_step(ids, 1, MB, slots, tables, lens)
+                want = []
+                for s in ids:
+                    m.grow(s, live[s] + 1)
+                    want += m.slot_mapping([s], [live[s]], [1])
+                    live[s] += 1
+                assert slots.tolist() == want
+                assert tables.tolist() == m.block_tables(ids, MB)
+        elif op < 0.8 and live:
+            sid = rng.choice(sorted(live))
+            a.pa_seq_free(sid)
+            m.release(sid)
+            del live[sid]
+        else:
+            sid = next_id
+            next_id += 1
+            L = rng.randint(0, 6 * S)
+            try:
+                m.grow(sid, L)
+            except PoolError:
+                with pytest.raises(PagedAttnError):
+                    a.pa_seq_grow(sid, L)
+            else:
+                a.pa_seq_grow(sid, L)
+                live[sid] = L
+        if step % 25 == 0:
+            same_state(a, m, live)
+            same_sharing_state(a, m)
+            # every block is free or named by a table, with the right count
+            counts = [0] * NB
+            for t in m.tables.values():
+                for b in t:
+                    counts[b] += 1
+            assert counts == m.refs
+            assert sorted(set(b for t in m.tables.values() for b in t) | set(m.dump())) == \
+                list(range(NB))

@@ -230,3 +230,94 @@ def test_pool_conservation_random_walk():
         held = [b for t in pool.tables.values() for b in t]
         assert sorted(held + pool.dump()) == list(range(NB))
         assert len(held) == sum(-(-L // S) for L in live.values())
+
+
+# ---------------------------------------------------------------------------
+# Prefix sharing and copy-on-write ("vLLM KV Cache and PagedAttention
+# Explained", Step 9 "Safe Sharing with Copy-on-Write").
+# ---------------------------------------------------------------------------
+
+def _order_first(*ids, n=100):
+    return list(ids) + [b for b in range(n) if b not in ids]
+
+
+def test_shared_prefix_block_refcount_three():
+    """A system prompt of 8 tokens in physical block 5, shared by requests A, B
+    and C: reference count 3, all three tables name block 5."""
+    pool = BlockPoolModel(100, 16, initial_order=_order_first(5))
+    pool.grow("prompt", 8)
+    assert pool.block_table("prompt") == [5]
+    for r in "ABC":
+        pool.fork("prompt", r)
+    pool.release("prompt")
+    assert pool.refs[5] == 3
+    assert [pool.block_table(r) for r in "ABC"] == [[5], [5], [5]]
+    assert 5 not in pool.dump()
+
+
+def test_page_tables_for_a_block_aligned_prefix():
+    """Step 9's tables: block 5 shared, logical block 1 private per request
+    (12, 37, 61). They arise when the shared prefix fills its block, so each
+    request's own tokens start a new block and nothing is copied."""
+    pool = BlockPoolModel(100, 16, initial_order=_order_first(5, 12, 37, 61))
+    pool.grow("prompt", 16)
+    for r in "ABC":
+        pool.fork("prompt", r)
+    pool.release("prompt")
+    for r in "ABC":
+        pool.grow(r, 17)
+    assert [pool.block_table(r) for r in "ABC"] == [[5, 12], [5, 37], [5, 61]]
+    assert pool.refs[5] == 3 and pool.take_copies() == []
+
+
+def test_copy_on_write_repoints_only_the_writer():
+    """Writing into the shared, partly filled block copies it for the writer;
+    the others keep block 5; the last holder writes in place."""
+    pool = BlockPoolModel(100, 16, initial_order=_order_first(5, 40, 41))
+    pool.grow("prompt", 8)
+    for r in "ABC":
+        pool.fork("prompt", r)
+    pool.release("prompt")
+    pool.grow("A", 9)                       # A's 9th token goes into block 5's slot 8
+    assert pool.block_table("A") == [40] and pool.take_copies() == [(5, 40)]
+    assert pool.block_table("B") == [5] and pool.block_table("C") == [5] and pool.refs[5] == 2
+    pool.grow("B", 10)
+    assert pool.block_table("B") == [41] and pool.take_copies() == [(5, 41)]
+    pool.grow("C", 9)                       # only C still names block 5: no copy
+    assert pool.block_table("C") == [5] and pool.take_copies() == [] and pool.refs[5] == 1
+    assert pool.slot_mapping(["C"], [8], [1]) == [5 * 16 + 8]
+    for r in "ABC":
+        pool.release(r)
+    assert sorted(pool.dump()) == list(range(100)) and set(pool.refs) == {0}
+
+
+def test_parallel_sampling_saves_blocks():
+    """n samples forked from one prompt hold the prompt's full blocks once."""
+    S, prompt, n, gen = 16, 1000, 8, 100
+    shared = BlockPoolModel(1000, S)
+    shared.grow("p", prompt)
+    for k in range(n):
+        shared.fork("p", k)
+    shared.release("p")
+    for k in range(n):
+        shared.grow(k, prompt + gen)
+    private = BlockPoolModel(1000, S)
+    for k in range(n):
+        private.grow(k, prompt + gen)
+    used_shared = 1000 - len(shared.free)
+    used_private = 1000 - len(private.free)
+    full_prompt_blocks = prompt // S
+    assert used_private - used_shared == (n - 1) * full_prompt_blocks
+    assert len(shared.take_copies()) == n - 1   # the partly filled prompt block, per writer but the last
+
+
+def test_cow_counts_in_oom_and_leaves_state_unchanged():
+    pool = BlockPoolModel(2, 16)
+    pool.grow("p", 8)
+    pool.fork("p", "q")
+    pool.grow("x", 16)          # the pool is now empty
+    before = (pool.dump(), dict(pool.tables), list(pool.refs))
+    with pytest.raises(PoolError) as e:
+        pool.grow("q", 9)       # needs a private copy of the shared block
+    assert e.value.code == OOM
+    assert (pool.dump(), dict(pool.tables), list(pool.refs)) == before
