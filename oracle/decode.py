@@ -32,7 +32,7 @@ def _load():
         lib = ctypes.CDLL(_build.build())
         p = ctypes.c_void_p
         i64 = ctypes.c_int64
-        lib.oracle_paged_decode.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64,
+        lib.oracle_paged_decode.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64,
                                             ctypes.c_double, ctypes.c_int, p, i64, ctypes.c_int, p]
         lib.oracle_paged_decode.restype = ctypes.c_int
         lib.oracle_partition_stats.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64,
@@ -75,15 +75,17 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs=None,
                  dtype=None):
     """fp64 attention output.
 
-    q [B, H, D]; k_cache, v_cache [NB, H, S, D] (fp16 or bf16, same dtype as q);
+    q [B, H, D]; k_cache, v_cache [NB, Hkv, S, D] (fp16 or bf16, same dtype as q),
+    Hkv dividing H: query head h reads KV head h // (H // Hkv) (grouped-query
+    attention; Hkv == H is the pages' one KV head per query head);
     block_tables [B, MB] int32; seq_lens [B] int32. ``pairs`` is an optional
     sequence of (request, head) pairs; the result is then [len(pairs), D],
     otherwise [B, H, D]. ``threads`` = 0 uses every host core. The 16-bit inputs
     may also be uint16 numpy arrays of bit patterns, with ``dtype`` naming them.
     """
     B, H, D = q.shape
-    NB, H2, S, D2 = k_cache.shape
-    if (H2, D2) != (H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
+    NB, Hkv, S, D2 = k_cache.shape
+    if D2 != D or H % Hkv != 0 or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise OracleError("shape mismatch")
     if dtype is None:
         if q.dtype != k_cache.dtype or q.dtype != v_cache.dtype:
@@ -99,7 +101,7 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs=None,
         pa = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
         n, out = pa.shape[0], np.zeros((pa.shape[0], D), np.float64)
     rc = _load().oracle_paged_decode(
-        _ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), _ptr(sl), B, H, D, S, NB, MB, float(scale),
+        _ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), _ptr(sl), B, H, Hkv, D, S, NB, MB, float(scale),
         _DTYPE_CODE[dtype], None if pa is None else _ptr(pa), n, int(threads), _ptr(out))
     if rc:
         raise OracleError(f"oracle_paged_decode returned {rc}")

@@ -25,7 +25,10 @@
 //   * token t of request i sits at physical block table[i][t / S], offset t % S;
 //   * the query attends to exactly the first seq_lens[i] cached tokens;
 //   * seq_len == 0 gives an all-zero output row;
-//   * K and V share the [NB, H, S, D] layout; as many KV heads as query heads.
+//   * K and V share the [NB, Hkv, S, D] layout. With as many KV heads as query
+//     heads (Hkv == H) this is the pages' multi-head attention; with Hkv < H
+//     (grouped-query attention, not on the pages) query head h reads KV head
+//     h / (H / Hkv), consecutive query heads sharing one KV head.
 //
 // Build: g++ -O2 -std=c++17 -shared -fPIC -pthread oracle.cpp -o liboracle.so
 
@@ -83,21 +86,23 @@ struct Problem {
   const int32_t* seq_lens;
   int64_t B, H, D, S, NB, MB;
   double scale;
-  int dtype;  // 0 = binary16, 1 = bfloat16
+  int dtype;    // 0 = binary16, 1 = bfloat16
+  int64_t Hkv;  // KV heads; query head h reads KV head h / (H / Hkv)
 };
 
 double elem(const Problem& p, const uint16_t* base, int64_t idx) {
   return p.dtype == 0 ? decode_binary16(base[idx]) : decode_bfloat16(base[idx]);
 }
 
-// Offset of element (token t, dim 0) of request i, head h, in the cache tensor.
-// Returns -1 when the block table names a block outside the pool.
+// Offset of element (token t, dim 0) of request i, query head h, in the cache
+// tensor. Returns -1 when the block table names a block outside the pool.
 int64_t token_row(const Problem& p, int64_t i, int64_t h, int64_t t) {
   const int64_t logical_block = t / p.S;
   const int64_t offset = t % p.S;
   const int64_t physical_block = p.block_tables[i * p.MB + logical_block];
   if (physical_block < 0 || physical_block >= p.NB) return -1;
-  return ((physical_block * p.H + h) * p.S + offset) * p.D;
+  const int64_t kv_head = h / (p.H / p.Hkv);
+  return ((physical_block * p.Hkv + kv_head) * p.S + offset) * p.D;
 }
 
 // Scores s_t = scale * q . K_t for tokens [t0, t1) of (i, h).
@@ -197,7 +202,8 @@ int parallel_for(int64_t n, int n_threads, Fn fn) {
 
 bool valid_problem(const Problem& p) {
   return p.q && p.k_cache && p.v_cache && p.block_tables && p.seq_lens && p.B >= 0 && p.H > 0 &&
-         p.D > 0 && p.S > 0 && p.NB >= 0 && p.MB >= 0 && (p.dtype == 0 || p.dtype == 1);
+         p.D > 0 && p.S > 0 && p.NB >= 0 && p.MB >= 0 && (p.dtype == 0 || p.dtype == 1) &&
+         p.Hkv > 0 && p.H % p.Hkv == 0;
 }
 
 }  // namespace
@@ -209,9 +215,10 @@ double oracle_decode16(uint16_t bits, int dtype) {
   return dtype == 0 ? decode_binary16(bits) : decode_bfloat16(bits);
 }
 
-// softmax(q K^T * scale) V for each (request, head) pair, in fp64.
+// softmax(q K^T * scale) V for each (request, query head) pair, in fp64.
 //   q        [B, H, D]        16-bit elements
-//   k_cache, v_cache [NB, H, S, D]
+//   k_cache, v_cache [NB, Hkv, S, D]; Hkv divides H (Hkv == H: one KV head per
+//            query head)
 //   block_tables [B, MB] int32 (entries past ceil(L/S) are never read)
 //   seq_lens [B] int32
 //   pairs    optional [n_pairs, 2] int64 (request, head); null = every pair in
@@ -220,9 +227,11 @@ double oracle_decode16(uint16_t bits, int dtype) {
 // Returns 0, 1 on a bad argument, 3 when a block id or seq_len is out of range.
 int oracle_paged_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
                         const int32_t* block_tables, const int32_t* seq_lens, int64_t B, int64_t H,
-                        int64_t D, int64_t S, int64_t NB, int64_t MB, double scale, int dtype,
-                        const int64_t* pairs, int64_t n_pairs, int n_threads, double* out) {
-  const Problem p{q, k_cache, v_cache, block_tables, seq_lens, B, H, D, S, NB, MB, scale, dtype};
+                        int64_t Hkv, int64_t D, int64_t S, int64_t NB, int64_t MB, double scale,
+                        int dtype, const int64_t* pairs, int64_t n_pairs, int n_threads,
+                        double* out) {
+  const Problem p{q, k_cache, v_cache, block_tables, seq_lens, B, H, D, S, NB, MB, scale, dtype,
+                  Hkv};
   if (!valid_problem(p) || !out) return 1;
   const int64_t n = pairs ? n_pairs : B * H;
   for (int64_t k = 0; pairs && k < n; ++k)
@@ -243,7 +252,8 @@ int oracle_partition_stats(const uint16_t* q, const uint16_t* k_cache, const uin
                            int64_t H, int64_t D, int64_t S, int64_t NB, int64_t MB, double scale,
                            int dtype, int64_t P, int64_t NP, int n_threads, double* m, double* l,
                            double* acc) {
-  const Problem p{q, k_cache, v_cache, block_tables, seq_lens, B, H, D, S, NB, MB, scale, dtype};
+  const Problem p{q, k_cache, v_cache, block_tables, seq_lens, B, H, D, S, NB, MB, scale, dtype,
+                  H};
   if (!valid_problem(p) || P <= 0 || NP < 0 || !m || !l || !acc) return 1;
   return parallel_for(B * H * NP, n_threads, [&](int64_t k) {
     const int64_t ih = k / NP;

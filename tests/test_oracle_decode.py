@@ -251,3 +251,28 @@ def test_oracle_sensitivity_to_plausible_mistakes(oracle_lib):
     sl2 = sl.clone()
     sl2[0] -= 1
     assert np.abs(oracle_decode.paged_decode(q, kc, vc, bt, sl2, 0.125) - want).max() > 4e-3
+
+
+@pytest.mark.parametrize("G", [2, 4, 8])
+def test_grouped_query_heads_equal_sdpa_with_gqa(oracle_lib, G):
+    """Grouped-query attention (query head h reads KV head h // G; not on the
+    pages): equal to torch SDPA with enable_gqa on the contiguous K/V, and to
+    the one-KV-head-per-query-head oracle on a cache with every KV head
+    repeated G times."""
+    gen = torch.Generator().manual_seed(G)
+    Hkv, D, S = 2, 64, 16
+    H = Hkv * G
+    lens = [1, 17, 40, 130]
+    ks = [torch.randn(L, Hkv, D, generator=gen).to(torch.bfloat16) for L in lens]
+    vs = [torch.randn(L, Hkv, D, generator=gen).to(torch.bfloat16) for L in lens]
+    q = torch.randn(len(lens), H, D, generator=gen).to(torch.bfloat16)
+    kc, vc, bt, sl = make_paged(ks, vs, S, 3, gen)
+    got = oracle_decode.paged_decode(q, kc, vc, bt, sl, 0.125)
+    for i in range(len(lens)):
+        want = F.scaled_dot_product_attention(
+            q[i].double().unsqueeze(1), ks[i].double().transpose(0, 1),
+            vs[i].double().transpose(0, 1), scale=0.125, enable_gqa=True).squeeze(1)
+        np.testing.assert_allclose(got[i], want.numpy(), rtol=1e-12, atol=1e-12)
+    rep = oracle_decode.paged_decode(q, kc.repeat_interleave(G, dim=1),
+                                     vc.repeat_interleave(G, dim=1), bt, sl, 0.125)
+    assert np.array_equal(got, rep)
