@@ -408,12 +408,14 @@ def run_reference(args):
 
 
 def decode_bytes_case(case):
-    """Algorithmic bytes of one pa_decode call on a workloads.DecodeCase."""
-    B, Hc, Dc = case.q.shape
-    Sc = case.k_cache.shape[2]
+    """Algorithmic bytes of one decode call on a workloads.DecodeCase: K and V of
+    every live token of every KV head, q and out of every query head, the table
+    entries read and the lengths."""
+    B, Hq, Dc = case.q.shape
+    Hkv, Sc = case.k_cache.shape[1], case.k_cache.shape[2]
     e = case.q.element_size()
-    return sum(Hc * (2 * L * Dc * e + 2 * Dc * e) + 4 * (-(-L // Sc)) for L in case.seq_lens_host) \
-        + 4 * B
+    return sum(Hkv * 2 * L * Dc * e + Hq * 2 * Dc * e + 4 * (-(-L // Sc))
+               for L in case.seq_lens_host) + 4 * B
 
 
 def time_decode_case(case, iters, warmup, partition=0):
@@ -430,8 +432,14 @@ def time_decode_case(case, iters, warmup, partition=0):
         flush.fill_(k & 0xff)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        binding.pa_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables,
-                          case.seq_lens, case.scale, maxlen, partition=partition, workspace=ws)
+        if case.k_cache.shape[1] != Hc:
+            binding.pa_decode_gqa(out, case.q, case.k_cache, case.v_cache, case.block_tables,
+                                  case.seq_lens, case.scale, maxlen, partition=partition,
+                                  workspace=ws)
+        else:
+            binding.pa_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables,
+                              case.seq_lens, case.scale, maxlen, partition=partition,
+                              workspace=ws)
         b.record()
         torch.cuda.synchronize()
         if k >= warmup:
@@ -449,6 +457,9 @@ def run_shape_workloads(args):
     if args.workload == "long_context":
         cases = [("long_context", lambda: workloads.long_context_decode(seed=args.seed,
                                                                         device=device))]
+    elif args.workload == "llama70b":
+        cases = [("llama70b_gqa_64q_8kv", lambda: workloads.llama70b_decode(seed=args.seed,
+                                                                            device=device))]
     else:
         cases = []
         for Sx in (8, 16, 32):
@@ -489,9 +500,11 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="llama13b", choices=["llama13b", "long_context", "sweep"],
+    ap.add_argument("--workload", default="llama13b",
+                    choices=["llama13b", "long_context", "sweep", "llama70b"],
                     help="llama13b: the headline step (default); the others time decode-only "
-                         "calls of the long-context and shape-sweep configurations")
+                         "calls of the long-context, shape-sweep and LLaMA-2-70B-shaped "
+                         "grouped-query configurations")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

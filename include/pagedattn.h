@@ -140,6 +140,25 @@ pa_status pa_decode_append(void* out, pa_dtype out_dt, const void* q, const void
                            int partition, int max_seq_len, void* workspace, size_t ws_bytes,
                            void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Grouped-query decode (not on the pages, which have one KV head per query
+ * head): the cache holds Hkv KV heads, [NB, Hkv, S, D]; q and out hold H query
+ * heads, H a multiple of Hkv, and query head h reads KV head h / (H / Hkv)
+ * (consecutive query heads share a KV head). When H / Hkv is even, one CTA
+ * serves up to 8 query heads of a KV head from one staged copy of each K/V
+ * unit, so every K/V byte is read from HBM once per group. k_new, v_new
+ * ([B, Hkv, D]) are optional together: when given, the step's new token is
+ * appended at position seq_lens[i] - 1 first, exactly as pa_decode_append.
+ * Everything else (dtypes, D, S, partition, workspace sized by
+ * pa_decode_workspace_bytes(B, H, ...) with H the query heads, errors) is as
+ * pa_decode. H == Hkv gives pa_decode / pa_decode_append bit for bit.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k_new,
+                        const void* v_new, void* k_cache, void* v_cache,
+                        const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
+                        int B, int H, int Hkv, int D, int S, int NB, pa_dtype dt, int partition,
+                        int max_seq_len, void* workspace, size_t ws_bytes, void* stream);
+
 /* Split-KV workspace layout, for tests that inspect the partition pass
  * (NP = number of partitions, all fp32, offsets in bytes from `workspace`):
  *   m   [B, H, NP] at 0                 max of scale * q.k * log2(e) (base-2 units)

@@ -34,6 +34,8 @@ _SIGNATURES = {
     "pa_get_device_error": ([_vp, _vp], _i32),
     "pa_decode_append": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32,
                           _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
+    "pa_decode_gqa": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32,
+                       _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_decode_noalloc": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32,
                            _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "pa_stepper_create": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
@@ -151,7 +153,9 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_l
     if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
         raise ValueError("block_tables and seq_lens must be int32")
     B, H, D = q.shape
-    NB, _, S, _ = k_cache.shape
+    NB, Hc, S, _ = k_cache.shape
+    if Hc != H:
+        raise ValueError("the cache has a different head count: use pa_decode_gqa")
     MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     if workspace is not None:
@@ -182,6 +186,33 @@ def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_l
                                   _ptr(seq_lens), float(scale), B, H, D, S, NB, _DT[q.dtype],
                                   int(partition), int(max_seq_len), _ptr(workspace), ws_bytes,
                                   _stream(stream)), "pa_decode_append")
+
+
+def pa_decode_gqa(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,
+                  k_new=None, v_new=None, partition=0, workspace=None, stream=None):
+    """Grouped-query decode: q/out [B, H, D], caches [NB, Hkv, S, D] with H a
+    multiple of Hkv; optional k_new, v_new [B, Hkv, D] appended first."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                 ("block_tables", block_tables), ("seq_lens", seq_lens)):
+        _cuda(t, n)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    B, H, D = q.shape
+    NB, Hkv, S, _ = k_cache.shape
+    if k_new is not None:
+        _cuda(k_new, "k_new")
+        _cuda(v_new, "v_new")
+        if tuple(k_new.shape) != (B, Hkv, D) or tuple(v_new.shape) != (B, Hkv, D):
+            raise ValueError("k_new, v_new must be [B, Hkv, D]")
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_decode_gqa(_ptr(out), _DT[out.dtype], _ptr(q), _ptr(k_new), _ptr(v_new),
+                               _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), MB,
+                               _ptr(seq_lens), float(scale), B, H, Hkv, D, S, NB, _DT[q.dtype],
+                               int(partition), int(max_seq_len), _ptr(workspace), ws_bytes,
+                               _stream(stream)), "pa_decode_gqa")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

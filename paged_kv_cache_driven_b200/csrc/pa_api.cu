@@ -2,6 +2,8 @@
 // planning and kernel dispatch for pa_kv_append and pa_decode, and the device
 // error word. Every check runs on the host before anything is launched.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -9,6 +11,9 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
 
 #include "pa_append.cuh"
 #include "pa_decode.cuh"
@@ -90,34 +95,134 @@ pa_status cuda_status() {
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <typename T, typename TO, int D, int S, bool APPEND>
-pa_status launch_decode(const pa::DecodeParams& prm, cudaStream_t stream) {
-  using Tl = pa::DecodeTiling<D, S>;
-  auto kern = pa::paged_decode_partition_kernel<T, TO, D, S, APPEND>;
-  // The shared-memory opt-in is a per-device property of the function.
-  static bool configured[kMaxDevices] = {};
+// The shared-memory opt-in is a per-device property of a kernel function.
+template <typename K>
+bool opt_in_smem(K kern, int bytes, bool (&configured)[kMaxDevices]) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tl::SMEM) !=
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
         cudaSuccess)
-      return PA_ERR_CUDA;
+      return false;
     configured[dev] = true;
   }
-  const dim3 grid(prm.NP, prm.H, prm.B);
-  kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
+  return true;
+}
+
+template <typename TO, int D>
+void launch_reduce(const pa::DecodeParams& prm, cudaStream_t stream) {
   if (prm.NP > 1) {
     const int64_t pairs = static_cast<int64_t>(prm.B) * prm.H;
     pa::splitkv_reduce_kernel<TO, D>
         <<<static_cast<unsigned>((pairs + 3) / 4), 128, 0, stream>>>(prm);
   }
+}
+
+// One KV head per query head (or an odd group size): the multi-head kernel,
+// each CTA reading its query head's KV head.
+template <typename T, typename TO, int D, int S, bool APPEND>
+pa_status launch_decode(const pa::DecodeParams& prm, cudaStream_t stream) {
+  using Tl = pa::DecodeTiling<D, S>;
+  auto kern = pa::paged_decode_partition_kernel<T, TO, D, S, APPEND>;
+  static bool configured[kMaxDevices] = {};
+  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
+  const dim3 grid(prm.NP, prm.H, prm.B);
+  kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
+  launch_reduce<TO, D>(prm, stream);
+  return cuda_status();
+}
+
+// ---- tensor maps of the caches, for the tiled TMA loads ---------------------
+// Each cache [NB, Hkv, S, D] is viewed as a 2-D array of NB * Hkv * S rows of D
+// elements; a box is 64 elements x min(S, 16) rows with the 128-byte swizzle.
+// Encoding goes through the driver's cuTensorMapEncodeTiled (looked up once);
+// the last few maps are kept, keyed by everything they encode, since a cache is
+// decoded over and over.
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+struct RowMapKey {
+  const void* base;
+  int64_t rows;
+  int D, box_rows, dt;
+  bool operator==(const RowMapKey& o) const {
+    return base == o.base && rows == o.rows && D == o.D && box_rows == o.box_rows && dt == o.dt;
+  }
+};
+
+bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows, pa_dtype dt) {
+  static std::mutex mu;
+  static RowMapKey keys[16];
+  static CUtensorMap maps[16];
+  static int used = 0, next = 0;
+  const RowMapKey key{base, rows, D, box_rows, static_cast<int>(dt)};
+  std::lock_guard<std::mutex> lock(mu);
+  for (int k = 0; k < used; ++k)
+    if (keys[k] == key) {
+      *out = maps[k];
+      return true;
+    }
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUtensorMap map;
+  if (fn(&map, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+         2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int slot = used < 16 ? used++ : next;
+  next = (slot + 1) % 16;
+  keys[slot] = key;
+  maps[slot] = map;
+  *out = map;
+  return true;
+}
+
+// Grouped query heads: one CTA per (partition, KV head, request, chunk of up to
+// 16 query heads), the contraction on the tensor cores.
+template <typename T, typename TO, int D, int S, bool APPEND>
+pa_status launch_grouped(const pa::DecodeParams& prm, cudaStream_t stream) {
+  using Tg = pa::GqaTiling<D>;
+  auto kern = pa::paged_decode_gqa_kernel<T, TO, D, S, APPEND>;
+  static bool configured[kMaxDevices] = {};
+  if (!opt_in_smem(kern, Tg::SMEM, configured)) return PA_ERR_CUDA;
+  const int64_t rows = static_cast<int64_t>(prm.NB) * prm.Hkv * S;
+  if (rows <= 0 || rows > INT_MAX) return PA_ERR_INVALID;  // TMA row coordinates are int32
+  const pa_dtype dt = std::is_same<T, __half>::value ? PA_F16 : PA_BF16;
+  CUtensorMap tmk, tmv;
+  if (!row_map(&tmk, prm.k_cache, rows, D, S < 16 ? S : 16, dt) ||
+      !row_map(&tmv, prm.v_cache, rows, D, S < 16 ? S : 16, dt))
+    return PA_ERR_CUDA;
+  const int G = prm.H / prm.Hkv;
+  const dim3 grid(prm.NP, prm.Hkv * ((G + 15) / 16), prm.B);
+  kern<<<grid, (Tg::NC + 1) * 32, Tg::SMEM, stream>>>(prm, tmk, tmv);
+  launch_reduce<TO, D>(prm, stream);
   return cuda_status();
 }
 
 template <typename T, typename TO, bool APPEND>
 pa_status dispatch_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t st) {
-#define PA_CASE(DD, SS) \
-  if (D == DD && S == SS) return launch_decode<T, TO, DD, SS, APPEND>(prm, st);
+  const bool grouped = prm.H != prm.Hkv;
+#define PA_CASE(DD, SS)                                                            \
+  if (D == DD && S == SS)                                                          \
+    return grouped ? launch_grouped<T, TO, DD, SS, APPEND>(prm, st)                \
+                   : launch_decode<T, TO, DD, SS, APPEND>(prm, st);
   PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
   PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
   PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
@@ -219,9 +324,10 @@ namespace {
 pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_new,
                       const void* v_new, const void* k_cache, const void* v_cache,
                       const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
-                      int B, int H, int D, int S, int NB, pa_dtype dt, int partition,
+                      int B, int H, int Hkv, int D, int S, int NB, pa_dtype dt, int partition,
                       int max_seq_len, void* workspace, size_t ws_bytes, void* stream) {
   if (B < 0 || H <= 0 || NB < 0 || MB < 0) return PA_ERR_INVALID;
+  if (Hkv <= 0 || H % Hkv != 0) return PA_ERR_INVALID;
   if (!cache_dtype_ok(dt) || !out_dtype_ok(out_dt) || !decode_shape_ok(D, S)) return PA_ERR_INVALID;
   if (!std::isfinite(scale)) return PA_ERR_INVALID;
   if (B > 65535 || H > 65535) return PA_ERR_INVALID;  // grid y / z limits
@@ -248,6 +354,7 @@ pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_n
   prm.MB = MB;
   prm.B = B;
   prm.H = H;
+  prm.Hkv = Hkv;
   prm.NB = NB;
   if (NP > 1) {
     const size_t n = static_cast<size_t>(B) * H * NP;
@@ -284,7 +391,7 @@ pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cac
                     pa_dtype dt, int partition, int max_seq_len, void* workspace,
                     size_t ws_bytes, void* stream) {
   return decode_impl(out, out_dt, q, nullptr, nullptr, k_cache, v_cache, block_tables, MB,
-                     seq_lens, scale, B, H, D, S, NB, dt, partition, max_seq_len, workspace,
+                     seq_lens, scale, B, H, H, D, S, NB, dt, partition, max_seq_len, workspace,
                      ws_bytes, stream);
 }
 
@@ -297,7 +404,19 @@ pa_status pa_decode_append(void* out, pa_dtype out_dt, const void* q, const void
   if (B > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)))
     return PA_ERR_INVALID;
   return decode_impl(out, out_dt, q, B > 0 ? k_new : nullptr, v_new, k_cache, v_cache,
-                     block_tables, MB, seq_lens, scale, B, H, D, S, NB, dt, partition,
+                     block_tables, MB, seq_lens, scale, B, H, H, D, S, NB, dt, partition,
+                     max_seq_len, workspace, ws_bytes, stream);
+}
+
+pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k_new,
+                        const void* v_new, void* k_cache, void* v_cache,
+                        const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
+                        int B, int H, int Hkv, int D, int S, int NB, pa_dtype dt, int partition,
+                        int max_seq_len, void* workspace, size_t ws_bytes, void* stream) {
+  if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_INVALID;
+  if (k_new && B > 0 && (!aligned16(k_new) || !aligned16(v_new))) return PA_ERR_INVALID;
+  return decode_impl(out, out_dt, q, B > 0 ? k_new : nullptr, v_new, k_cache, v_cache,
+                     block_tables, MB, seq_lens, scale, B, H, Hkv, D, S, NB, dt, partition,
                      max_seq_len, workspace, ws_bytes, stream);
 }
 

@@ -32,6 +32,8 @@
 //   * no tensor cores: one query per head is a matrix-vector product.
 #pragma once
 
+#include <cuda.h>
+
 #include "pa_device.cuh"
 
 namespace pa {
@@ -50,6 +52,7 @@ struct DecodeParams {
   const void* v_new;           // [B, H, D] fused append: the new token's V (or null)
   float q_scale;               // scale * log2(e)
   int MB, B, H, NB;
+  int Hkv;   // KV heads in the cache; query head h reads KV head h / (H / Hkv)
   int P;     // tokens per partition (multiple of S)
   int NP;    // partitions in the grid
   int L_cap; // lengths are clamped to this (MB*S, or NP*P when split)
@@ -186,9 +189,10 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
   uint64_t* bar = bars + w * NS;
   uint8_t* stage0 = smem + w * NS * STAGE;
   const int32_t* trow = p.block_tables + static_cast<int64_t>(i) * p.MB;
-  const uint8_t* kbase = static_cast<const uint8_t*>(p.k_cache) + static_cast<int64_t>(h) * SLAB;
-  const uint8_t* vbase = static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(h) * SLAB;
-  const int64_t block_stride = static_cast<int64_t>(p.H) * SLAB;  // bytes per physical block
+  const int hk = h / (p.H / p.Hkv);  // this query head's KV head
+  const uint8_t* kbase = static_cast<const uint8_t*>(p.k_cache) + static_cast<int64_t>(hk) * SLAB;
+  const uint8_t* vbase = static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(hk) * SLAB;
+  const int64_t block_stride = static_cast<int64_t>(p.Hkv) * SLAB;  // bytes per physical block
   const uint64_t policy = policy_evict_first();
 
   // Fused append: does this warp own the new token?
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
   RawFrag k_row, v_row;
   int id_new = -1;
   if (appender && g == 0) {
-    const int64_t off = ((static_cast<int64_t>(i) * p.H + h) * D + pl * EPL) * 2;
+    const int64_t off = ((static_cast<int64_t>(i) * p.Hkv + hk) * D + pl * EPL) * 2;
     k_row.load(static_cast<const uint8_t*>(p.k_new) + off);
     v_row.load(static_cast<const uint8_t*>(p.v_new) + off);
     id_new = __ldg(trow + t_new / S);
@@ -382,6 +386,458 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
   if (!direct && threadIdx.x == 0) {
     p.ws_m[ih * p.NP + part] = M;
     p.ws_l[ih * p.NP + part] = Ltot;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Grouped-query decode on the tensor cores.
+//
+// With G query heads per KV head, a unit of 16 tokens is a small dense
+// contraction: S = Q K^T with Q [G x D] and K [16 x D], then O += P V with
+// V [16 x D]. One CTA per (partition, KV head, request, chunk of up to 16 query
+// heads) has two warps:
+//   * the producer loads each unit's 16 K rows and 16 V rows with tiled TMA
+//     copies through tensor maps that view each cache as a 2-D array of
+//     D-element rows (row (block * Hkv + head) * S + offset): boxes of 64
+//     elements x 16 rows (two boxes of 8 rows from two blocks when S = 8), with
+//     the 128-byte swizzle, so that the 8 rows an ldmatrix reads fall in 8
+//     different bank groups; D / 64 boxes per tile, an NS-stage ring with full /
+//     empty barriers, all waits bounded;
+//   * NC consumer warps take the units in turn (unit u to warp u % NC, two
+//     stages each), each keeping its own running (m, l, O), merged through
+//     shared memory at the end; several warps per SM hide the latency of the
+//     MMA / softmax dependency chain of one unit. Each consumer keeps Q (rows
+//     >= G zero) in shared memory and runs, per unit,
+//     mma.sync m16n8k16 (fp32 accumulate): S over D/16 k-steps for the two 8-token
+//     halves, the online softmax on the accumulator fragments (row max / sum over
+//     each lane quad), and O += P V with P passed as a bf16 (or fp16) hi + lo
+//     pair, so its rounding (2^-9) does not reach the output (2^-17); O stays
+//     in registers, D/8 fragments of 16 x 8.
+// Tokens past the end or in a skipped block are masked: their scores by
+// selection, their V rows by zeroing the fragment halves (rows never copied
+// may hold anything, NaN included). The fused append patches the new token's
+// rows into the staged unit (one consumer per CTA, so no cross-warp barrier)
+// and one CTA per KV head stores them to the cache.
+// tcgen05 (M >= 64) would pad an 8-head group eightfold and move the running
+// softmax through TMEM; the path is bound by HBM, and m16n8k16 keeps S, P and
+// O in registers.
+template <int D>
+struct GqaTiling {
+  static constexpr int ROWS = 16;               // tokens per unit = one MMA k-step of P V
+  static constexpr int BOX = 16 * 128;          // one swizzled box: 16 rows x 64 elements
+  static constexpr int TILE = (D / 64) * BOX;   // one K (or V) unit
+  static constexpr int STAGE = 2 * TILE;
+  static constexpr int QPITCH = (D + 8) * 2;    // the Q tile, padded rows
+  static constexpr int SMEM_Q = ROWS * QPITCH;
+  static constexpr int NC = 4;                  // consumer warps; unit u goes to warp u % NC
+  static constexpr int NS = 2 * NC;             // two stages per consumer
+  static constexpr int SMEM_MERGE = NC * ROWS * (D + 2) * 4;  // reuses the stages at the end
+  static constexpr int SMEM_STAGES = NS * STAGE > SMEM_MERGE ? NS * STAGE : SMEM_MERGE;
+  // + 1024: the stages start on a 1024-byte boundary (the swizzle period)
+  static constexpr int SMEM = 1024 + SMEM_STAGES + SMEM_Q + 2 * NS * 8 + NS * 4;
+};
+
+// Byte offset of 16-byte chunk cc (0 .. D/8 - 1) of row r (0 .. 15) in a unit tile
+// of D/64 boxes, each 16 rows x 128 bytes with the 128-byte swizzle (chunk c of
+// row r stored at chunk c ^ (r % 8)).
+__device__ __forceinline__ int swz(int r, int cc) {
+  return (cc >> 3) * 2048 + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+}
+
+template <typename T>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1);
+template <>
+__device__ __forceinline__ void mma16816<__nv_bfloat16>(float (&d)[4], const uint32_t (&a)[4],
+                                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+template <>
+__device__ __forceinline__ void mma16816<__half>(float (&d)[4], const uint32_t (&a)[4],
+                                                 uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+
+// Two fp32 -> a packed pair of 16-bit values (low half = first), round to nearest.
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
+  const __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+// The fp32 value of the low / high 16-bit half of a packed pair.
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t x) {
+  return Elem<T>::pair(x);
+}
+
+template <typename T, typename TO, int D, int S, bool APPEND>
+__global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
+    paged_decode_gqa_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
+                            const __grid_constant__ CUtensorMap tmv) {
+  using Tg = GqaTiling<D>;
+  constexpr int ROWS = Tg::ROWS, PITCH = Tg::QPITCH, TILE = Tg::TILE, STAGE = Tg::STAGE;
+  constexpr int NS = Tg::NS, NC = Tg::NC;
+  constexpr int BR = S < 16 ? S : 16;  // rows per box
+  constexpr int SLAB = S * D * 2;
+  constexpr int NT = D / 8;   // 8-wide n-tiles of O
+  constexpr int KS = D / 16;  // k-steps of S
+
+  const int part = blockIdx.x;
+  const int G = p.H / p.Hkv;
+  const int chunks = (G + 15) / 16;
+  const int hk = blockIdx.y / chunks;
+  const int c0 = (blockIdx.y % chunks) * 16;  // first query head (within the group) of this CTA
+  const int gc = min(16, G - c0);             // query heads served here
+  const int i = blockIdx.z;
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+
+  int L = __ldg(p.seq_lens + i);
+  const bool len_ok = L >= 0 && L <= p.L_cap;
+  if (!len_ok) {
+    if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) raise_error(PA_DEVERR_SEQ_LEN);
+    L = L < 0 ? 0 : p.L_cap;
+  }
+  const int nparts = (L + p.P - 1) / p.P;
+  if (part > 0 && part >= nparts) return;
+  const bool direct = nparts <= 1;
+
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* stages = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* qtile = stages + Tg::SMEM_STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(qtile + Tg::SMEM_Q);
+  uint64_t* empty = full + NS;
+  uint32_t* rowmask = reinterpret_cast<uint32_t*>(empty + NS);  // per stage: rows copied
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int t_beg = part * p.P;
+  const int t_end = min(t_beg + p.P, L);
+  const int nunits = t_end > t_beg ? (t_end - t_beg + ROWS - 1) / ROWS : 0;
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(i) * p.MB;
+  const int64_t block_stride = static_cast<int64_t>(p.Hkv) * SLAB;
+  const uint8_t* kbase = static_cast<const uint8_t*>(p.k_cache) + static_cast<int64_t>(hk) * SLAB;
+  const uint8_t* vbase = static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(hk) * SLAB;
+
+  if (w == NC) {
+    // ---- producer: lane 0 issues the unit's box loads ----
+    const uint64_t policy = policy_evict_first();
+    const int blk0 = t_beg / S;
+    const int blk1 = t_end > t_beg ? (t_end + S - 1) / S : blk0;
+    int base = 0;
+    int ids_a = (blk0 + lane < blk1) ? __ldg(trow + blk0 + lane) : -1;
+    int ids_b = (blk0 + 32 + lane < blk1) ? __ldg(trow + blk0 + 32 + lane) : -1;
+    for (int u = 0; u < nunits; ++u) {
+      const int s = u % NS;
+      if (u >= NS && !mbar_wait_bounded(&empty[s], ((u / NS) - 1) & 1)) {
+        if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+        break;
+      }
+      const int t0 = t_beg + u * ROWS;
+      if (t0 / S - blk0 >= base + 32) {  // slide the id window (a unit spans <= 2 blocks)
+        base += 32;
+        ids_a = ids_b;
+        const int nx = blk0 + base + 32 + lane;
+        ids_b = nx < blk1 ? __ldg(trow + nx) : -1;
+      }
+      const int rel = t0 / S - blk0 - base;  // 0 .. 31
+      const int id0 = __shfl_sync(kFullMask, ids_a, rel);
+      const int id1a = __shfl_sync(kFullMask, ids_a, (rel + 1) & 31);
+      const int id1b = __shfl_sync(kFullMask, ids_b, (rel + 1) & 31);
+      if (lane == 0) {
+        // the unit's rows in one box group (S >= 16) or two (S = 8)
+        uint32_t okmask = 0, bytes = 0;
+        int rows_y[2] = {0, 0};
+        bool issue[2] = {false, false};
+        constexpr int NH = ROWS / BR;
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          const int th = t0 + hh * BR;
+          if (th >= t_end) continue;
+          const int id = hh == 0 ? id0 : (rel + 1 < 32 ? id1a : id1b);
+          if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.NB)) {
+            raise_error(PA_DEVERR_BLOCK_ID);
+            continue;
+          }
+          issue[hh] = true;
+          rows_y[hh] = (id * p.Hkv + hk) * S + th % S;
+          const int nrow = min(BR, t_end - th);
+          okmask |= ((1u << nrow) - 1u) << (hh * BR);
+          bytes += 2u * (D / 64) * BR * 128u;
+        }
+        rowmask[s] = okmask;
+        mbar_arrive_expect_tx(&full[s], bytes);
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          if (!issue[hh]) continue;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint8_t* dst = stages + s * STAGE + c * Tg::BOX + hh * BR * 128;
+            tma_load_2d(dst, &tmk, c * 64, rows_y[hh], &full[s], policy);
+            tma_load_2d(dst + TILE, &tmv, c * 64, rows_y[hh], &full[s], policy);
+          }
+        }
+      }
+      __syncwarp();
+    }
+    return;
+  }
+
+  // ---- consumers ----
+  const int gq = lane >> 2;  // accumulator row (and row + 8)
+  const int tq = lane & 3;   // accumulator column pair
+  // Q tile: rows < gc are query heads hk * G + c0 + row, the rest zero
+  for (int idx = threadIdx.x; idx < ROWS * (D / 8); idx += NC * 32) {
+    const int row = idx / (D / 8), ch = idx % (D / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (row < gc) {
+      const int64_t hq = static_cast<int64_t>(hk) * G + c0 + row;
+      val = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
+                                            ((static_cast<int64_t>(i) * p.H + hq) * D + ch * 8) * 2);
+    }
+    *reinterpret_cast<uint4*>(qtile + row * PITCH + ch * 16) = val;
+  }
+  // consumers only: the Q tile is complete before anyone reads it
+  asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
+  // fused append: the new token's rows, one 16-byte chunk per lane; the warp
+  // that consumes the new token's unit patches them in
+  const int t_new = L - 1;
+  const bool has_new = APPEND && len_ok && L >= 1 && t_new >= t_beg && t_new < t_end &&
+                       ((t_new - t_beg) / ROWS) % NC == w;
+  uint4 k_chunk = make_uint4(0, 0, 0, 0), v_chunk = make_uint4(0, 0, 0, 0);
+  const bool chunk_lane = lane < D / 8;
+  if (has_new && chunk_lane) {
+    const int64_t off = ((static_cast<int64_t>(i) * p.Hkv + hk) * D + lane * 8) * 2;
+    k_chunk = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.k_new) + off);
+    v_chunk = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.v_new) + off);
+    if (c0 == 0) {  // one CTA per KV head stores the row to the cache
+      const int id_new = __ldg(trow + t_new / S);
+      if (static_cast<unsigned>(id_new) < static_cast<unsigned>(p.NB)) {
+        const int64_t goff = static_cast<int64_t>(id_new) * block_stride +
+                             (static_cast<int64_t>(t_new % S) * D + lane * 8) * 2;
+        *reinterpret_cast<uint4*>(const_cast<uint8_t*>(kbase) + goff) = k_chunk;
+        *reinterpret_cast<uint4*>(const_cast<uint8_t*>(vbase) + goff) = v_chunk;
+      }
+    }
+  }
+  __syncwarp();
+
+  float o[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY;  // running max of rows gq and gq + 8 (base 2)
+  float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums
+  // ldmatrix lane addresses: A (Q) rows lane % 16, k half lane / 16; B (K) token
+  // (lane & 7) + 8 * (lane >> 4), k half (lane >> 3) & 1; B (V, transposed) token
+  // (lane & 7) + 8 * ((lane >> 3) & 1), d half lane >> 4; K and V through the swizzle
+  const int a_row = lane & 15, a_k8 = (lane >> 4) * 8;
+  const int kb_tok = (lane & 7) + 8 * (lane >> 4), kb_k8 = ((lane >> 3) & 1) * 8;
+  const int vb_tok = (lane & 7) + 8 * ((lane >> 3) & 1), vb_d8 = (lane >> 4) * 8;
+
+  for (int k = w; k < nunits; k += NC) {
+    const int s = k % NS;
+    if (!mbar_wait_bounded(&full[s], (k / NS) & 1)) {
+      if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+      break;
+    }
+    uint8_t* ktile = stages + s * STAGE;
+    uint8_t* vtile = ktile + TILE;
+    const int t0 = t_beg + k * ROWS;
+    uint32_t valid = rowmask[s];
+    if (has_new && t_new >= t0 && t_new < t0 + ROWS) {
+      const int rnew = t_new - t0;
+      if (chunk_lane) {
+        *reinterpret_cast<uint4*>(ktile + swz(rnew, lane)) = k_chunk;
+        *reinterpret_cast<uint4*>(vtile + swz(rnew, lane)) = v_chunk;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+    }
+
+    // S = Q K^T for tokens 0-7 (sacc[0]) and 8-15 (sacc[1])
+    float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      uint32_t a[4], b[4];
+      ldsm_x4(a, qtile + a_row * PITCH + (kk * 16 + a_k8) * 2);
+      ldsm_x4(b, ktile + swz(kb_tok, (kk * 16 + kb_k8) >> 3));
+      mma16816<T>(sacc[0], a, b[0], b[1]);
+      mma16816<T>(sacc[1], a, b[2], b[3]);
+    }
+    // scores (base 2), masked by selection: accumulator element e of n-tile j is
+    // row gq + 8 * (e >> 1), token 8 * j + 2 * tq + (e & 1)
+    float sc[2][4];
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = 8 * j + 2 * tq + (e & 1);
+        const bool ok = (valid >> tok) & 1u;
+        sc[j][e] = ok ? sacc[j][e] * p.q_scale : -INFINITY;
+        if (e < 2) mx0 = fmaxf(mx0, sc[j][e]); else mx1 = fmaxf(mx1, sc[j][e]);
+      }
+#pragma unroll
+    for (int off = 1; off <= 2; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    // a unit with no valid token for a row keeps its max at -inf: guard the exponent
+    const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m0 - mn0);
+    const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
+    float pr[2][4];
+    float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float mref = e < 2 ? mn0 : mn1;
+        pr[j][e] = sc[j][e] == -INFINITY ? 0.f : exp2f(sc[j][e] - mref);
+        if (e < 2) ls0 += pr[j][e]; else ls1 += pr[j][e];
+      }
+    l0 = l0 * al0 + ls0;
+    l1 = l1 * al1 + ls1;
+    m0 = mn0;
+    m1 = mn1;
+    // once the running max settles, most units change no row's max: skip the
+    // rescale of O unless some row of the warp needs it
+    if (__any_sync(kFullMask, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        o[n][0] *= al0;
+        o[n][1] *= al0;
+        o[n][2] *= al1;
+        o[n][3] *= al1;
+      }
+    }
+    // P as the A operand (16 x 16 tokens), as a hi + lo pair of 16-bit values
+    uint32_t ph[4], plo[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      ph[2 * j] = pack2<T>(pr[j][0], pr[j][1]);      // row gq, tokens 8j + 2tq, +1
+      ph[2 * j + 1] = pack2<T>(pr[j][2], pr[j][3]);  // row gq + 8
+      const float2 h0 = unpack2<T>(ph[2 * j]), h1 = unpack2<T>(ph[2 * j + 1]);
+      plo[2 * j] = pack2<T>(pr[j][0] - h0.x, pr[j][1] - h0.y);
+      plo[2 * j + 1] = pack2<T>(pr[j][2] - h1.x, pr[j][3] - h1.y);
+    }
+    // A-fragment order: (row gq, k 0-7), (row gq+8, k 0-7), (row gq, k 8-15), (row gq+8, k 8-15)
+    const uint32_t ahi[4] = {ph[0], ph[1], ph[2], ph[3]};
+    const uint32_t alo[4] = {plo[0], plo[1], plo[2], plo[3]};
+    // V rows that were not copied are zeroed in the B fragments (0 * NaN would be NaN)
+    const bool partial = valid != 0xffffu;
+    const uint32_t vm0 = (((valid >> (2 * tq)) & 1u) ? 0x0000ffffu : 0u) |
+                         (((valid >> (2 * tq + 1)) & 1u) ? 0xffff0000u : 0u);
+    const uint32_t vm1 = (((valid >> (2 * tq + 8)) & 1u) ? 0x0000ffffu : 0u) |
+                         (((valid >> (2 * tq + 9)) & 1u) ? 0xffff0000u : 0u);
+#pragma unroll
+    for (int n2 = 0; n2 < NT / 2; ++n2) {
+      uint32_t b[4];
+      ldsm_x4_trans(b, vtile + swz(vb_tok, (n2 * 16 + vb_d8) >> 3));
+      if (partial) {
+        b[0] &= vm0;
+        b[1] &= vm1;
+        b[2] &= vm0;
+        b[3] &= vm1;
+      }
+      mma16816<T>(o[2 * n2], ahi, b[0], b[1]);
+      mma16816<T>(o[2 * n2], alo, b[0], b[1]);
+      mma16816<T>(o[2 * n2 + 1], ahi, b[2], b[3]);
+      mma16816<T>(o[2 * n2 + 1], alo, b[2], b[3]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+
+  // row sums over the lane quad
+#pragma unroll
+  for (int off = 1; off <= 2; off <<= 1) {
+    l0 += __shfl_xor_sync(kFullMask, l0, off);
+    l1 += __shfl_xor_sync(kFullMask, l1, off);
+  }
+  // merge the NC consumers' (m, l, O) per row through shared memory (the stages
+  // are free: every unit has been consumed once all consumers pass the barrier)
+  asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
+  float* mg = reinterpret_cast<float*>(stages);  // [NC][ROWS][D + 2]: m, l, O
+  {
+    float* mine = mg + w * ROWS * (D + 2);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float* rowp = mine + (gq + 8 * half) * (D + 2);
+      if (tq == 0) {
+        rowp[0] = half ? m1 : m0;
+        rowp[1] = half ? l1 : l0;
+      }
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        rowp[2 + 8 * n + 2 * tq] = o[n][2 * half];
+        rowp[2 + 8 * n + 2 * tq + 1] = o[n][2 * half + 1];
+      }
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
+  // consumer w finishes rows w, w + NC, ...: M = max m, out = sum 2^(m - M) O / sum 2^(m - M) l
+  for (int row = w; row < gc; row += NC) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) M = fmaxf(M, mg[(c * ROWS + row) * (D + 2)]);
+    float wt[NC];
+    float lsum = 0.f;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const float mc = mg[(c * ROWS + row) * (D + 2)];
+      wt[c] = mc == -INFINITY ? 0.f : exp2f(mc - M);
+      lsum = fmaf(wt[c], mg[(c * ROWS + row) * (D + 2) + 1], lsum);
+    }
+    const int64_t hq = static_cast<int64_t>(hk) * G + c0 + row;
+    const int64_t ih = static_cast<int64_t>(i) * p.H + hq;
+    for (int d = lane; d < D; d += 32) {
+      float a = 0.f;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) a = fmaf(wt[c], mg[(c * ROWS + row) * (D + 2) + 2 + d], a);
+      if (direct) {
+        static_cast<TO*>(p.out)[ih * D + d] = to_out<TO>(lsum > 0.f ? a / lsum : 0.f);
+      } else {
+        p.ws_acc[(ih * p.NP + part) * D + d] = a;
+      }
+    }
+    if (!direct && lane == 0) {
+      p.ws_m[ih * p.NP + part] = M;
+      p.ws_l[ih * p.NP + part] = lsum;
+    }
   }
 }
 

@@ -89,6 +89,19 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Two-dimensional tiled TMA load global -> this CTA's shared memory through a
+// tensor map (in kernel-parameter space), completing on `bar`. x is the
+// innermost coordinate; x * element size must be a multiple of 16 bytes. No
+// multicast.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // ---- 16-bit element conversions -------------------------------------------------
 
 template <typename T>
@@ -143,6 +156,18 @@ __device__ __forceinline__ void load_row(const void* p, float (&f)[DL]) {
       f[2 * k] = a.x;
       f[2 * k + 1] = a.y;
     }
+  }
+}
+
+// 8 consecutive 16-bit elements held in a uint4 -> fp32 registers.
+template <typename T>
+__device__ __forceinline__ void convert_frag(const uint4& x, float (&f)[8]) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 a = Elem<T>::pair(w[k]);
+    f[2 * k] = a.x;
+    f[2 * k + 1] = a.y;
   }
 }
 

@@ -66,8 +66,9 @@ def lognormal_lengths(n, median, sigma, lo, hi, gen):
 
 
 def decode_case(seq_lens, H, D, S, dtype, seed, device, pool_blocks=None, poison=True,
-                max_blocks=None):
-    """A batch of single-query decode inputs.
+                max_blocks=None, Hkv=None):
+    """A batch of single-query decode inputs (Hkv KV heads in the cache, H query
+    heads; Hkv defaults to H).
 
     Request i holds the first ceil(L_i / S) ids of its share of a random
     permutation of the pool; ``pool_blocks`` (default: exactly enough) sets the
@@ -91,9 +92,10 @@ def decode_case(seq_lens, H, D, S, dtype, seed, device, pool_blocks=None, poison
         tables_host.append(ids.tolist())
         off += n
     dgen = _dev_gen(seed, device)
+    Hc = H if Hkv is None else Hkv
     q = torch.randn((B, H, D), generator=dgen, device=device, dtype=torch.float32).to(dtype)
-    k_cache = torch.randn((NB, H, S, D), generator=dgen, device=device, dtype=dtype)
-    v_cache = torch.randn((NB, H, S, D), generator=dgen, device=device, dtype=dtype)
+    k_cache = torch.randn((NB, Hc, S, D), generator=dgen, device=device, dtype=dtype)
+    v_cache = torch.randn((NB, Hc, S, D), generator=dgen, device=device, dtype=dtype)
     if poison:
         unused = perm[need:].to(device)
         if unused.numel():
@@ -136,6 +138,15 @@ def long_context_decode(seed=0, device="cpu", batch=8, lo=32768, hi=131072, H=32
     32 heads, head_dim 128, block 16, bf16, permuted pool."""
     lens = uniform_lengths(batch, lo, hi, seed)
     return decode_case(lens, H=H, D=128, S=16, dtype=torch.bfloat16, seed=seed, device=device)
+
+
+def llama70b_decode(seed=0, device="cpu", batch=64, max_len=2048):
+    """LLaMA-2-70B-shaped single-layer decode (grouped-query attention, not on the
+    pages): 64 query heads sharing 8 KV heads, head_dim 128, block 16, bf16,
+    seq_lens uniform in [1, 2048]."""
+    lens = uniform_lengths(batch, 1, max_len, seed)
+    return decode_case(lens, H=64, D=128, S=16, dtype=torch.bfloat16, seed=seed, device=device,
+                       Hkv=8)
 
 
 def sweep_case(S, D, B, dtype, seed=0, device="cpu", H=32, lo=16, hi=8192):

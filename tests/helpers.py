@@ -37,8 +37,14 @@ def run_decode(case, out_dtype=torch.float32, partition=0, max_seq_len=None, str
     out = torch.empty((B, H, D), dtype=out_dtype, device=case.q.device)
     ws_bytes = binding.pa_decode_workspace_bytes(B, H, D, S, max_seq_len, partition)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=case.q.device) if ws_bytes else None
-    binding.pa_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
-                      case.scale, max_seq_len, partition=partition, workspace=ws, stream=stream)
+    if case.k_cache.shape[1] != H:  # grouped query heads
+        binding.pa_decode_gqa(out, case.q, case.k_cache, case.v_cache, case.block_tables,
+                              case.seq_lens, case.scale, max_seq_len, partition=partition,
+                              workspace=ws, stream=stream)
+    else:
+        binding.pa_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables,
+                          case.seq_lens, case.scale, max_seq_len, partition=partition,
+                          workspace=ws, stream=stream)
     return out, ws
 
 
@@ -59,6 +65,7 @@ def oracle_pairs(case, pairs, threads=0):
     """
     S = case.k_cache.shape[2]
     D = case.q.shape[2]
+    G = case.q.shape[1] // case.k_cache.shape[1]  # query heads per KV head
     ks, vs, qs, tables, lens = [], [], [], [], []
     off = 0
     for i, h in pairs:
@@ -66,8 +73,8 @@ def oracle_pairs(case, pairs, threads=0):
         blocks = case.tables_host[i][: -(-L // S)]
         n = len(blocks)
         idx = torch.tensor(blocks, dtype=torch.long, device=case.k_cache.device)
-        ks.append(case.k_cache[idx, h].unsqueeze(1).cpu())
-        vs.append(case.v_cache[idx, h].unsqueeze(1).cpu())
+        ks.append(case.k_cache[idx, h // G].unsqueeze(1).cpu())
+        vs.append(case.v_cache[idx, h // G].unsqueeze(1).cpu())
         qs.append(case.q[i, h].view(1, 1, D).cpu())
         tables.append(list(range(off, off + n)))
         lens.append(L)
