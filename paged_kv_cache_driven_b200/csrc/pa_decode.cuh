@@ -34,6 +34,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "pa_device.cuh"
 
 namespace pa {
@@ -410,9 +412,9 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
 //     >= G zero) in shared memory and runs, per unit,
 //     mma.sync m16n8k16 (fp32 accumulate): S over D/16 k-steps for the two 8-token
 //     halves, the online softmax on the accumulator fragments (row max / sum over
-//     each lane quad), and O += P V with P passed as a bf16 (or fp16) hi + lo
-//     pair, so its rounding (2^-9) does not reach the output (2^-17); O stays
-//     in registers, D/8 fragments of 16 x 8.
+//     each lane quad), and O += P V with P passed, for bf16, as a hi + lo pair,
+//     so its rounding (2^-9) does not reach the output (2^-17); fp16 P (2^-11)
+//     goes in alone; O stays in registers, D/8 fragments of 16 x 8.
 // Tokens past the end or in a skipped block are masked: their scores by
 // selection, their V rows by zeroing the fragment halves (rows never copied
 // may hold anything, NaN included). The fused append patches the new token's
@@ -687,16 +689,24 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
       __syncwarp();
     }
 
-    // S = Q K^T for tokens 0-7 (sacc[0]) and 8-15 (sacc[1])
+    // S = Q K^T for tokens 0-7 (sacc[0]) and 8-15 (sacc[1]); even and odd
+    // k-steps accumulate in separate registers so two MMA chains run at once
     float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float sodd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       uint32_t a[4], b[4];
       ldsm_x4(a, qtile + a_row * PITCH + (kk * 16 + a_k8) * 2);
       ldsm_x4(b, ktile + swz(kb_tok, (kk * 16 + kb_k8) >> 3));
-      mma16816<T>(sacc[0], a, b[0], b[1]);
-      mma16816<T>(sacc[1], a, b[2], b[3]);
+      float (&acc0)[4] = (kk & 1) ? sodd[0] : sacc[0];
+      float (&acc1)[4] = (kk & 1) ? sodd[1] : sacc[1];
+      mma16816<T>(acc0, a, b[0], b[1]);
+      mma16816<T>(acc1, a, b[2], b[3]);
     }
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[j][e] += sodd[j][e];
     // scores (base 2), masked by selection: accumulator element e of n-tile j is
     // row gq + 8 * (e >> 1), token 8 * j + 2 * tq + (e & 1)
     float sc[2][4];
@@ -744,15 +754,20 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
         o[n][3] *= al1;
       }
     }
-    // P as the A operand (16 x 16 tokens), as a hi + lo pair of 16-bit values
+    // P as the A operand (16 x 16 tokens). bf16 keeps 8 bits, so P goes in as a
+    // hi + lo pair (its rounding drops from 2^-9 to 2^-17); fp16 keeps 11, within
+    // the tolerance on its own, so only the hi part is used.
+    constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
     uint32_t ph[4], plo[4];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       ph[2 * j] = pack2<T>(pr[j][0], pr[j][1]);      // row gq, tokens 8j + 2tq, +1
       ph[2 * j + 1] = pack2<T>(pr[j][2], pr[j][3]);  // row gq + 8
-      const float2 h0 = unpack2<T>(ph[2 * j]), h1 = unpack2<T>(ph[2 * j + 1]);
-      plo[2 * j] = pack2<T>(pr[j][0] - h0.x, pr[j][1] - h0.y);
-      plo[2 * j + 1] = pack2<T>(pr[j][2] - h1.x, pr[j][3] - h1.y);
+      if (kSplitP) {
+        const float2 h0 = unpack2<T>(ph[2 * j]), h1 = unpack2<T>(ph[2 * j + 1]);
+        plo[2 * j] = pack2<T>(pr[j][0] - h0.x, pr[j][1] - h0.y);
+        plo[2 * j + 1] = pack2<T>(pr[j][2] - h1.x, pr[j][3] - h1.y);
+      }
     }
     // A-fragment order: (row gq, k 0-7), (row gq+8, k 0-7), (row gq, k 8-15), (row gq+8, k 8-15)
     const uint32_t ahi[4] = {ph[0], ph[1], ph[2], ph[3]};
@@ -774,9 +789,11 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
         b[3] &= vm1;
       }
       mma16816<T>(o[2 * n2], ahi, b[0], b[1]);
-      mma16816<T>(o[2 * n2], alo, b[0], b[1]);
       mma16816<T>(o[2 * n2 + 1], ahi, b[2], b[3]);
-      mma16816<T>(o[2 * n2 + 1], alo, b[2], b[3]);
+      if (kSplitP) {
+        mma16816<T>(o[2 * n2], alo, b[0], b[1]);
+        mma16816<T>(o[2 * n2 + 1], alo, b[2], b[3]);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
