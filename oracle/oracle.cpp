@@ -262,4 +262,60 @@ int oracle_partition_stats(const uint16_t* q, const uint16_t* k_cache, const uin
   });
 }
 
+// Paged prefill attention, causal ("vLLM KV Cache and PagedAttention
+// Explained", 7단계 and Step 6 "Prefill and Decode": all prompt tokens run at
+// once; each token attends to the tokens before it and itself). Request i has
+// seq_lens[i] tokens in the cache, the last n_i = q_start[i+1] - q_start[i] of
+// them new; new token j (absolute position seq_lens[i] - n_i + j) attends to
+// cache tokens 0 .. that position. q and out are [q_start[B], H, D]; the
+// query rows of request i are q_start[i] .. q_start[i+1) - 1.
+int oracle_paged_prefill(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                         const int32_t* block_tables, const int32_t* seq_lens,
+                         const int32_t* q_start, int64_t B, int64_t H, int64_t D, int64_t S,
+                         int64_t NB, int64_t MB, double scale, int dtype, int n_threads,
+                         double* out) {
+  if (!q_start || !seq_lens || B < 0 || q_start[0] != 0) return 1;
+  const int64_t T = q_start[B];
+  // one Problem per query row would duplicate q; instead reuse the decode
+  // pieces with a per-row length: row t of request i is a decode of length pos+1
+  std::vector<int64_t> row_req(static_cast<size_t>(T)), row_pos(static_cast<size_t>(T));
+  for (int64_t i = 0; i < B; ++i) {
+    const int64_t n = q_start[i + 1] - q_start[i];
+    if (n < 0 || n > seq_lens[i] || seq_lens[i] > MB * S) return 1;
+    for (int64_t j = 0; j < n; ++j) {
+      row_req[q_start[i] + j] = i;
+      row_pos[q_start[i] + j] = seq_lens[i] - n + j;
+    }
+  }
+  const Problem p{q, k_cache, v_cache, block_tables, seq_lens, T, H, D, S, NB, MB, scale, dtype, H};
+  if (!valid_problem(p) || !out) return 1;
+  return parallel_for(T * H, n_threads, [&](int64_t k) {
+    const int64_t t = k / H, h = k % H;
+    const int64_t i = row_req[t];
+    const int64_t L = row_pos[t] + 1;  // tokens this row attends to
+    double* o = out + k * D;
+    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    std::vector<double> sc(static_cast<size_t>(L));
+    std::vector<int64_t> rows(static_cast<size_t>(L));
+    const int64_t qoff = (t * H + h) * D;
+    for (int64_t tt = 0; tt < L; ++tt) {
+      const int64_t row = token_row(p, i, h, tt);
+      if (row < 0) return 3;
+      rows[tt] = row;
+      double dot = 0.0;
+      for (int64_t d = 0; d < D; ++d) dot += elem(p, q, qoff + d) * elem(p, k_cache, row + d);
+      sc[tt] = scale * dot;
+    }
+    double m = -std::numeric_limits<double>::infinity();
+    for (double x : sc) m = std::max(m, x);
+    double z = 0.0;
+    for (double x : sc) z += std::exp(x - m);
+    for (int64_t tt = 0; tt < L; ++tt) {
+      const double w = std::exp(sc[tt] - m) / z;
+      for (int64_t d = 0; d < D; ++d) o[d] += w * elem(p, v_cache, rows[tt] + d);
+    }
+    return 0;
+  });
+}
+
 }  // extern "C"

@@ -276,3 +276,33 @@ def test_grouped_query_heads_equal_sdpa_with_gqa(oracle_lib, G):
     rep = oracle_decode.paged_decode(q, kc.repeat_interleave(G, dim=1),
                                      vc.repeat_interleave(G, dim=1), bt, sl, 0.125)
     assert np.array_equal(got, rep)
+
+
+@pytest.mark.parametrize("ctx", [0, 5, 37])
+def test_prefill_equals_causal_sdpa(oracle_lib, ctx):
+    """Causal prefill over the paged cache ("vLLM KV Cache and PagedAttention
+    Explained", Step 6 "Prefill"): equal to torch SDPA with a causal mask shifted
+    by the context already cached; its last row equals the decode of that
+    request."""
+    gen = torch.Generator().manual_seed(ctx + 1)
+    H, D, S = 2, 32, 8
+    news = [1, 9, 30]
+    lens = [ctx + n for n in news]
+    ks = [torch.randn(L, H, D, generator=gen).to(torch.bfloat16) for L in lens]
+    vs = [torch.randn(L, H, D, generator=gen).to(torch.bfloat16) for L in lens]
+    kc, vc, bt, sl = make_paged(ks, vs, S, 2, gen)
+    q = torch.randn(sum(news), H, D, generator=gen).to(torch.bfloat16)
+    q_start = torch.tensor([0] + list(np.cumsum(news)), dtype=torch.int32)
+    got = oracle_decode.paged_prefill(q, kc, vc, bt, sl, q_start, 0.2)
+    for i, (L, n) in enumerate(zip(lens, news)):
+        qi = q[q_start[i]:q_start[i + 1]].double().transpose(0, 1)       # [H, n, D]
+        ki, vi = ks[i].double().transpose(0, 1), vs[i].double().transpose(0, 1)
+        pos = torch.arange(L - n, L).unsqueeze(1)
+        mask = torch.arange(L).unsqueeze(0) <= pos                         # [n, L]
+        want = F.scaled_dot_product_attention(qi, ki, vi, attn_mask=mask, scale=0.2)
+        np.testing.assert_allclose(got[q_start[i]:q_start[i + 1]], want.transpose(0, 1).numpy(),
+                                   rtol=1e-12, atol=1e-12)
+    last = torch.stack([q[q_start[i + 1] - 1] for i in range(len(news))])
+    dec = oracle_decode.paged_decode(last, kc, vc, bt, sl, 0.2)
+    for i in range(len(news)):
+        assert np.array_equal(got[q_start[i + 1] - 1], dec[i])
