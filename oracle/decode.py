@@ -39,7 +39,7 @@ def _load():
                                                ctypes.c_double, ctypes.c_int, i64, i64,
                                                ctypes.c_int, p, p, p]
         lib.oracle_partition_stats.restype = ctypes.c_int
-        lib.oracle_paged_prefill.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, i64, i64,
+        lib.oracle_paged_prefill.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64,
                                              ctypes.c_double, ctypes.c_int, ctypes.c_int, p]
         lib.oracle_paged_prefill.restype = ctypes.c_int
         lib.oracle_decode16.argtypes = [ctypes.c_uint16, ctypes.c_int]
@@ -142,10 +142,11 @@ def paged_prefill(q, k_cache, v_cache, block_tables, seq_lens, q_start, scale, t
     PagedAttention Explained", Step 6 "Prefill"): q [T, H, D] holds the new tokens
     of every request (request i's rows q_start[i] .. q_start[i+1] - 1, the last
     q_start[i+1] - q_start[i] of its seq_lens[i] cached tokens); row j of request
-    i attends to cache tokens 0 .. seq_lens[i] - n_i + j. Returns [T, H, D]."""
+    i attends to cache tokens 0 .. seq_lens[i] - n_i + j; query head h reads KV
+    head h // (H // Hkv) of the [NB, Hkv, S, D] caches. Returns [T, H, D]."""
     T, H, D = q.shape
-    NB, H2, S, D2 = k_cache.shape
-    if (H2, D2) != (H, D):
+    NB, Hkv, S, D2 = k_cache.shape
+    if D2 != D or H % Hkv:
         raise OracleError("shape mismatch")
     qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
     sl = _i32(seq_lens).reshape(-1)
@@ -154,7 +155,7 @@ def paged_prefill(q, k_cache, v_cache, block_tables, seq_lens, q_start, scale, t
     qs = _i32(q_start).reshape(B + 1)
     out = np.zeros((T, H, D), np.float64)
     rc = _load().oracle_paged_prefill(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), _ptr(sl), _ptr(qs),
-                                      B, H, D, S, NB, bt.shape[1], float(scale),
+                                      B, H, Hkv, D, S, NB, bt.shape[1], float(scale),
                                       _DTYPE_CODE[q.dtype], int(threads), _ptr(out))
     if rc:
         raise OracleError(f"oracle_paged_prefill returned {rc}")

@@ -268,12 +268,13 @@ int oracle_partition_stats(const uint16_t* q, const uint16_t* k_cache, const uin
 // seq_lens[i] tokens in the cache, the last n_i = q_start[i+1] - q_start[i] of
 // them new; new token j (absolute position seq_lens[i] - n_i + j) attends to
 // cache tokens 0 .. that position. q and out are [q_start[B], H, D]; the
-// query rows of request i are q_start[i] .. q_start[i+1) - 1.
+// query rows of request i are q_start[i] .. q_start[i+1) - 1; query head h
+// reads KV head h / (H / Hkv).
 int oracle_paged_prefill(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
                          const int32_t* block_tables, const int32_t* seq_lens,
-                         const int32_t* q_start, int64_t B, int64_t H, int64_t D, int64_t S,
-                         int64_t NB, int64_t MB, double scale, int dtype, int n_threads,
-                         double* out) {
+                         const int32_t* q_start, int64_t B, int64_t H, int64_t Hkv, int64_t D,
+                         int64_t S, int64_t NB, int64_t MB, double scale, int dtype,
+                         int n_threads, double* out) {
   if (!q_start || !seq_lens || B < 0 || q_start[0] != 0) return 1;
   const int64_t T = q_start[B];
   // one Problem per query row would duplicate q; instead reuse the decode
@@ -287,7 +288,7 @@ int oracle_paged_prefill(const uint16_t* q, const uint16_t* k_cache, const uint1
       row_pos[q_start[i] + j] = seq_lens[i] - n + j;
     }
   }
-  const Problem p{q, k_cache, v_cache, block_tables, seq_lens, T, H, D, S, NB, MB, scale, dtype, H};
+  const Problem p{q, k_cache, v_cache, block_tables, seq_lens, T, H, D, S, NB, MB, scale, dtype, Hkv};
   if (!valid_problem(p) || !out) return 1;
   return parallel_for(T * H, n_threads, [&](int64_t k) {
     const int64_t t = k / H, h = k % H;

@@ -306,3 +306,26 @@ def test_prefill_equals_causal_sdpa(oracle_lib, ctx):
     dec = oracle_decode.paged_decode(last, kc, vc, bt, sl, 0.2)
     for i in range(len(news)):
         assert np.array_equal(got[q_start[i + 1] - 1], dec[i])
+
+
+def test_prefill_grouped_heads_equal_sdpa_gqa(oracle_lib):
+    """Grouped KV heads in prefill: query head h reads KV head h // G; equal to
+    torch SDPA with enable_gqa and the shifted causal mask."""
+    gen = torch.Generator().manual_seed(11)
+    H, Hkv, D, S = 6, 2, 16, 4
+    ctx, news = [3, 0], [7, 10]
+    lens = [c + n for c, n in zip(ctx, news)]
+    ks = [torch.randn(L, Hkv, D, generator=gen).to(torch.float16) for L in lens]
+    vs = [torch.randn(L, Hkv, D, generator=gen).to(torch.float16) for L in lens]
+    kc, vc, bt, sl = make_paged(ks, vs, S, 3, gen)
+    q = torch.randn(sum(news), H, D, generator=gen).to(torch.float16)
+    q_start = torch.tensor([0, news[0], sum(news)], dtype=torch.int32)
+    got = oracle_decode.paged_prefill(q, kc, vc, bt, sl, q_start, 0.3)
+    for i, (L, n) in enumerate(zip(lens, news)):
+        qi = q[q_start[i]:q_start[i + 1]].double().transpose(0, 1)
+        ki, vi = ks[i].double().transpose(0, 1), vs[i].double().transpose(0, 1)
+        mask = torch.arange(L).unsqueeze(0) <= torch.arange(L - n, L).unsqueeze(1)
+        want = F.scaled_dot_product_attention(qi, ki, vi, attn_mask=mask, scale=0.3,
+                                              enable_gqa=True)
+        np.testing.assert_allclose(got[q_start[i]:q_start[i + 1]], want.transpose(0, 1).numpy(),
+                                   rtol=1e-12, atol=1e-12)
