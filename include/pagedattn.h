@@ -141,6 +141,46 @@ pa_status pa_decode_append(void* out, pa_dtype out_dt, const void* q, const void
                            void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Paged prefill attention ("vLLM KV Cache and PagedAttention Explained", Step 6
+ * "Prefill and Decode": every prompt token is processed at once, and each one
+ * attends to the tokens before it and to itself; the attention formula of its
+ * Appendix). Request i holds L = seq_lens[i] tokens in the cache, of which the
+ * last n = q_start[i+1] - q_start[i] are new and already appended (for example
+ * by pa_kv_append); the first L - n are context cached earlier (a plain prompt
+ * has none). New token j of request i sits at position L - n + j and
+ *   out[q_start[i] + j, h] = softmax_t(scale * q[q_start[i] + j, h] . K_t) V_t
+ * over cache tokens t = 0 .. L - n + j, read through block_tables[i] as in
+ * pa_decode; query head h reads KV head h / (H / Hkv).
+ *
+ * out        [T, H, D] device, out_dt (F32, F16, BF16), 16-byte aligned.
+ * q          [T, H, D] device, dt (F16 or BF16), 16-byte aligned; the rows of
+ *            all requests packed back to back.
+ * k_cache,   [NB, Hkv, S, D] device, dt, 16-byte aligned; read only.
+ * v_cache
+ * block_tables [B, MB] int32 device; seq_lens [B] int32 device.
+ * q_start    [B + 1] int32 device: q_start[0] = 0, non-decreasing, q_start[B] = T.
+ * T          rows of q and out (host copy of q_start[B]).
+ * max_q_len  host bound on q_start[i+1] - q_start[i]; sets the launch grid.
+ * D          64 or 128; S one of 8, 16, 32, 64, 128; NB * Hkv * S <= 2^31 - 1.
+ * scale      finite and > 0 (the usual 1 / sqrt(D)).
+ * The contraction runs on the tensor cores with fp32 accumulation; for bf16
+ * the softmax weights enter the second product as two bf16 terms (value and
+ * rounding residue), for f16 as one f16 term.
+ * Errors: PA_ERR_INVALID for bad sizes, dtypes, null or misaligned pointers
+ * (nothing launched); B, T or max_q_len of 0 is a no-op. On the device, a
+ * request whose seq_lens/q_start are inconsistent (n < 0, n > L, L > MB * S,
+ * rows outside [0, T), n > max_q_len) is skipped with PA_DEVERR_SEQ_LEN, a table
+ * entry outside [0, NB) is skipped with PA_DEVERR_BLOCK_ID (that request's
+ * output is then undefined), and a wait that exceeds about a second sets
+ * PA_DEVERR_TIMEOUT; see pa_get_device_error. Asynchronous on `stream`.
+ * ------------------------------------------------------------------------- */
+pa_status pa_prefill(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
+                     const void* v_cache, const int32_t* block_tables, int MB,
+                     const int32_t* seq_lens, const int32_t* q_start, float scale, int B, int H,
+                     int Hkv, int D, int S, int NB, pa_dtype dt, int T, int max_q_len,
+                     void* stream);
+
+/* ---------------------------------------------------------------------------
  * Grouped-query decode (not on the pages, which have one KV head per query
  * head): the cache holds Hkv KV heads, [NB, Hkv, S, D]; q and out hold H query
  * heads, H a multiple of Hkv, and query head h reads KV head h / (H / Hkv)

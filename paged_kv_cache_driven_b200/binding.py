@@ -38,6 +38,10 @@ _SIGNATURES = {
                        _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_decode_noalloc": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32,
                            _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    # out, out_dt, q, k_cache, v_cache, block_tables, MB, seq_lens, q_start, scale,
+    # B, H, Hkv, D, S, NB, dt, T, max_q_len, stream
+    "pa_prefill": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_float, _i32, _i32,
+                    _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "pa_stepper_create": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                            ctypes.c_float, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
     "pa_stepper_destroy": ([_vp], None),
@@ -213,6 +217,29 @@ def pa_decode_gqa(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_s
                                _ptr(seq_lens), float(scale), B, H, Hkv, D, S, NB, _DT[q.dtype],
                                int(partition), int(max_seq_len), _ptr(workspace), ws_bytes,
                                _stream(stream)), "pa_decode_gqa")
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, q_start, scale, max_q_len,
+               stream=None):
+    """Causal paged prefill attention: q/out [T, H, D] packed by request
+    (request i's rows q_start[i] .. q_start[i+1] - 1, the last of its seq_lens[i]
+    cached tokens); caches [NB, Hkv, S, D]; q_start int32 [B + 1] on the device."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                 ("block_tables", block_tables), ("seq_lens", seq_lens), ("q_start", q_start)):
+        _cuda(t, n)
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32 or \
+            q_start.dtype != torch.int32:
+        raise ValueError("block_tables, seq_lens and q_start must be int32")
+    T, H, D = q.shape
+    NB, Hkv, S, _ = k_cache.shape
+    B = seq_lens.numel()
+    if q_start.numel() != B + 1 or tuple(out.shape) != (T, H, D):
+        raise ValueError("q_start must be [B + 1] and out [T, H, D]")
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    _check(lib().pa_prefill(_ptr(out), _DT[out.dtype], _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                            _ptr(block_tables), MB, _ptr(seq_lens), _ptr(q_start), float(scale),
+                            B, H, Hkv, D, S, NB, _DT[q.dtype], T, int(max_q_len),
+                            _stream(stream)), "pa_prefill")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

@@ -17,6 +17,7 @@
 
 #include "pa_append.cuh"
 #include "pa_decode.cuh"
+#include "pa_prefill.cuh"
 #include "pagedattn.h"
 
 namespace {
@@ -241,6 +242,64 @@ pa_status dispatch_out(const pa::DecodeParams& prm, pa_dtype out_dt, int D, int 
   return PA_ERR_INVALID;
 }
 
+// ---- paged prefill -------------------------------------------------------------
+// The packed queries [T, H, D] as a 3-D tensor map (D, H, T) whose box is one
+// 64-element column block of one head for 128 consecutive query rows; rows
+// past T read as zeros.
+bool query_map(CUtensorMap* out, const void* q, int64_t T, int H, int D, pa_dtype dt) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(H) * D * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(out, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+            3, const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, typename TO, int D, int S>
+pa_status launch_prefill(const pa::PrefillParams& prm, const void* q, cudaStream_t stream) {
+  using Tl = pa::PrefillTiling<D, std::is_same<T, __nv_bfloat16>::value>;
+  auto kern = pa::paged_prefill_kernel<T, TO, D, S>;
+  static bool configured[kMaxDevices] = {};
+  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
+  const pa_dtype dt = std::is_same<T, __half>::value ? PA_F16 : PA_BF16;
+  const int64_t rows = static_cast<int64_t>(prm.NB) * prm.Hkv * S;
+  CUtensorMap tmq, tmk, tmv;
+  if (!query_map(&tmq, q, prm.T, prm.H, D, dt) || !row_map(&tmk, prm.k_cache, rows, D, S, dt) ||
+      !row_map(&tmv, prm.v_cache, rows, D, S, dt))
+    return PA_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(ceil_div(prm.max_q_len, Tl::BM)), prm.H, prm.B);
+  kern<<<grid, Tl::THREADS, Tl::SMEM, stream>>>(prm, tmq, tmk, tmv);
+  return cuda_status();
+}
+
+template <typename T, typename TO>
+pa_status dispatch_prefill_shape(const pa::PrefillParams& prm, const void* q, int D, int S,
+                                 cudaStream_t st) {
+#define PA_CASE(DD, SS) \
+  if (D == DD && S == SS) return launch_prefill<T, TO, DD, SS>(prm, q, st);
+  PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32) PA_CASE(64, 64) PA_CASE(64, 128)
+  PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32) PA_CASE(128, 64) PA_CASE(128, 128)
+#undef PA_CASE
+  return PA_ERR_INVALID;
+}
+
+template <typename T>
+pa_status dispatch_prefill(const pa::PrefillParams& prm, const void* q, pa_dtype out_dt, int D,
+                           int S, cudaStream_t st) {
+  switch (out_dt) {
+    case PA_F32: return dispatch_prefill_shape<T, float>(prm, q, D, S, st);
+    case PA_F16: return dispatch_prefill_shape<T, __half>(prm, q, D, S, st);
+    case PA_BF16: return dispatch_prefill_shape<T, __nv_bfloat16>(prm, q, D, S, st);
+  }
+  return PA_ERR_INVALID;
+}
+
 }  // namespace
 
 extern "C" {
@@ -418,6 +477,44 @@ pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k
   return decode_impl(out, out_dt, q, B > 0 ? k_new : nullptr, v_new, k_cache, v_cache,
                      block_tables, MB, seq_lens, scale, B, H, Hkv, D, S, NB, dt, partition,
                      max_seq_len, workspace, ws_bytes, stream);
+}
+
+pa_status pa_prefill(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
+                     const void* v_cache, const int32_t* block_tables, int MB,
+                     const int32_t* seq_lens, const int32_t* q_start, float scale, int B, int H,
+                     int Hkv, int D, int S, int NB, pa_dtype dt, int T, int max_q_len,
+                     void* stream) {
+  if (B < 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || T < 0 || max_q_len < 0 || MB < 0 || NB < 0)
+    return PA_ERR_INVALID;
+  if (!cache_dtype_ok(dt) || !out_dtype_ok(out_dt)) return PA_ERR_INVALID;
+  if (!(D == 64 || D == 128) || !(S == 8 || S == 16 || S == 32 || S == 64 || S == 128))
+    return PA_ERR_INVALID;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return PA_ERR_INVALID;
+  if (B == 0 || T == 0 || max_q_len == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !q_start)
+    return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  if (NB == 0 || static_cast<int64_t>(NB) * Hkv * S > INT_MAX) return PA_ERR_INVALID;
+  if (ceil_div(max_q_len, 128) > INT_MAX / 2 || H > 65535 || B > 65535) return PA_ERR_INVALID;
+  pa::PrefillParams prm;
+  prm.out = out;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.block_tables = block_tables;
+  prm.seq_lens = seq_lens;
+  prm.q_start = q_start;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.MB = MB;
+  prm.B = B;
+  prm.H = H;
+  prm.Hkv = Hkv;
+  prm.NB = NB;
+  prm.T = T;
+  prm.max_q_len = max_q_len;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dt == PA_BF16 ? dispatch_prefill<__nv_bfloat16>(prm, q, out_dt, D, S, st)
+                       : dispatch_prefill<__half>(prm, q, out_dt, D, S, st);
 }
 
 pa_status pa_get_device_error(void* stream, uint32_t* flags) {

@@ -1,0 +1,489 @@
+// Paged prefill attention on the fifth-generation tensor cores.
+//
+// What it computes ("vLLM KV Cache and PagedAttention Explained", Step 6
+// "Prefill and Decode", and the attention formula of its Appendix): request i
+// holds seq_lens[i] = L tokens in the paged cache, the last n = q_start[i+1] -
+// q_start[i] of them new (already appended). New token j sits at position
+// L - n + j and attends, causally, to cache tokens 0 .. L - n + j:
+//   out[q_start[i] + j, h] = softmax_t(scale * q . K_t) V_t over those tokens,
+// K_t / V_t read through the block table (token t in block
+// block_tables[i][t / S], slot t % S), query head h reading KV head h / (H / Hkv).
+//
+// One CTA per (128-row query tile, query head, request), 192 threads in three
+// roles:
+//   warps 0-3  softmax: thread r owns query row r of the tile (tensor-memory
+//              lane r); reads the score tile from tensor memory, keeps the
+//              running max / sum in fp32, writes P to shared memory as 16-bit
+//              (bf16 as hi + lo halves, so the weights keep ~16 bits), rescales
+//              the output accumulator in tensor memory when its max grows;
+//   warp 4     producer: TMA loads of the Q tile and of 128-key K / V tiles,
+//              one box per (block, 64-column block), two stages;
+//   warp 5     MMA issuer (one thread) and tensor-memory owner:
+//              S = Q K^T (M = 128, N = 128, both operands K-major) and
+//              O += P V (V as an MN-major operand), fp32 accumulators in tensor
+//              memory (S in columns 0-127, O in columns 128 ..).
+// All shared tiles use the 128-byte swizzle, so the TMA boxes land directly in
+// the canonical operand layout. Every wait is bounded (about a second); a
+// timeout sets PA_DEVERR_TIMEOUT, stops all roles, waits for the copies and
+// MMAs in flight and frees tensor memory.
+#pragma once
+
+#include <cuda.h>
+
+#include "pa_device.cuh"
+#include "pa_tcgen05.cuh"
+
+namespace pa {
+
+struct PrefillParams {
+  void* out;                    // [T, H, D] TO
+  const void* k_cache;          // [NB, Hkv, S, D] T
+  const void* v_cache;
+  const int32_t* block_tables;  // [B, MB]
+  const int32_t* seq_lens;      // [B] tokens in the cache, new ones included
+  const int32_t* q_start;       // [B + 1] first query row of each request
+  float scale_log2;             // scale * log2(e)
+  int MB, B, H, Hkv, NB, T, max_q_len;
+};
+
+template <int D, bool LO>
+struct PrefillTiling {
+  static constexpr int BM = 128;              // query rows per tile (MMA M)
+  static constexpr int BN = 128;              // keys per tile
+  static constexpr int NSTG = 2;              // K / V stages
+  static constexpr int COLB = D / 64;         // 64-element (128-byte) column blocks
+  static constexpr int CB_BYTES = 128 * 128;  // one column block of 128 rows
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NSTG * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + NSTG * KV_BYTES;
+  static constexpr int OFF_PLO = OFF_P + P_BYTES;
+  static constexpr int OFF_BAR = OFF_PLO + (LO ? P_BYTES : 0);
+  static constexpr int SMEM = 1024 + OFF_BAR + 256;  // + alignment slack, barriers
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t TMEM_COLS = 256;  // S: 128 columns, O: D columns
+  static_assert(D == 64 || D == 128, "head size 64 or 128");
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+};
+
+// mbarrier wait bounded by time and by the CTA's abort flag.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort_flag = 1;
+      raise_error(PA_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d_nohint(void* dst, const void* tmap, int x, int y,
+                                                   uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack_pair(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack_pair<__nv_bfloat16>(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+template <>
+__device__ __forceinline__ uint32_t pack_pair<__half>(float a, float b) {
+  const __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 2^x with the hardware approximation (relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <typename TO>
+__device__ __forceinline__ void store_row32(TO* dst, const float (&v)[32]);
+template <>
+__device__ __forceinline__ void store_row32<float>(float* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    reinterpret_cast<float4*>(dst)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2],
+                                                    v[4 * k + 3]);
+}
+template <>
+__device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst,
+                                                           const float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    reinterpret_cast<uint4*>(dst)[k] = make_uint4(
+        pack_pair<__nv_bfloat16>(v[8 * k], v[8 * k + 1]),
+        pack_pair<__nv_bfloat16>(v[8 * k + 2], v[8 * k + 3]),
+        pack_pair<__nv_bfloat16>(v[8 * k + 4], v[8 * k + 5]),
+        pack_pair<__nv_bfloat16>(v[8 * k + 6], v[8 * k + 7]));
+}
+template <>
+__device__ __forceinline__ void store_row32<__half>(__half* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    reinterpret_cast<uint4*>(dst)[k] =
+        make_uint4(pack_pair<__half>(v[8 * k], v[8 * k + 1]),
+                   pack_pair<__half>(v[8 * k + 2], v[8 * k + 3]),
+                   pack_pair<__half>(v[8 * k + 4], v[8 * k + 5]),
+                   pack_pair<__half>(v[8 * k + 6], v[8 * k + 7]));
+}
+
+template <typename T, typename TO, int D, int S>
+__global__ void __launch_bounds__(192, 1)
+    paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmq,
+                         const __grid_constant__ CUtensorMap tmk,
+                         const __grid_constant__ CUtensorMap tmv) {
+  constexpr bool LO = std::is_same<T, __nv_bfloat16>::value;
+  using Tl = PrefillTiling<D, LO>;
+  constexpr int BPT = Tl::BN / S;  // cache blocks per key tile
+  static_assert(S >= 8 && S <= 128 && Tl::BN % S == 0, "block size 8 .. 128, dividing 128");
+
+  const int i = blockIdx.z, h = blockIdx.y;
+  const int L = p.seq_lens[i];
+  const int q0 = p.q_start[i], q1 = p.q_start[i + 1];
+  const int n = q1 - q0;
+  if (L < 0 || L > static_cast<int64_t>(p.MB) * S || n < 0 || n > L || q0 < 0 || q1 > p.T ||
+      n > p.max_q_len) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) raise_error(PA_DEVERR_SEQ_LEN);
+    return;
+  }
+  const int ntq = (n + Tl::BM - 1) / Tl::BM;
+  const int qt = ntq - 1 - static_cast<int>(blockIdx.x);  // longest tiles first
+  if (qt < 0) return;
+  const int row0 = qt * Tl::BM;
+  const int ctx = L - n;  // tokens cached before the first new one
+  const int last_pos = ctx + min(n, row0 + Tl::BM) - 1;
+  const int ntk = last_pos / Tl::BN + 1;  // key tiles this query tile needs
+  const int hk = h / (p.H / p.Hkv);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = sm;
+  uint8_t* sK = sm + Tl::OFF_K;
+  uint8_t* sV = sm + Tl::OFF_V;
+  uint8_t* sP = sm + Tl::OFF_P;
+  uint8_t* sPlo = sm + Tl::OFF_PLO;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Tl::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;                 // [NSTG]
+  uint64_t* v_full = k_full + Tl::NSTG;        // [NSTG]
+  uint64_t* kv_empty = v_full + Tl::NSTG;      // [NSTG]
+  uint64_t* s_full = kv_empty + Tl::NSTG;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_free + 1;
+  uint64_t* o_done = p_full + 1;
+  uint64_t* mma_done = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < Tl::NSTG; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    __syncwarp();
+    tc::tmem_alloc(tmem_slot, Tl::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + Tl::BN;
+
+  if (warp == 4) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int last_j[Tl::NSTG];
+#pragma unroll
+      for (int s = 0; s < Tl::NSTG; ++s) last_j[s] = -1;
+      mbar_arrive_expect_tx(q_full, Tl::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < Tl::COLB; ++c)
+        tc::tma_load_3d(sQ + c * Tl::CB_BYTES, &tmq, c * 64, h, q0 + row0, q_full);
+      const int nblk = (L + S - 1) / S;
+      const int32_t* table = p.block_tables + static_cast<int64_t>(i) * p.MB;
+      for (int j = 0; j < ntk; ++j) {
+        const int st = j % Tl::NSTG;
+        if (j >= Tl::NSTG && !wait_or_abort(&kv_empty[st], ((j / Tl::NSTG) - 1) & 1, abort_flag))
+          break;
+        int ids[BPT];
+        int nvalid = 0;
+#pragma unroll
+        for (int b = 0; b < BPT; ++b) {
+          const int lb = j * BPT + b;
+          int id = -1;
+          if (lb < nblk) {
+            id = table[lb];
+            if (id < 0 || id >= p.NB) {
+              raise_error(PA_DEVERR_BLOCK_ID);
+              id = -1;
+            }
+          }
+          ids[b] = id;
+          nvalid += id >= 0;
+        }
+        const uint32_t bytes = static_cast<uint32_t>(nvalid) * S * 128 * Tl::COLB;
+        uint8_t* dk = sK + st * Tl::KV_BYTES;
+        uint8_t* dv = sV + st * Tl::KV_BYTES;
+        mbar_arrive_expect_tx(&k_full[st], bytes);
+#pragma unroll
+        for (int b = 0; b < BPT; ++b) {
+          if (ids[b] < 0) continue;
+          const int y = (ids[b] * p.Hkv + hk) * S;
+#pragma unroll
+          for (int c = 0; c < Tl::COLB; ++c)
+            tma_load_2d_nohint(dk + c * Tl::CB_BYTES + b * S * 128, &tmk, c * 64, y, &k_full[st]);
+        }
+        mbar_arrive_expect_tx(&v_full[st], bytes);
+#pragma unroll
+        for (int b = 0; b < BPT; ++b) {
+          if (ids[b] < 0) continue;
+          const int y = (ids[b] * p.Hkv + hk) * S;
+#pragma unroll
+          for (int c = 0; c < Tl::COLB; ++c)
+            tma_load_2d_nohint(dv + c * Tl::CB_BYTES + b * S * 128, &tmv, c * 64, y, &v_full[st]);
+        }
+        last_j[st] = j;
+      }
+      // copies in flight land before the CTA can exit
+      mbar_wait_bounded(q_full, 0);
+#pragma unroll
+      for (int s = 0; s < Tl::NSTG; ++s)
+        if (last_j[s] >= 0) {
+          const uint32_t par = (last_j[s] / Tl::NSTG) & 1;
+          mbar_wait_bounded(&k_full[s], par);
+          mbar_wait_bounded(&v_full[s], par);
+        }
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr int fmt = LO ? 1 : 0;
+      constexpr uint32_t idesc_s = tc::instr_desc_f16(fmt, 0, 0, Tl::BM, Tl::BN);
+      constexpr uint32_t idesc_o = tc::instr_desc_f16(fmt, 0, 1, Tl::BM, D);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      const uint32_t aP = smem_u32(sP), aPlo = smem_u32(sPlo);
+      bool ok = wait_or_abort(q_full, 0, abort_flag);
+      for (int j = 0; ok && j <= ntk; ++j) {
+        if (j < ntk) {
+          const int st = j % Tl::NSTG;
+          if (!wait_or_abort(&k_full[st], (j / Tl::NSTG) & 1, abort_flag)) break;
+          if (j > 0 && !wait_or_abort(s_free, (j - 1) & 1, abort_flag)) break;
+          tc::fence_after_sync();
+          const uint32_t kb = aK + st * Tl::KV_BYTES;
+#pragma unroll
+          for (int s = 0; s < D / 16; ++s) {
+            const uint32_t off = (s >> 2) * Tl::CB_BYTES + (s & 3) * 32;
+            tc::mma_ss(tS, tc::smem_desc_sw128(aQ + off, 16, 1024),
+                       tc::smem_desc_sw128(kb + off, 16, 1024), idesc_s, s > 0);
+          }
+          tc::commit(s_full);
+        }
+        if (j > 0) {
+          const int jj = j - 1, st = jj % Tl::NSTG;
+          if (!wait_or_abort(&v_full[st], (jj / Tl::NSTG) & 1, abort_flag)) break;
+          if (!wait_or_abort(p_full, jj & 1, abort_flag)) break;
+          tc::fence_after_sync();
+          const uint32_t vb = aV + st * Tl::KV_BYTES;
+#pragma unroll
+          for (int s = 0; s < Tl::BN / 16; ++s) {
+            const uint32_t poff = (s >> 2) * Tl::CB_BYTES + (s & 3) * 32;
+            const uint64_t bdesc = tc::smem_desc_sw128(vb + s * 16 * 128, Tl::CB_BYTES, 1024);
+            tc::mma_ss(tO, tc::smem_desc_sw128(aP + poff, 16, 1024), bdesc, idesc_o,
+                       jj > 0 || s > 0);
+            if constexpr (LO)
+              tc::mma_ss(tO, tc::smem_desc_sw128(aPlo + poff, 16, 1024), bdesc, idesc_o, true);
+          }
+          tc::commit(o_done);
+          tc::commit(&kv_empty[st]);
+        }
+      }
+      // every MMA issued has completed before tensor memory is released
+      tc::commit(mma_done);
+      mbar_wait_bounded(mma_done, 0);
+    }
+  } else {
+    // ---------------- softmax (warps 0-3, thread r = row r) ----------------
+    const int r = threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int qrow = row0 + r;
+    const int lim = min(ctx + qrow, L - 1);  // last key this row sees
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntk; ++j) {
+      ok = wait_or_abort(s_full, j & 1, abort_flag);
+      if (!__all_sync(kFullMask, ok)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      float x[Tl::BN];
+#pragma unroll
+      for (int c4 = 0; c4 < Tl::BN / 32; ++c4) {
+        uint32_t u[32];
+        tc::tmem_ld32(tS + lane_base + c4 * 32, u);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c4 * 32 + c] = __uint_as_float(u[c]);
+      }
+      tc::fence_before_sync();
+      mbar_arrive(s_free);
+      const int kb = j * Tl::BN;
+      // keys past this row's last one read as -inf (scale > 0, so the order of
+      // raw scores is the order of scaled ones)
+      if (kb + Tl::BN - 1 > lim) {
+#pragma unroll
+        for (int c = 0; c < Tl::BN; ++c) x[c] = kb + c <= lim ? x[c] : -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = x[k];
+#pragma unroll
+      for (int c = 8; c < Tl::BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+      const float tmax =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
+      // The reference max only moves when the tile max exceeds it by more than
+      // 2^8 in weight; the weights stay <= 256, exact in the final ratio.
+      const float m_new = fmaxf(m, tmax);
+      const bool grow = m_new > m + 8.f;
+      const float m_use = grow ? m_new : m;
+      const float alpha = grow ? fast_exp2(m - m_use) : 1.f;
+      float sm8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
+#pragma unroll
+      for (int c = 0; c < Tl::BN; ++c) {
+        x[c] = fast_exp2(fmaf(x[c], p.scale_log2, -m_use));
+        sm8[c & 7] += x[c];
+      }
+      l = l * alpha + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
+                       ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
+      m = m_use;
+      if (j > 0) {
+        ok = wait_or_abort(o_done, (j - 1) & 1, abort_flag);
+        if (!__all_sync(kFullMask, ok)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+      }
+      // P -> shared memory, K-major with the 128-byte swizzle; for bf16 also
+      // the rounding residue p - bf16(p), itself rounded to bf16
+#pragma unroll
+      for (int cb = 0; cb < Tl::BN / 64; ++cb) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const float* v = &x[cb * 64 + cc * 8];
+          const int off = cb * Tl::CB_BYTES + r * 128 + ((cc ^ (r & 7)) << 4);
+          uint32_t hi[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) hi[e] = pack_pair<T>(v[2 * e], v[2 * e + 1]);
+          *reinterpret_cast<uint4*>(sP + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          if constexpr (LO) {
+            uint32_t lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              // bf16 pair -> the two fp32 values it holds: exact bit moves
+              const float h0 = __uint_as_float(hi[e] << 16);
+              const float h1 = __uint_as_float(hi[e] & 0xffff0000u);
+              lo[e] = pack_pair<T>(v[2 * e] - h0, v[2 * e + 1] - h1);
+            }
+            *reinterpret_cast<uint4*>(sPlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
+        }
+      }
+      // rescale the accumulator rows whose reference max moved
+      if (j > 0 && __any_sync(kFullMask, grow)) {
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          uint32_t u[32];
+          tc::tmem_ld32(tO + lane_base + c4 * 32, u);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+          tc::tmem_st32(tO + lane_base + c4 * 32, u);
+        }
+        tc::tmem_wait_st();
+      }
+      // keys past the end of the request: zero their V rows (P is 0 there, and
+      // 0 * NaN would not be)
+      if (j == ntk - 1 && kb + r >= L) {
+        const int st = j % Tl::NSTG;
+        ok = wait_or_abort(&v_full[st], (j / Tl::NSTG) & 1, abort_flag);
+        if (ok) {
+          uint8_t* row = sV + st * Tl::KV_BYTES + r * 128;
+#pragma unroll
+          for (int c = 0; c < Tl::COLB; ++c)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              reinterpret_cast<uint4*>(row + c * Tl::CB_BYTES)[k] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (!__all_sync(kFullMask, ok)) {
+        ok = false;
+        break;
+      }
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(p_full);
+    }
+    // epilogue: O / l -> out
+    if (ok) ok = wait_or_abort(o_done, (ntk - 1) & 1, abort_flag);
+    if (__all_sync(kFullMask, ok)) {
+      tc::fence_after_sync();
+      const float inv = 1.f / l;
+      TO* dst = reinterpret_cast<TO*>(p.out) +
+                (static_cast<int64_t>(q0 + qrow) * p.H + h) * D;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t u[32];
+        tc::tmem_ld32(tO + lane_base + c4 * 32, u);
+        tc::tmem_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(u[c]) * inv;
+        if (qrow < n) store_row32<TO>(dst + c4 * 32, v);
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Tl::TMEM_COLS);
+  }
+}
+
+}  // namespace pa

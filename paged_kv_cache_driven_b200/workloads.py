@@ -156,6 +156,47 @@ def sweep_case(S, D, B, dtype, seed=0, device="cpu", H=32, lo=16, hi=8192):
 
 
 @dataclass
+class PrefillCase:
+    """Prefill inputs: the cache already holds every request's tokens (context
+    and new), q [T, H, D] packs the new tokens' queries request after request."""
+
+    cache: DecodeCase        # caches, tables, seq_lens (total tokens per request)
+    q: torch.Tensor          # [T, H, D]
+    q_start: torch.Tensor    # [B + 1] int32, on the device
+    new_lens: list           # new tokens per request
+    ctx_lens: list           # tokens cached before them
+
+    @property
+    def max_q_len(self):
+        return max(self.new_lens + [0])
+
+
+def prefill_case(ctx_lens, new_lens, H, D, S, dtype, seed, device, Hkv=None, pool_blocks=None):
+    """Request i has ctx_lens[i] tokens cached earlier and new_lens[i] new ones,
+    all already in the (poisoned, permuted) cache; q holds the new tokens' queries."""
+    lens = [int(c) + int(n) for c, n in zip(ctx_lens, new_lens)]
+    cache = decode_case(lens, H=H, D=D, S=S, dtype=dtype, seed=seed, device=device, Hkv=Hkv,
+                        pool_blocks=pool_blocks)
+    T = sum(int(n) for n in new_lens)
+    g = _dev_gen(seed + 77, device)
+    q = torch.randn((T, H, D), generator=g, device=device, dtype=torch.float32).to(dtype)
+    starts = [0]
+    for n in new_lens:
+        starts.append(starts[-1] + int(n))
+    return PrefillCase(cache=cache, q=q, q_start=torch.tensor(starts, dtype=torch.int32,
+                                                               device=device),
+                       new_lens=[int(n) for n in new_lens], ctx_lens=[int(c) for c in ctx_lens])
+
+
+def prompt_prefill(seed=0, device="cpu", n_req=16, lo=512, hi=4096, H=32, D=128, S=16,
+                   dtype=torch.bfloat16):
+    """Prompt prefill attention: 16 prompts of uniform [512, 4096] tokens, no
+    earlier context, 32 heads, head_dim 128, block 16, bf16, permuted pool."""
+    n_tok = torch.randint(lo, hi + 1, (n_req,), generator=_cpu_gen(seed)).tolist()
+    return prefill_case([0] * n_req, n_tok, H=H, D=D, S=S, dtype=dtype, seed=seed, device=device)
+
+
+@dataclass
 class AppendCase:
     """Tokens to scatter: k, v [T, H, D], plus where each request's tokens go."""
 

@@ -102,3 +102,54 @@ def sample_pairs(case, n, seed=0):
         h = int(torch.randint(0, H, (1,), generator=g))
         picks.append((i, h))
     return picks[:n]
+
+
+def run_prefill(pc, out_dtype=torch.float32, max_q_len=None, stream=None):
+    """pa_prefill on a workloads.PrefillCase; returns out [T, H, D]."""
+    T, H, D = pc.q.shape
+    out = torch.empty((T, H, D), dtype=out_dtype, device=pc.q.device)
+    c = pc.cache
+    binding.pa_prefill(out, pc.q, c.k_cache, c.v_cache, c.block_tables, c.seq_lens, pc.q_start,
+                       c.scale, pc.max_q_len if max_q_len is None else max_q_len, stream=stream)
+    return out
+
+
+def oracle_prefill_full(pc, threads=0):
+    """The oracle's causal prefill over a whole small case."""
+    c = pc.cache
+    return oracle_decode.paged_prefill(pc.q.cpu(), c.k_cache.cpu(), c.v_cache.cpu(),
+                                       c.block_tables.cpu(), c.seq_lens.cpu(), pc.q_start.cpu(),
+                                       c.scale, threads=threads)
+
+
+def oracle_prefill_rows(pc, picks, threads=0):
+    """The oracle on sampled (request, new-token index, head) triples of a case of
+    any size. Row j of request i is the decode of that query over the first
+    ctx_i + j + 1 cached tokens (the oracle's pins show the two agree), so each
+    triple becomes a one-head decode over only the blocks it reads. Returns
+    [len(picks), D] fp64."""
+    c = pc.cache
+    S = c.k_cache.shape[2]
+    D = pc.q.shape[2]
+    G = pc.q.shape[1] // c.k_cache.shape[1]
+    qs = pc.q_start.cpu().tolist()
+    ks, vs, qrows, tables, lens = [], [], [], [], []
+    off = 0
+    for i, j, h in picks:
+        L = pc.ctx_lens[i] + j + 1
+        blocks = c.tables_host[i][: -(-L // S)]
+        idx = torch.tensor(blocks, dtype=torch.long, device=c.k_cache.device)
+        ks.append(c.k_cache[idx, h // G].unsqueeze(1).cpu())
+        vs.append(c.v_cache[idx, h // G].unsqueeze(1).cpu())
+        qrows.append(pc.q[qs[i] + j, h].view(1, 1, D).cpu())
+        tables.append(list(range(off, off + len(blocks))))
+        lens.append(L)
+        off += len(blocks)
+    MB = max(len(t) for t in tables)
+    bt = torch.full((len(picks), MB), -1, dtype=torch.int32)
+    for r, t in enumerate(tables):
+        bt[r, :len(t)] = torch.tensor(t, dtype=torch.int32)
+    out = oracle_decode.paged_decode(torch.cat(qrows), torch.cat(ks), torch.cat(vs), bt,
+                                     torch.tensor(lens, dtype=torch.int32), c.scale,
+                                     threads=threads)
+    return out[:, 0, :]
