@@ -273,7 +273,7 @@ pa_status launch_prefill(const pa::PrefillParams& prm, const void* q, cudaStream
   if (!query_map(&tmq, q, prm.T, prm.H, D, dt) || !row_map(&tmk, prm.k_cache, rows, D, S, dt) ||
       !row_map(&tmv, prm.v_cache, rows, D, S, dt))
     return PA_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>(ceil_div(prm.max_q_len, Tl::BM)), prm.H, prm.B);
+  const dim3 grid(static_cast<unsigned>(ceil_div(prm.max_q_len, Tl::NQT * Tl::BM)), prm.H, prm.B);
   kern<<<grid, Tl::THREADS, Tl::SMEM, stream>>>(prm, tmq, tmk, tmv);
   return cuda_status();
 }

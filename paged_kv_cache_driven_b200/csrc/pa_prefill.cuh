@@ -9,23 +9,28 @@
 // K_t / V_t read through the block table (token t in block
 // block_tables[i][t / S], slot t % S), query head h reading KV head h / (H / Hkv).
 //
-// One CTA per (128-row query tile, query head, request), 192 threads in three
-// roles:
-//   warps 0-3  softmax: thread r owns query row r of the tile (tensor-memory
-//              lane r); reads the score tile from tensor memory, keeps the
-//              running max / sum in fp32, writes P to shared memory as 16-bit
-//              (bf16 as hi + lo halves, so the weights keep ~16 bits), rescales
-//              the output accumulator in tensor memory when its max grows;
-//   warp 4     producer: TMA loads of the Q tile and of 128-key K / V tiles,
-//              one box per (block, 64-column block), two stages;
-//   warp 5     MMA issuer (one thread) and tensor-memory owner:
-//              S = Q K^T (M = 128, N = 128, both operands K-major) and
-//              O += P V (V as an MN-major operand), fp32 accumulators in tensor
-//              memory (S in columns 0-127, O in columns 128 ..).
-// All shared tiles use the 128-byte swizzle, so the TMA boxes land directly in
-// the canonical operand layout. Every wait is bounded (about a second); a
-// timeout sets PA_DEVERR_TIMEOUT, stops all roles, waits for the copies and
-// MMAs in flight and frees tensor memory.
+// One CTA per (256 query rows = two 128-row tiles, query head, request), 320
+// threads in four roles:
+//   warps 0-3, 4-7  softmax for query tile 0 / 1: thread r owns row r of its
+//              tile (tensor-memory lane r); reads the tile's scores from tensor
+//              memory (twice: max, then weights), keeps the running max / sum
+//              in fp32, writes the weights P back over the scores as 16-bit
+//              pairs (bf16 as hi + lo halves, so the weights keep ~16 bits), and
+//              rescales the tile's output accumulator when its reference max
+//              moves;
+//   warp 8     producer: TMA loads of the two Q tiles and of 128-key K / V
+//              tiles, one box per (cache block, 64-column block), two stages;
+//   warp 9     MMA issuer (lane 0) and tensor-memory owner, also zeroing V rows
+//              past the end of the request in the last key tile:
+//              S_t = Q_t K^T (both operands K-major in shared memory) and
+//              O_t += P_t V (P_t from tensor memory, V an MN-major operand),
+//              fp32 accumulators in tensor memory: tile t's S/P in columns
+//              256 t .. 256 t + 127, its O in the next 128.
+// The two tiles ping-pong: while one tile's softmax runs, the tensor cores
+// work on the other tile's products. All shared tiles use the 128-byte swizzle,
+// so the TMA boxes land directly in the canonical operand layout. Every wait is
+// bounded (about a second); a timeout sets PA_DEVERR_TIMEOUT, stops all roles,
+// waits for the copies and MMAs in flight and frees tensor memory.
 #pragma once
 
 #include <cuda.h>
@@ -49,21 +54,21 @@ struct PrefillParams {
 template <int D, bool LO>
 struct PrefillTiling {
   static constexpr int BM = 128;              // query rows per tile (MMA M)
+  static constexpr int NQT = 2;               // query tiles per CTA
   static constexpr int BN = 128;              // keys per tile
   static constexpr int NSTG = 2;              // K / V stages
   static constexpr int COLB = D / 64;         // 64-element (128-byte) column blocks
   static constexpr int CB_BYTES = 128 * 128;  // one column block of 128 rows
-  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int Q_BYTES = BM * D * 2;  // one query tile
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_K = NQT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSTG * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NSTG * KV_BYTES;
-  static constexpr int OFF_PLO = OFF_P + P_BYTES;
-  static constexpr int OFF_BAR = OFF_PLO + (LO ? P_BYTES : 0);
-  static constexpr int SMEM = 1024 + OFF_BAR + 256;  // + alignment slack, barriers
-  static constexpr int THREADS = 192;
-  static constexpr uint32_t TMEM_COLS = 256;  // S: 128 columns, O: D columns
+  static constexpr int OFF_BAR = OFF_V + NSTG * KV_BYTES;
+  // + alignment slack and barriers; at least 120 KB, so that one CTA holds an
+  // SM (it allocates all 512 tensor-memory columns)
+  static constexpr int SMEM = 1024 + OFF_BAR + 256 > 120 * 1024 ? 1024 + OFF_BAR + 256 : 120 * 1024;
+  static constexpr int THREADS = NQT * 128 + 64;
+  static constexpr uint32_t TMEM_COLS = 512;  // per tile: S/P 128 columns, O 128
   static_assert(D == 64 || D == 128, "head size 64 or 128");
   static_assert(SMEM <= 232448, "shared memory per CTA");
 };
@@ -144,8 +149,15 @@ __device__ __forceinline__ void store_row32<__half>(__half* dst, const float (&v
                    pack_pair<__half>(v[8 * k + 6], v[8 * k + 7]));
 }
 
+// All 32 lanes wait; false (for every lane) if any lane's wait failed.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag) {
+  const bool ok = wait_or_abort(bar, parity, abort_flag);
+  return __all_sync(kFullMask, ok);
+}
+
 template <typename T, typename TO, int D, int S>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmq,
                          const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv) {
@@ -163,13 +175,21 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) raise_error(PA_DEVERR_SEQ_LEN);
     return;
   }
-  const int ntq = (n + Tl::BM - 1) / Tl::BM;
-  const int qt = ntq - 1 - static_cast<int>(blockIdx.x);  // longest tiles first
-  if (qt < 0) return;
-  const int row0 = qt * Tl::BM;
+  constexpr int ROWS = Tl::NQT * Tl::BM;
+  const int ncta = (n + ROWS - 1) / ROWS;
+  const int ct = ncta - 1 - static_cast<int>(blockIdx.x);  // longest first
+  if (ct < 0) return;
+  const int row0 = ct * ROWS;
   const int ctx = L - n;  // tokens cached before the first new one
-  const int last_pos = ctx + min(n, row0 + Tl::BM) - 1;
-  const int ntk = last_pos / Tl::BN + 1;  // key tiles this query tile needs
+  // key tiles each query tile needs (0: the tile holds no rows of this request)
+  int nk[Tl::NQT];
+#pragma unroll
+  for (int t = 0; t < Tl::NQT; ++t) {
+    const int first = row0 + t * Tl::BM;
+    nk[t] = first >= n ? 0 : (ctx + min(n, first + Tl::BM) - 1) / Tl::BN + 1;
+  }
+  const int NK = max(nk[0], nk[1]);
+  const int nq = nk[1] > 0 ? 2 : 1;
   const int hk = h / (p.H / p.Hkv);
 
   extern __shared__ uint8_t smem_raw[];
@@ -178,18 +198,15 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sQ = sm;
   uint8_t* sK = sm + Tl::OFF_K;
   uint8_t* sV = sm + Tl::OFF_V;
-  uint8_t* sP = sm + Tl::OFF_P;
-  uint8_t* sPlo = sm + Tl::OFF_PLO;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Tl::OFF_BAR);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;                 // [NSTG]
-  uint64_t* v_full = k_full + Tl::NSTG;        // [NSTG]
-  uint64_t* kv_empty = v_full + Tl::NSTG;      // [NSTG]
-  uint64_t* s_full = kv_empty + Tl::NSTG;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_free + 1;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* mma_done = o_done + 1;
+  uint64_t* k_full = bars + 1;                // [NSTG]
+  uint64_t* v_full = k_full + Tl::NSTG;       // [NSTG]
+  uint64_t* kv_empty = v_full + Tl::NSTG;     // [NSTG]
+  uint64_t* s_full = kv_empty + Tl::NSTG;     // [NQT]
+  uint64_t* p_full = s_full + Tl::NQT;        // [NQT]
+  uint64_t* o_done = p_full + Tl::NQT;        // [NQT]
+  uint64_t* mma_done = o_done + Tl::NQT;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -201,15 +218,16 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    for (int t = 0; t < Tl::NQT; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_done[t], 1);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc::tmem_alloc(tmem_slot, Tl::TMEM_COLS);
     tc::tmem_relinquish();
@@ -218,21 +236,22 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + Tl::BN;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- producer ----------------
     if (lane == 0) {
       int last_j[Tl::NSTG];
 #pragma unroll
       for (int s = 0; s < Tl::NSTG; ++s) last_j[s] = -1;
-      mbar_arrive_expect_tx(q_full, Tl::Q_BYTES);
+      mbar_arrive_expect_tx(q_full, nq * Tl::Q_BYTES);
+      for (int t = 0; t < nq; ++t)
 #pragma unroll
-      for (int c = 0; c < Tl::COLB; ++c)
-        tc::tma_load_3d(sQ + c * Tl::CB_BYTES, &tmq, c * 64, h, q0 + row0, q_full);
+        for (int c = 0; c < Tl::COLB; ++c)
+          tc::tma_load_3d(sQ + t * Tl::Q_BYTES + c * Tl::CB_BYTES, &tmq, c * 64, h,
+                          q0 + row0 + t * Tl::BM, q_full);
       const int nblk = (L + S - 1) / S;
       const int32_t* table = p.block_tables + static_cast<int64_t>(i) * p.MB;
-      for (int j = 0; j < ntk; ++j) {
+      for (int j = 0; j < NK; ++j) {
         const int st = j % Tl::NSTG;
         if (j >= Tl::NSTG && !wait_or_abort(&kv_empty[st], ((j / Tl::NSTG) - 1) & 1, abort_flag))
           break;
@@ -285,91 +304,111 @@ __global__ void __launch_bounds__(192, 1)
           mbar_wait_bounded(&v_full[s], par);
         }
     }
-  } else if (warp == 5) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr int fmt = LO ? 1 : 0;
-      constexpr uint32_t idesc_s = tc::instr_desc_f16(fmt, 0, 0, Tl::BM, Tl::BN);
-      constexpr uint32_t idesc_o = tc::instr_desc_f16(fmt, 0, 1, Tl::BM, D);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      const uint32_t aP = smem_u32(sP), aPlo = smem_u32(sPlo);
-      bool ok = wait_or_abort(q_full, 0, abort_flag);
-      for (int j = 0; ok && j <= ntk; ++j) {
-        if (j < ntk) {
-          const int st = j % Tl::NSTG;
-          if (!wait_or_abort(&k_full[st], (j / Tl::NSTG) & 1, abort_flag)) break;
-          if (j > 0 && !wait_or_abort(s_free, (j - 1) & 1, abort_flag)) break;
-          tc::fence_after_sync();
-          const uint32_t kb = aK + st * Tl::KV_BYTES;
+  } else if (warp == 9) {
+    // ---------------- MMA issuer (lane 0), V tail zeroing (whole warp) ----------------
+    constexpr int fmt = LO ? 1 : 0;
+    constexpr uint32_t idesc_s = tc::instr_desc_f16(fmt, 0, 0, Tl::BM, Tl::BN);
+    constexpr uint32_t idesc_o = tc::instr_desc_f16(fmt, 0, 1, Tl::BM, D);
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+    auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
+      const uint32_t qb = aQ + t * Tl::Q_BYTES;
+      const uint32_t kb = aK + (j % Tl::NSTG) * Tl::KV_BYTES;
 #pragma unroll
-          for (int s = 0; s < D / 16; ++s) {
-            const uint32_t off = (s >> 2) * Tl::CB_BYTES + (s & 3) * 32;
-            tc::mma_ss(tS, tc::smem_desc_sw128(aQ + off, 16, 1024),
-                       tc::smem_desc_sw128(kb + off, 16, 1024), idesc_s, s > 0);
-          }
-          tc::commit(s_full);
-        }
-        if (j > 0) {
-          const int jj = j - 1, st = jj % Tl::NSTG;
-          if (!wait_or_abort(&v_full[st], (jj / Tl::NSTG) & 1, abort_flag)) break;
-          if (!wait_or_abort(p_full, jj & 1, abort_flag)) break;
-          tc::fence_after_sync();
-          const uint32_t vb = aV + st * Tl::KV_BYTES;
+      for (int s = 0; s < D / 16; ++s) {
+        const uint32_t off = (s >> 2) * Tl::CB_BYTES + (s & 3) * 32;
+        tc::mma_ss(tmem + t * 256, tc::smem_desc_sw128(qb + off, 16, 1024),
+                   tc::smem_desc_sw128(kb + off, 16, 1024), idesc_s, s > 0);
+      }
+      tc::commit(&s_full[t]);
+    };
+    bool ok = wait_warp(q_full, 0, abort_flag) && wait_warp(&k_full[0], 0, abort_flag);
+    if (ok) {
+      tc::fence_after_sync();
+      if (lane == 0)
+        for (int t = 0; t < nq; ++t) issue_s(t, 0);
+    }
+    for (int j = 0; ok && j < NK; ++j) {
+      const int st = j % Tl::NSTG;
+      ok = wait_warp(&v_full[st], (j / Tl::NSTG) & 1, abort_flag);
+      if (!ok) break;
+      const int kb = j * Tl::BN;
+      if (j == NK - 1 && kb + Tl::BN > L) {
+        // keys past the end of the request: P is 0 there, and 0 * NaN would not be
+        uint8_t* vs = sV + st * Tl::KV_BYTES;
+        for (int r = max(L - kb, 0) + lane; r < Tl::BN; r += 32)
+#pragma unroll
+          for (int c = 0; c < Tl::COLB; ++c)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              reinterpret_cast<uint4*>(vs + c * Tl::CB_BYTES + r * 128)[k] = make_uint4(0, 0, 0, 0);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+      }
+      const uint32_t vb = aV + st * Tl::KV_BYTES;
+      for (int t = 0; ok && t < Tl::NQT; ++t) {
+        if (j >= nk[t]) continue;
+        ok = wait_warp(&p_full[t], j & 1, abort_flag);
+        if (!ok) break;
+        tc::fence_after_sync();
+        if (lane == 0) {
+          const uint32_t tS = tmem + t * 256, tO = tS + 128;
 #pragma unroll
           for (int s = 0; s < Tl::BN / 16; ++s) {
-            const uint32_t poff = (s >> 2) * Tl::CB_BYTES + (s & 3) * 32;
             const uint64_t bdesc = tc::smem_desc_sw128(vb + s * 16 * 128, Tl::CB_BYTES, 1024);
-            tc::mma_ss(tO, tc::smem_desc_sw128(aP + poff, 16, 1024), bdesc, idesc_o,
-                       jj > 0 || s > 0);
-            if constexpr (LO)
-              tc::mma_ss(tO, tc::smem_desc_sw128(aPlo + poff, 16, 1024), bdesc, idesc_o, true);
+            const uint32_t pa = tS + 32 * (s >> 1) + 8 * (s & 1);  // keys 16s .. 16s + 15
+            tc::mma_ts(tO, pa, bdesc, idesc_o, j > 0 || s > 0);
+            if constexpr (LO) tc::mma_ts(tO, pa + 16, bdesc, idesc_o, true);
           }
-          tc::commit(o_done);
-          tc::commit(&kv_empty[st]);
+          if (j == nk[t] - 1) tc::commit(&o_done[t]);
+        }
+        if (j + 1 < nk[t]) {
+          ok = wait_warp(&k_full[(j + 1) % Tl::NSTG], ((j + 1) / Tl::NSTG) & 1, abort_flag);
+          if (!ok) break;
+          tc::fence_after_sync();
+          if (lane == 0) issue_s(t, j + 1);
         }
       }
-      // every MMA issued has completed before tensor memory is released
+      if (ok && lane == 0) tc::commit(&kv_empty[st]);
+    }
+    // every MMA issued has completed before tensor memory is released
+    if (lane == 0) {
       tc::commit(mma_done);
       mbar_wait_bounded(mma_done, 0);
     }
+    __syncwarp();
   } else {
-    // ---------------- softmax (warps 0-3, thread r = row r) ----------------
-    const int r = threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int qrow = row0 + r;
+    // ---------------- softmax (warps 4t .. 4t + 3: tile t, thread r = row r) ----------------
+    const int t = warp >> 2;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + t * 256 + lane_base, tO = tS + 128;
+    const int qrow = row0 + t * Tl::BM + r;
     const int lim = min(ctx + qrow, L - 1);  // last key this row sees
     float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < ntk; ++j) {
-      ok = wait_or_abort(s_full, j & 1, abort_flag);
-      if (!__all_sync(kFullMask, ok)) {
-        ok = false;
-        break;
-      }
+    bool ok = nk[t] > 0;
+    for (int j = 0; ok && j < nk[t]; ++j) {
+      ok = wait_warp(&s_full[t], j & 1, abort_flag);
+      if (!ok) break;
       tc::fence_after_sync();
-      float x[Tl::BN];
+      const int kb = j * Tl::BN;
+      // keys past this row's last one count as -inf (scale > 0, so the order of
+      // raw scores is the order of scaled ones)
+      const bool diag = kb + Tl::BN - 1 > lim;
+      // pass 1: the tile's max
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
       for (int c4 = 0; c4 < Tl::BN / 32; ++c4) {
         uint32_t u[32];
-        tc::tmem_ld32(tS + lane_base + c4 * 32, u);
+        tc::tmem_ld32(tS + c4 * 32, u);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) x[c4 * 32 + c] = __uint_as_float(u[c]);
+        for (int c = 0; c < 32; ++c) {
+          const float v = diag && kb + c4 * 32 + c > lim ? -INFINITY : __uint_as_float(u[c]);
+          mx[c & 7] = fmaxf(mx[c & 7], v);
+        }
       }
-      tc::fence_before_sync();
-      mbar_arrive(s_free);
-      const int kb = j * Tl::BN;
-      // keys past this row's last one read as -inf (scale > 0, so the order of
-      // raw scores is the order of scaled ones)
-      if (kb + Tl::BN - 1 > lim) {
-#pragma unroll
-        for (int c = 0; c < Tl::BN; ++c) x[c] = kb + c <= lim ? x[c] : -INFINITY;
-      }
-      float mx[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = x[k];
-#pragma unroll
-      for (int c = 8; c < Tl::BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
       const float tmax =
           fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
@@ -379,96 +418,70 @@ __global__ void __launch_bounds__(192, 1)
       const bool grow = m_new > m + 8.f;
       const float m_use = grow ? m_new : m;
       const float alpha = grow ? fast_exp2(m - m_use) : 1.f;
-      float sm8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
-#pragma unroll
-      for (int c = 0; c < Tl::BN; ++c) {
-        x[c] = fast_exp2(fmaf(x[c], p.scale_log2, -m_use));
-        sm8[c & 7] += x[c];
-      }
-      l = l * alpha + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
-                       ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
       m = m_use;
-      if (j > 0) {
-        ok = wait_or_abort(o_done, (j - 1) & 1, abort_flag);
-        if (!__all_sync(kFullMask, ok)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-      }
-      // P -> shared memory, K-major with the 128-byte swizzle; for bf16 also
-      // the rounding residue p - bf16(p), itself rounded to bf16
-#pragma unroll
-      for (int cb = 0; cb < Tl::BN / 64; ++cb) {
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const float* v = &x[cb * 64 + cc * 8];
-          const int off = cb * Tl::CB_BYTES + r * 128 + ((cc ^ (r & 7)) << 4);
-          uint32_t hi[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) hi[e] = pack_pair<T>(v[2 * e], v[2 * e + 1]);
-          *reinterpret_cast<uint4*>(sP + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          if constexpr (LO) {
-            uint32_t lo[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              // bf16 pair -> the two fp32 values it holds: exact bit moves
-              const float h0 = __uint_as_float(hi[e] << 16);
-              const float h1 = __uint_as_float(hi[e] & 0xffff0000u);
-              lo[e] = pack_pair<T>(v[2 * e] - h0, v[2 * e + 1] - h1);
-            }
-            *reinterpret_cast<uint4*>(sPlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-          }
-        }
-      }
-      // rescale the accumulator rows whose reference max moved
+      // The product of the previous key tile has completed (the commit that
+      // released these scores covers it): rescale the rows whose max moved.
       if (j > 0 && __any_sync(kFullMask, grow)) {
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t u[32];
-          tc::tmem_ld32(tO + lane_base + c4 * 32, u);
+          tc::tmem_ld32(tO + c4 * 32, u);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
-          tc::tmem_st32(tO + lane_base + c4 * 32, u);
-        }
-        tc::tmem_wait_st();
-      }
-      // keys past the end of the request: zero their V rows (P is 0 there, and
-      // 0 * NaN would not be)
-      if (j == ntk - 1 && kb + r >= L) {
-        const int st = j % Tl::NSTG;
-        ok = wait_or_abort(&v_full[st], (j / Tl::NSTG) & 1, abort_flag);
-        if (ok) {
-          uint8_t* row = sV + st * Tl::KV_BYTES + r * 128;
-#pragma unroll
-          for (int c = 0; c < Tl::COLB; ++c)
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              reinterpret_cast<uint4*>(row + c * Tl::CB_BYTES)[k] = make_uint4(0, 0, 0, 0);
+          tc::tmem_st32(tO + c4 * 32, u);
         }
       }
-      if (!__all_sync(kFullMask, ok)) {
-        ok = false;
-        break;
+      // pass 2: P over the scores, 32 keys at a time into their own 32 columns:
+      // keys 2k, 2k+1 as one 16-bit pair in column 32q + k, and for bf16 the
+      // rounding residue p - bf16(p), itself rounded, in column 32q + 16 + k
+      float sm8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
+#pragma unroll 1
+      for (int q = 0; q < Tl::BN / 32; ++q) {
+        uint32_t u[32];
+        tc::tmem_ld32(tS + q * 32, u);
+        tc::tmem_wait_ld();
+        float x[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float v = diag && kb + q * 32 + c > lim ? -INFINITY : __uint_as_float(u[c]);
+          x[c] = fast_exp2(fmaf(v, p.scale_log2, -m_use));
+          sm8[c & 7] += x[c];
+        }
+        uint32_t hi[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) hi[e] = pack_pair<T>(x[2 * e], x[2 * e + 1]);
+        tc::tmem_st16(tS + 32 * q, hi);
+        if constexpr (LO) {
+          uint32_t lo[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            // bf16 pair -> the two fp32 values it holds: exact bit moves
+            const float h0 = __uint_as_float(hi[e] << 16);
+            const float h1 = __uint_as_float(hi[e] & 0xffff0000u);
+            lo[e] = pack_pair<T>(x[2 * e] - h0, x[2 * e + 1] - h1);
+          }
+          tc::tmem_st16(tS + 32 * q + 16, lo);
+        }
       }
-      tc::fence_proxy_async_smem();
+      l = l * alpha + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
+                       ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
+      tc::tmem_wait_st();
       tc::fence_before_sync();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[t]);
     }
     // epilogue: O / l -> out
-    if (ok) ok = wait_or_abort(o_done, (ntk - 1) & 1, abort_flag);
-    if (__all_sync(kFullMask, ok)) {
+    if (ok) ok = wait_warp(&o_done[t], 0, abort_flag);
+    if (ok) {
       tc::fence_after_sync();
       const float inv = 1.f / l;
-      TO* dst = reinterpret_cast<TO*>(p.out) +
-                (static_cast<int64_t>(q0 + qrow) * p.H + h) * D;
+      TO* dst = reinterpret_cast<TO*>(p.out) + (static_cast<int64_t>(q0 + qrow) * p.H + h) * D;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t u[32];
-        tc::tmem_ld32(tO + lane_base + c4 * 32, u);
+        tc::tmem_ld32(tO + c4 * 32, u);
         tc::tmem_wait_ld();
         float v[32];
 #pragma unroll
@@ -479,7 +492,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, Tl::TMEM_COLS);
