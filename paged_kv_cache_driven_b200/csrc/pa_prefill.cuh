@@ -20,6 +20,8 @@
 //              moves;
 //   warp 8     producer: TMA loads of the two Q tiles and of 128-key K / V
 //              tiles, one box per (cache block, 64-column block), two stages;
+//              lane b reads the table entry of block b of a tile and issues its
+//              boxes, so a tile's boxes go out in parallel;
 //   warp 9     MMA issuer (lane 0) and tensor-memory owner, also zeroing V rows
 //              past the end of the request in the last key tile:
 //              S_t = Q_t K^T (both operands K-major in shared memory) and
@@ -238,63 +240,60 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 8) {
-    // ---------------- producer ----------------
-    if (lane == 0) {
-      int last_j[Tl::NSTG];
+    // ---------------- producer: lane b loads cache block b of each key tile ----------------
+    int last_j[Tl::NSTG];
 #pragma unroll
-      for (int s = 0; s < Tl::NSTG; ++s) last_j[s] = -1;
+    for (int s = 0; s < Tl::NSTG; ++s) last_j[s] = -1;
+    if (lane == 0) {
       mbar_arrive_expect_tx(q_full, nq * Tl::Q_BYTES);
       for (int t = 0; t < nq; ++t)
 #pragma unroll
         for (int c = 0; c < Tl::COLB; ++c)
           tc::tma_load_3d(sQ + t * Tl::Q_BYTES + c * Tl::CB_BYTES, &tmq, c * 64, h,
                           q0 + row0 + t * Tl::BM, q_full);
-      const int nblk = (L + S - 1) / S;
-      const int32_t* table = p.block_tables + static_cast<int64_t>(i) * p.MB;
-      for (int j = 0; j < NK; ++j) {
-        const int st = j % Tl::NSTG;
-        if (j >= Tl::NSTG && !wait_or_abort(&kv_empty[st], ((j / Tl::NSTG) - 1) & 1, abort_flag))
-          break;
-        int ids[BPT];
-        int nvalid = 0;
-#pragma unroll
-        for (int b = 0; b < BPT; ++b) {
-          const int lb = j * BPT + b;
-          int id = -1;
-          if (lb < nblk) {
-            id = table[lb];
-            if (id < 0 || id >= p.NB) {
-              raise_error(PA_DEVERR_BLOCK_ID);
-              id = -1;
-            }
-          }
-          ids[b] = id;
-          nvalid += id >= 0;
+    }
+    const int nblk = (L + S - 1) / S;
+    const int32_t* table = p.block_tables + static_cast<int64_t>(i) * p.MB;
+    // this lane's block id in key tile j (-1: none or invalid)
+    auto block_id = [&](int j) {
+      const int lb = j * BPT + lane;
+      int id = -1;
+      if (lane < BPT && lb < nblk) {
+        id = table[lb];
+        if (id < 0 || id >= p.NB) {
+          raise_error(PA_DEVERR_BLOCK_ID);
+          id = -1;
         }
-        const uint32_t bytes = static_cast<uint32_t>(nvalid) * S * 128 * Tl::COLB;
-        uint8_t* dk = sK + st * Tl::KV_BYTES;
-        uint8_t* dv = sV + st * Tl::KV_BYTES;
-        mbar_arrive_expect_tx(&k_full[st], bytes);
-#pragma unroll
-        for (int b = 0; b < BPT; ++b) {
-          if (ids[b] < 0) continue;
-          const int y = (ids[b] * p.Hkv + hk) * S;
-#pragma unroll
-          for (int c = 0; c < Tl::COLB; ++c)
-            tma_load_2d_nohint(dk + c * Tl::CB_BYTES + b * S * 128, &tmk, c * 64, y, &k_full[st]);
-        }
-        mbar_arrive_expect_tx(&v_full[st], bytes);
-#pragma unroll
-        for (int b = 0; b < BPT; ++b) {
-          if (ids[b] < 0) continue;
-          const int y = (ids[b] * p.Hkv + hk) * S;
-#pragma unroll
-          for (int c = 0; c < Tl::COLB; ++c)
-            tma_load_2d_nohint(dv + c * Tl::CB_BYTES + b * S * 128, &tmv, c * 64, y, &v_full[st]);
-        }
-        last_j[st] = j;
       }
-      // copies in flight land before the CTA can exit
+      return id;
+    };
+    int id = block_id(0);
+    for (int j = 0; j < NK; ++j) {
+      const int st = j % Tl::NSTG;
+      if (j >= Tl::NSTG && !wait_warp(&kv_empty[st], ((j / Tl::NSTG) - 1) & 1, abort_flag)) break;
+      const int nvalid = __popc(__ballot_sync(kFullMask, id >= 0));
+      const uint32_t bytes = static_cast<uint32_t>(nvalid) * S * 128 * Tl::COLB;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&k_full[st], bytes);
+        mbar_arrive_expect_tx(&v_full[st], bytes);
+      }
+      __syncwarp();
+      if (id >= 0) {
+        const int y = (id * p.Hkv + hk) * S;
+        uint8_t* dk = sK + st * Tl::KV_BYTES + lane * S * 128;
+        uint8_t* dv = sV + st * Tl::KV_BYTES + lane * S * 128;
+#pragma unroll
+        for (int c = 0; c < Tl::COLB; ++c)
+          tma_load_2d_nohint(dk + c * Tl::CB_BYTES, &tmk, c * 64, y, &k_full[st]);
+#pragma unroll
+        for (int c = 0; c < Tl::COLB; ++c)
+          tma_load_2d_nohint(dv + c * Tl::CB_BYTES, &tmv, c * 64, y, &v_full[st]);
+      }
+      last_j[st] = j;
+      if (j + 1 < NK) id = block_id(j + 1);  // the next tile's ids load while this one lands
+    }
+    // copies in flight land before the CTA can exit
+    if (lane == 0) {
       mbar_wait_bounded(q_full, 0);
 #pragma unroll
       for (int s = 0; s < Tl::NSTG; ++s)
@@ -304,6 +303,7 @@ __global__ void __launch_bounds__(320, 1)
           mbar_wait_bounded(&v_full[s], par);
         }
     }
+    __syncwarp();
   } else if (warp == 9) {
     // ---------------- MMA issuer (lane 0), V tail zeroing (whole warp) ----------------
     constexpr int fmt = LO ? 1 : 0;
