@@ -19,7 +19,8 @@
 //              rescales the tile's output accumulator when its reference max
 //              moves;
 //   warp 8     producer: TMA loads of the two Q tiles and of 128-key K / V
-//              tiles, one box per (cache block, 64-column block), two stages;
+//              tiles, one box per (cache block, 64-column block); K runs up to
+//              three tiles ahead, V two (four each for head size 64);
 //              lane b reads the table entry of block b of a tile and issues its
 //              boxes, so a tile's boxes go out in parallel;
 //   warp 9     MMA issuer (lane 0) and tensor-memory owner, also zeroing V rows
@@ -58,14 +59,17 @@ struct PrefillTiling {
   static constexpr int BM = 128;              // query rows per tile (MMA M)
   static constexpr int NQT = 2;               // query tiles per CTA
   static constexpr int BN = 128;              // keys per tile
-  static constexpr int NSTG = 2;              // K / V stages
+  // K runs further ahead than V: S needs K(j + 1) right after P(j) is ready,
+  // V(j + 1) only after the next softmax
+  static constexpr int KST = D == 128 ? 3 : 4;  // K stages
+  static constexpr int VST = D == 128 ? 2 : 4;  // V stages
   static constexpr int COLB = D / 64;         // 64-element (128-byte) column blocks
   static constexpr int CB_BYTES = 128 * 128;  // one column block of 128 rows
   static constexpr int Q_BYTES = BM * D * 2;  // one query tile
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int OFF_K = NQT * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NSTG * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NSTG * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
   // + alignment slack and barriers; at least 120 KB, so that one CTA holds an
   // SM (it allocates all 512 tensor-memory columns)
   static constexpr int SMEM = 1024 + OFF_BAR + 256 > 120 * 1024 ? 1024 + OFF_BAR + 256 : 120 * 1024;
@@ -202,10 +206,11 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sV = sm + Tl::OFF_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Tl::OFF_BAR);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;                // [NSTG]
-  uint64_t* v_full = k_full + Tl::NSTG;       // [NSTG]
-  uint64_t* kv_empty = v_full + Tl::NSTG;     // [NSTG]
-  uint64_t* s_full = kv_empty + Tl::NSTG;     // [NQT]
+  uint64_t* k_full = bars + 1;                // [KST]
+  uint64_t* k_empty = k_full + Tl::KST;       // [KST]
+  uint64_t* v_full = k_empty + Tl::KST;       // [VST]
+  uint64_t* v_empty = v_full + Tl::VST;       // [VST]
+  uint64_t* s_full = v_empty + Tl::VST;       // [NQT]
   uint64_t* p_full = s_full + Tl::NQT;        // [NQT]
   uint64_t* o_done = p_full + Tl::NQT;        // [NQT]
   uint64_t* mma_done = o_done + Tl::NQT;
@@ -215,10 +220,13 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < Tl::NSTG; ++s) {
+    for (int s = 0; s < Tl::KST; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < Tl::VST; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int t = 0; t < Tl::NQT; ++t) {
       mbar_init(&s_full[t], 1);
@@ -241,9 +249,6 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ---------------- producer: lane b loads cache block b of each key tile ----------------
-    int last_j[Tl::NSTG];
-#pragma unroll
-    for (int s = 0; s < Tl::NSTG; ++s) last_j[s] = -1;
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, nq * Tl::Q_BYTES);
       for (int t = 0; t < nq; ++t)
@@ -267,42 +272,51 @@ __global__ void __launch_bounds__(320, 1)
       }
       return id;
     };
-    int id = block_id(0);
-    for (int j = 0; j < NK; ++j) {
-      const int st = j % Tl::NSTG;
-      if (j >= Tl::NSTG && !wait_warp(&kv_empty[st], ((j / Tl::NSTG) - 1) & 1, abort_flag)) break;
+    // one K or V tile: every lane issues the boxes of its block
+    auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full, int id) {
       const int nvalid = __popc(__ballot_sync(kFullMask, id >= 0));
-      const uint32_t bytes = static_cast<uint32_t>(nvalid) * S * 128 * Tl::COLB;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&k_full[st], bytes);
-        mbar_arrive_expect_tx(&v_full[st], bytes);
-      }
+      if (lane == 0)
+        mbar_arrive_expect_tx(full, static_cast<uint32_t>(nvalid) * S * 128 * Tl::COLB);
       __syncwarp();
       if (id >= 0) {
         const int y = (id * p.Hkv + hk) * S;
-        uint8_t* dk = sK + st * Tl::KV_BYTES + lane * S * 128;
-        uint8_t* dv = sV + st * Tl::KV_BYTES + lane * S * 128;
 #pragma unroll
         for (int c = 0; c < Tl::COLB; ++c)
-          tma_load_2d_nohint(dk + c * Tl::CB_BYTES, &tmk, c * 64, y, &k_full[st]);
-#pragma unroll
-        for (int c = 0; c < Tl::COLB; ++c)
-          tma_load_2d_nohint(dv + c * Tl::CB_BYTES, &tmv, c * 64, y, &v_full[st]);
+          tma_load_2d_nohint(dst + c * Tl::CB_BYTES + lane * S * 128, map, c * 64, y, full);
       }
-      last_j[st] = j;
-      if (j + 1 < NK) id = block_id(j + 1);  // the next tile's ids load while this one lands
+    };
+    // K(j + 1) goes out before V(j); block ids are read one tile ahead
+    int id_v = block_id(0), id_k = id_v;
+    int k_issued = 0, v_issued = 0;
+    bool ok = true;
+    load_tile(&tmk, sK, &k_full[0], id_k);
+    k_issued = 1;
+    if (NK > 1) id_k = block_id(1);
+    for (int j = 0; j < NK; ++j) {
+      if (j + 1 < NK) {
+        const int kj = j + 1, st = kj % Tl::KST;
+        if (kj >= Tl::KST && !(ok = wait_warp(&k_empty[st], ((kj / Tl::KST) - 1) & 1, abort_flag)))
+          break;
+        load_tile(&tmk, sK + st * Tl::KV_BYTES, &k_full[st], id_k);
+        k_issued = kj + 1;
+      }
+      const int st = j % Tl::VST;
+      if (j >= Tl::VST && !(ok = wait_warp(&v_empty[st], ((j / Tl::VST) - 1) & 1, abort_flag)))
+        break;
+      load_tile(&tmv, sV + st * Tl::KV_BYTES, &v_full[st], id_v);
+      v_issued = j + 1;
+      id_v = id_k;
+      if (j + 2 < NK) id_k = block_id(j + 2);
     }
     // copies in flight land before the CTA can exit
     if (lane == 0) {
       mbar_wait_bounded(q_full, 0);
-#pragma unroll
-      for (int s = 0; s < Tl::NSTG; ++s)
-        if (last_j[s] >= 0) {
-          const uint32_t par = (last_j[s] / Tl::NSTG) & 1;
-          mbar_wait_bounded(&k_full[s], par);
-          mbar_wait_bounded(&v_full[s], par);
-        }
+      for (int kj = max(k_issued - Tl::KST, 0); kj < k_issued; ++kj)
+        mbar_wait_bounded(&k_full[kj % Tl::KST], (kj / Tl::KST) & 1);
+      for (int vj = max(v_issued - Tl::VST, 0); vj < v_issued; ++vj)
+        mbar_wait_bounded(&v_full[vj % Tl::VST], (vj / Tl::VST) & 1);
     }
+    (void)ok;
     __syncwarp();
   } else if (warp == 9) {
     // ---------------- MMA issuer (lane 0), V tail zeroing (whole warp) ----------------
@@ -312,7 +326,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
     auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
       const uint32_t qb = aQ + t * Tl::Q_BYTES;
-      const uint32_t kb = aK + (j % Tl::NSTG) * Tl::KV_BYTES;
+      const uint32_t kb = aK + (j % Tl::KST) * Tl::KV_BYTES;
 #pragma unroll
       for (int s = 0; s < D / 16; ++s) {
         const uint32_t off = (s >> 2) * Tl::CB_BYTES + (s & 3) * 32;
@@ -324,12 +338,14 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = wait_warp(q_full, 0, abort_flag) && wait_warp(&k_full[0], 0, abort_flag);
     if (ok) {
       tc::fence_after_sync();
-      if (lane == 0)
+      if (lane == 0) {
         for (int t = 0; t < nq; ++t) issue_s(t, 0);
+        tc::commit(&k_empty[0]);
+      }
     }
     for (int j = 0; ok && j < NK; ++j) {
-      const int st = j % Tl::NSTG;
-      ok = wait_warp(&v_full[st], (j / Tl::NSTG) & 1, abort_flag);
+      const int st = j % Tl::VST;
+      ok = wait_warp(&v_full[st], (j / Tl::VST) & 1, abort_flag);
       if (!ok) break;
       const int kb = j * Tl::BN;
       if (j == NK - 1 && kb + Tl::BN > L) {
@@ -362,13 +378,17 @@ __global__ void __launch_bounds__(320, 1)
           if (j == nk[t] - 1) tc::commit(&o_done[t]);
         }
         if (j + 1 < nk[t]) {
-          ok = wait_warp(&k_full[(j + 1) % Tl::NSTG], ((j + 1) / Tl::NSTG) & 1, abort_flag);
+          ok = wait_warp(&k_full[(j + 1) % Tl::KST], ((j + 1) / Tl::KST) & 1, abort_flag);
           if (!ok) break;
           tc::fence_after_sync();
           if (lane == 0) issue_s(t, j + 1);
         }
       }
-      if (ok && lane == 0) tc::commit(&kv_empty[st]);
+      // V(j) and, if any tile read it, K(j + 1) are free once these products finish
+      if (ok && lane == 0) {
+        tc::commit(&v_empty[st]);
+        if (j + 1 < NK) tc::commit(&k_empty[(j + 1) % Tl::KST]);
+      }
     }
     // every MMA issued has completed before tensor memory is released
     if (lane == 0) {
