@@ -492,6 +492,188 @@ def run_shape_workloads(args):
     print(json.dumps(summary), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# Prompt prefill: causal paged prefill attention (pa_prefill) on the tensor cores
+# ---------------------------------------------------------------------------
+
+PREFILL_METRIC = "paged prefill attention TFLOP/s"
+PREFILL_WORKLOAD = "prompt prefill: 16 prompts of U[512,4096] tokens, 32 heads, head_dim 128, " \
+                   "block 16, bf16, permuted pool, causal"
+
+
+def prefill_flops(new_lens, ctx_lens, Hq, Dh):
+    """Algorithmic FLOPs of causal prefill: q.k and p.v (2 * D each) for every
+    (new token, head, key it sees) triple; new token j of a request with c
+    cached tokens sees c + j + 1 keys."""
+    return sum(Hq * 4 * Dh * (n * c + n * (n + 1) // 2) for n, c in zip(new_lens, ctx_lens))
+
+
+def measured_tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
+    return 1590.0, "fallback"
+
+
+def prefill_cpu_baseline(target_seconds, cores, seed):
+    """The oracle's causal prefill on one prompt of the workload's shape (32 heads,
+    head_dim 128, block 16) on the host cores, its length sized to about
+    target_seconds: (TFLOP/s, description)."""
+    from oracle import decode as oracle_decode  # test infrastructure: CPU-baseline leg only
+
+    n, total, passes = 128, 0.0, 0
+    while True:
+        pc = workloads.prefill_case([0], [n], H=32, D=128, S=16, dtype=DTYPE, seed=seed,
+                                    device="cpu")
+        c = pc.cache
+        t0 = time.perf_counter()
+        oracle_decode.paged_prefill(pc.q, c.k_cache, c.v_cache, c.block_tables, c.seq_lens,
+                                    pc.q_start, c.scale, threads=cores)
+        dt = time.perf_counter() - t0
+        if dt >= target_seconds * 0.3 or n >= 4096:
+            total, passes = dt, 1
+            break
+        n = min(4096, int(n * max(1.5, min(4.0, (target_seconds * 0.5 / max(dt, 1e-3)) ** 0.5))))
+    fl = prefill_flops([n], [0], 32, 128)
+    return fl / total / 1e12, (f"one {n}-token prompt x 32 heads (causal, fp64) x {passes} pass, "
+                               f"{total:.1f} s on {cores} threads")
+
+
+def run_prefill_workload(args):
+    """--workload prompt_prefill: pa_prefill over the prompt prefill workload,
+    TFLOP/s against the measured bf16 tensor peak, plus an end-to-end prefill
+    step through the C ABI from host buffers (host allocator, uploads of the
+    prompts' q/k/v, pa_kv_append, pa_prefill, download of the output)."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    if args.workload == "prompt_prefill_small":  # a profiling-sized case of the same kernel
+        pc = workloads.prompt_prefill(seed=args.seed, device=device, n_req=4, lo=2048, hi=2048,
+                                      H=8)
+    else:
+        pc = workloads.prompt_prefill(seed=args.seed, device=device)
+    c = pc.cache
+    T, Hq, Dh = pc.q.shape
+    flops = prefill_flops(pc.new_lens, pc.ctx_lens, Hq, Dh)
+    out = torch.empty((T, Hq, Dh), dtype=DTYPE, device=device)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        binding.pa_prefill(out, pc.q, c.k_cache, c.v_cache, c.block_tables, c.seq_lens,
+                           pc.q_start, c.scale, pc.max_q_len)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        clk.mark_start()
+        start.record(stream)
+        for a, b in evs:
+            a.record(stream)
+            call()
+            b.record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        clk.mark_end()
+    total_ms = start.elapsed_time(end)
+    call_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    if binding.pa_get_device_error():
+        raise SystemExit("device error word set")
+    value = flops * args.steps / (total_ms / 1e3) / 1e12
+    achieved = flops / (call_ms / 1e3) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+
+    # ---- end to end: the same prompts from host buffers ------------------------
+    kh = torch.randn((T, c.k_cache.shape[1], Dh), dtype=torch.float32).to(DTYPE).pin_memory()
+    vh = torch.randn((T, c.k_cache.shape[1], Dh), dtype=torch.float32).to(DTYPE).pin_memory()
+    qh = pc.q.cpu().pin_memory()
+    oh = torch.empty((T, Hq, Dh), dtype=DTYPE).pin_memory()
+    B = len(pc.new_lens)
+    NB = c.k_cache.shape[0]
+    MB = c.block_tables.shape[1]
+    qs_h = pc.q_start.cpu().pin_memory()
+    dq = torch.empty_like(pc.q)
+    dk = torch.empty((T, c.k_cache.shape[1], Dh), dtype=DTYPE, device=device)
+    dv = torch.empty_like(dk)
+    dslots = torch.empty(T, dtype=torch.int64, device=device)
+    dtab = torch.empty((B, MB), dtype=torch.int32, device=device)
+    dlens = torch.empty(B, dtype=torch.int32, device=device)
+    dqs = torch.empty(B + 1, dtype=torch.int32, device=device)
+    h2d = d2h = 0
+
+    def e2e_step():
+        nonlocal h2d, d2h
+        alloc = binding.BlockAllocator(NB, c.k_cache.shape[2])
+        ids = list(range(B))
+        for i, n in zip(ids, pc.new_lens):
+            alloc.pa_seq_grow(i, n)
+        slots = alloc.pa_build_slot_mapping(ids, [0] * B, pc.new_lens).pin_memory()
+        tables = alloc.pa_build_block_tables(ids, MB).pin_memory()
+        lens = torch.tensor(pc.new_lens, dtype=torch.int32).pin_memory()
+        for dst, src in ((dq, qh), (dk, kh), (dv, vh), (dslots, slots), (dtab, tables),
+                         (dlens, lens), (dqs, qs_h)):
+            dst.copy_(src, non_blocking=True)
+        binding.pa_kv_append(dk, dv, dslots, c.k_cache, c.v_cache)
+        binding.pa_prefill(out, dq, c.k_cache, c.v_cache, dtab, dlens, dqs, c.scale,
+                           pc.max_q_len)
+        oh.copy_(out, non_blocking=True)
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, slots, tables, lens, qs_h))
+        d2h = oh.numel() * oh.element_size()
+        alloc.close()
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if binding.pa_get_device_error():
+        raise SystemExit("device error word set")
+    e2e_value = flops * args.steps / (e2e_ms / 1e3) / 1e12
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        v, desc = prefill_cpu_baseline(12.0, cores, args.seed)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+    line = {
+        "metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": PREFILL_WORKLOAD if args.workload == "prompt_prefill" else
+                   "prompt prefill, profiling size: 4 prompts of 2048 tokens, 8 heads",
+                   "prompt_tokens": T, "heads": Hq,
+                   "head_dim": Dh, "block_size": c.k_cache.shape[2], "flops_per_step": flops,
+                   "l2": "inputs larger than L2 (0.9 GB of q and K/V vs 126 MB L2)",
+                   "parallelism": "dp1"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "traffic": None, "kernel": "paged_prefill_kernel (one launch per step)",
+                     "call_ms": round(call_ms, 4), "algorithmic_flops_per_launch": flops,
+                     "tensor_work_per_launch": "bf16 weights enter P.V as two terms, so the "
+                                               "tensor cores do 1.5x the algorithmic FLOPs"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
+                "api": "host BlockAllocator (grow, slot mapping, tables), pinned uploads, "
+                       "pa_kv_append, pa_prefill, output download",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms / args.steps, 4)},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -501,15 +683,21 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="llama13b",
-                    choices=["llama13b", "long_context", "sweep", "llama70b"],
+                    choices=["llama13b", "long_context", "sweep", "llama70b", "prompt_prefill",
+                             "prompt_prefill_small"],
                     help="llama13b: the headline step (default); the others time decode-only "
                          "calls of the long-context, shape-sweep and LLaMA-2-70B-shaped "
-                         "grouped-query configurations")
+                         "grouped-query configurations, or paged prefill attention over "
+                         "16 prompts (prompt_prefill)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.workload.startswith("prompt_prefill"):
+        binding.lib()
+        run_prefill_workload(args)
         return
     if args.workload != "llama13b":
         binding.lib()
