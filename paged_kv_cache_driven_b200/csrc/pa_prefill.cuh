@@ -13,7 +13,7 @@
 // threads in four roles:
 //   warps 0-3, 4-7  softmax for query tile 0 / 1: thread r owns row r of its
 //              tile (tensor-memory lane r); reads the tile's scores from tensor
-//              memory (twice: max, then weights), keeps the running max / sum
+//              memory (one read of the whole row), keeps the running max / sum
 //              in fp32, writes the weights P back over the scores as 16-bit
 //              pairs (bf16 as hi + lo halves, so the weights keep ~16 bits), and
 //              rescales the tile's output accumulator when its reference max
@@ -115,6 +115,32 @@ template <>
 __device__ __forceinline__ uint32_t pack_pair<__half>(float a, float b) {
   const __half2 v = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Packed pairs of fp32 (one 64-bit register pair, two lanes of work per
+// instruction) and the three-input max.
+__device__ __forceinline__ uint64_t as_u64(float2 a) {
+  return static_cast<uint64_t>(__float_as_uint(a.x)) |
+         (static_cast<uint64_t>(__float_as_uint(a.y)) << 32);
+}
+__device__ __forceinline__ float2 as_f2(uint64_t u) {
+  return make_float2(__uint_as_float(static_cast<uint32_t>(u)),
+                     __uint_as_float(static_cast<uint32_t>(u >> 32)));
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(as_u64(a)), "l"(as_u64(b)), "l"(as_u64(c)));
+  return as_f2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(as_u64(a)), "l"(as_u64(b)));
+  return as_f2(d);
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // 2^x with the hardware approximation (relative error about 2^-22; 2^-inf = 0).
@@ -414,24 +440,24 @@ __global__ void __launch_bounds__(320, 1)
       // keys past this row's last one count as -inf (scale > 0, so the order of
       // raw scores is the order of scaled ones)
       const bool diag = kb + Tl::BN - 1 > lim;
-      // pass 1: the tile's max
-      float mx[8];
+      // the row's 128 scores: four loads in flight, one wait
+      float x[Tl::BN];
+      {
+        uint32_t u[Tl::BN];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
-#pragma unroll
-      for (int c4 = 0; c4 < Tl::BN / 32; ++c4) {
-        uint32_t u[32];
-        tc::tmem_ld32(tS + c4 * 32, u);
+        for (int c4 = 0; c4 < Tl::BN / 32; ++c4)
+          tc::tmem_ld32(tS + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c4 * 32]));
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float v = diag && kb + c4 * 32 + c > lim ? -INFINITY : __uint_as_float(u[c]);
-          mx[c & 7] = fmaxf(mx[c & 7], v);
-        }
+        for (int c = 0; c < Tl::BN; ++c)
+          x[c] = diag && kb + c > lim ? -INFINITY : __uint_as_float(u[c]);
       }
-      const float tmax =
-          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
+      float mx[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
+#pragma unroll
+      for (int c = 8; c < Tl::BN; c += 2) mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], x[c], x[c + 1]);
+      const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * p.scale_log2;
       // The reference max only moves when the tile max exceeds it by more than
       // 2^8 in weight; the weights stay <= 256, exact in the final ratio.
       const float m_new = fmaxf(m, tmax);
@@ -439,10 +465,38 @@ __global__ void __launch_bounds__(320, 1)
       const float m_use = grow ? m_new : m;
       const float alpha = grow ? fast_exp2(m - m_use) : 1.f;
       m = m_use;
+      // P over the scores, 8 keys at a time: keys 2k, 2k+1 of chunk q (32 keys)
+      // as one 16-bit pair in column 32q + k, and for bf16 the rounding residue
+      // p - bf16(p), itself rounded, in column 32q + 16 + k
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int g = 0; g < Tl::BN / 8; ++g) {  // 8 keys: 4 columns of P (and 4 of residues)
+        float* v = &x[8 * g];
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 t = ffma2(make_float2(v[2 * e], v[2 * e + 1]), sc2, nm2);
+          const float2 pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          acc[e & 1] = fadd2(acc[e & 1], pe);
+          hi[e] = pack_pair<T>(pe.x, pe.y);
+          if constexpr (LO) {
+            // bf16 pair -> the two fp32 values it holds: exact bit moves
+            const float2 h = make_float2(__uint_as_float(hi[e] << 16),
+                                         __uint_as_float(hi[e] & 0xffff0000u));
+            const float2 r = make_float2(pe.x - h.x, pe.y - h.y);
+            lo[e] = pack_pair<T>(r.x, r.y);
+          }
+        }
+        const uint32_t col = 32 * (g >> 2) + 4 * (g & 3);
+        tc::tmem_st4(tS + col, hi);
+        if constexpr (LO) tc::tmem_st4(tS + col + 16, lo);
+      }
       // The product of the previous key tile has completed (the commit that
       // released these scores covers it): rescale the rows whose max moved.
       if (j > 0 && __any_sync(kFullMask, grow)) {
-#pragma unroll
+#pragma unroll 1
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t u[32];
           tc::tmem_ld32(tO + c4 * 32, u);
@@ -452,42 +506,7 @@ __global__ void __launch_bounds__(320, 1)
           tc::tmem_st32(tO + c4 * 32, u);
         }
       }
-      // pass 2: P over the scores, 32 keys at a time into their own 32 columns:
-      // keys 2k, 2k+1 as one 16-bit pair in column 32q + k, and for bf16 the
-      // rounding residue p - bf16(p), itself rounded, in column 32q + 16 + k
-      float sm8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) sm8[k] = 0.f;
-#pragma unroll 1
-      for (int q = 0; q < Tl::BN / 32; ++q) {
-        uint32_t u[32];
-        tc::tmem_ld32(tS + q * 32, u);
-        tc::tmem_wait_ld();
-        float x[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float v = diag && kb + q * 32 + c > lim ? -INFINITY : __uint_as_float(u[c]);
-          x[c] = fast_exp2(fmaf(v, p.scale_log2, -m_use));
-          sm8[c & 7] += x[c];
-        }
-        uint32_t hi[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) hi[e] = pack_pair<T>(x[2 * e], x[2 * e + 1]);
-        tc::tmem_st16(tS + 32 * q, hi);
-        if constexpr (LO) {
-          uint32_t lo[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            // bf16 pair -> the two fp32 values it holds: exact bit moves
-            const float h0 = __uint_as_float(hi[e] << 16);
-            const float h1 = __uint_as_float(hi[e] & 0xffff0000u);
-            lo[e] = pack_pair<T>(x[2 * e] - h0, x[2 * e + 1] - h1);
-          }
-          tc::tmem_st16(tS + 32 * q + 16, lo);
-        }
-      }
-      l = l * alpha + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
-                       ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
+      l = l * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
       tc::tmem_wait_st();
       tc::fence_before_sync();
       mbar_arrive(&p_full[t]);
