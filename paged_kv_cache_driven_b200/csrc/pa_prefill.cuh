@@ -13,7 +13,7 @@
 // threads in four roles:
 //   warps 0-3, 4-7  softmax for query tile 0 / 1: thread r owns row r of its
 //              tile (tensor-memory lane r); reads the tile's scores from tensor
-//              memory (one read of the whole row), keeps the running max / sum
+//              memory (the whole row, read in two overlapped halves), keeps the running max / sum
 //              in fp32, writes the weights P back over the scores as 16-bit
 //              pairs (bf16 as hi + lo halves, so the weights keep ~16 bits), and
 //              rescales the tile's output accumulator when its reference max
@@ -440,23 +440,31 @@ __global__ void __launch_bounds__(320, 1)
       // keys past this row's last one count as -inf (scale > 0, so the order of
       // raw scores is the order of scaled ones)
       const bool diag = kb + Tl::BN - 1 > lim;
-      // the row's 128 scores: four loads in flight, one wait
+      // the row's 128 scores in two halves: the second half's loads are in
+      // flight while the first half's max is taken
       float x[Tl::BN];
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       {
         uint32_t u[Tl::BN];
+        constexpr int HALF = Tl::BN / 2;
 #pragma unroll
-        for (int c4 = 0; c4 < Tl::BN / 32; ++c4)
+        for (int c4 = 0; c4 < HALF / 32; ++c4)
           tc::tmem_ld32(tS + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c4 * 32]));
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < Tl::BN; ++c)
-          x[c] = diag && kb + c > lim ? -INFINITY : __uint_as_float(u[c]);
+        for (int c4 = HALF / 32; c4 < Tl::BN / 32; ++c4)
+          tc::tmem_ld32(tS + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c4 * 32]));
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          if (hf == 1) tc::tmem_wait_ld();
+#pragma unroll
+          for (int c = hf * HALF; c < (hf + 1) * HALF; ++c)
+            x[c] = diag && kb + c > lim ? -INFINITY : __uint_as_float(u[c]);
+#pragma unroll
+          for (int c = hf * HALF; c < (hf + 1) * HALF; c += 2)
+            mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], x[c], x[c + 1]);
+        }
       }
-      float mx[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
-#pragma unroll
-      for (int c = 8; c < Tl::BN; c += 2) mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], x[c], x[c + 1]);
       const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * p.scale_log2;
       // The reference max only moves when the tile max exceeds it by more than
       // 2^8 in weight; the weights stay <= 256, exact in the final ratio.
