@@ -555,7 +555,7 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   const uint8_t* vbase = static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(hk) * SLAB;
 
   if (w == NC) {
-    // ---- producer: lane 0 issues the unit's box loads ----
+    // ---- producer: one lane per box of a unit issues the loads ----
     const uint64_t policy = policy_evict_first();
     const int blk0 = t_beg / S;
     const int blk1 = t_end > t_beg ? (t_end + S - 1) / S : blk0;
@@ -564,7 +564,8 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
     int ids_b = (blk0 + 32 + lane < blk1) ? __ldg(trow + blk0 + 32 + lane) : -1;
     for (int u = 0; u < nunits; ++u) {
       const int s = u % NS;
-      if (u >= NS && !mbar_wait_bounded(&empty[s], ((u / NS) - 1) & 1)) {
+      // every lane waits; the warp leaves together if any lane gave up
+      if (u >= NS && !__all_sync(kFullMask, mbar_wait_bounded(&empty[s], ((u / NS) - 1) & 1))) {
         if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
         break;
       }
@@ -579,38 +580,39 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
       const int id0 = __shfl_sync(kFullMask, ids_a, rel);
       const int id1a = __shfl_sync(kFullMask, ids_a, (rel + 1) & 31);
       const int id1b = __shfl_sync(kFullMask, ids_b, (rel + 1) & 31);
-      if (lane == 0) {
-        // the unit's rows in one box group (S >= 16) or two (S = 8)
-        uint32_t okmask = 0, bytes = 0;
-        int rows_y[2] = {0, 0};
-        bool issue[2] = {false, false};
-        constexpr int NH = ROWS / BR;
+      // the unit's rows in one box group (S >= 16) or two (S = 8); every lane
+      // works out the plan, lane 0 arms the barrier, then one lane per box
+      // issues it, so a unit's boxes go out in parallel
+      uint32_t okmask = 0, bytes = 0;
+      int rows_y[2] = {0, 0};
+      bool issue[2] = {false, false};
+      constexpr int NH = ROWS / BR;
 #pragma unroll
-        for (int hh = 0; hh < NH; ++hh) {
-          const int th = t0 + hh * BR;
-          if (th >= t_end) continue;
-          const int id = hh == 0 ? id0 : (rel + 1 < 32 ? id1a : id1b);
-          if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.NB)) {
-            raise_error(PA_DEVERR_BLOCK_ID);
-            continue;
-          }
-          issue[hh] = true;
-          rows_y[hh] = (id * p.Hkv + hk) * S + th % S;
-          const int nrow = min(BR, t_end - th);
-          okmask |= ((1u << nrow) - 1u) << (hh * BR);
-          bytes += 2u * (D / 64) * BR * 128u;
+      for (int hh = 0; hh < NH; ++hh) {
+        const int th = t0 + hh * BR;
+        if (th >= t_end) continue;
+        const int id = hh == 0 ? id0 : (rel + 1 < 32 ? id1a : id1b);
+        if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.NB)) {
+          if (lane == 0) raise_error(PA_DEVERR_BLOCK_ID);
+          continue;
         }
+        issue[hh] = true;
+        rows_y[hh] = (id * p.Hkv + hk) * S + th % S;
+        const int nrow = min(BR, t_end - th);
+        okmask |= ((1u << nrow) - 1u) << (hh * BR);
+        bytes += 2u * (D / 64) * BR * 128u;
+      }
+      if (lane == 0) {
         rowmask[s] = okmask;
         mbar_arrive_expect_tx(&full[s], bytes);
-#pragma unroll
-        for (int hh = 0; hh < NH; ++hh) {
-          if (!issue[hh]) continue;
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            uint8_t* dst = stages + s * STAGE + c * Tg::BOX + hh * BR * 128;
-            tma_load_2d(dst, &tmk, c * 64, rows_y[hh], &full[s], policy);
-            tma_load_2d(dst + TILE, &tmv, c * 64, rows_y[hh], &full[s], policy);
-          }
+      }
+      __syncwarp();
+      constexpr int NBOX = NH * (D / 64) * 2;  // (row group, column block, K or V)
+      if (lane < NBOX) {
+        const int hh = lane / ((D / 64) * 2), c = (lane >> 1) % (D / 64), kv = lane & 1;
+        if (issue[hh]) {
+          uint8_t* dst = stages + s * STAGE + c * Tg::BOX + hh * BR * 128 + kv * TILE;
+          tma_load_2d(dst, kv ? &tmv : &tmk, c * 64, rows_y[hh], &full[s], policy);
         }
       }
       __syncwarp();
