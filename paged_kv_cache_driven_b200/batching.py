@@ -20,6 +20,15 @@ One step, in this order (the order is part of the contract the tests check):
 
 Random draws (lengths, budgets, token values, the shuffled free list) come from
 ``workloads.BatchingLoop``; everything else runs in the library.
+
+With ``graph=True`` the device part of step 2-3 (the three uploads from the
+pinned staging set and the append + decode launches) is a CUDA graph: the
+first step that uses a staging set runs it eagerly and captures it, later steps
+with that set replay it. The graph fixes every pointer and size, so the step's
+q/k/v are first copied into fixed device buffers and decode is planned for the
+largest length the loop can reach (``max_len``) instead of the step's own
+maximum; the eager path does the same when ``fixed_plan`` is set, so the two
+give the same bits.
 """
 
 import math
@@ -57,9 +66,12 @@ class StagingRing:
 
 
 class ContinuousBatching:
-    def __init__(self, loop, device, max_steps=64, poison=True, fused=False):
+    def __init__(self, loop, device, max_steps=64, poison=True, fused=False, graph=False,
+                 fixed_plan=False):
         self.loop = loop
         self.fused = fused  # pa_decode_append instead of pa_kv_append + pa_decode
+        self.graph = graph
+        self.fixed_plan = fixed_plan or graph
         self.device = device
         B, H, D, S = loop.batch, loop.H, loop.D, loop.S
         self.B, self.H, self.D, self.S = B, H, D, S
@@ -80,6 +92,10 @@ class ContinuousBatching:
         self.out = torch.empty((B, H, D), dtype=torch.float32, device=device)
         ws = binding.pa_decode_workspace_bytes(B, H, D, S, self.max_len, 0)
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        self.q_buf = torch.empty((B, H, D), dtype=loop.dtype, device=device)
+        self.k_buf = torch.empty_like(self.q_buf)
+        self.v_buf = torch.empty_like(self.q_buf)
+        self.graphs = [None] * len(self.staging.sets)
         self.events = []  # (kind, seq_id, serial, prompt_len) for admissions / retirements
         for b in range(B):
             self.slots.append(self._admit(loop.initial_lens[b], loop.budgets[b]))
@@ -98,17 +114,12 @@ class ContinuousBatching:
     def seq_ids(self):
         return [s[0] for s in self.slots]
 
-    def step(self, step_idx):
-        """One decode step; returns a record of what it did (for checking)."""
-        ids = self.seq_ids()
-        h = self.staging.acquire()
-        self.alloc.pa_prepare_step(ids, 1, self.MB, h["slots"], h["tables"], h["lens"])
+    def _device_step(self, h, max_len):
+        """Uploads from staging set h, then append + decode (eager or under capture)."""
         self.d_slots.copy_(h["slots"], non_blocking=True)
         self.d_tables.copy_(h["tables"], non_blocking=True)
         self.d_lens.copy_(h["lens"], non_blocking=True)
-        self.staging.release()
-        q, k, v = self.loop.token_kv(step_idx, self.B, self.device)
-        max_len = int(h["lens"].max())
+        q, k, v = (self.q_buf, self.k_buf, self.v_buf) if self.fixed_plan else self._qkv
         if self.fused:
             binding.pa_decode_append(self.out, q, k, v, self.k_cache, self.v_cache,
                                      self.d_tables, self.d_lens, self.scale, max_len,
@@ -117,6 +128,30 @@ class ContinuousBatching:
             binding.pa_kv_append(k, v, self.d_slots, self.k_cache, self.v_cache)
             binding.pa_decode(self.out, q, self.k_cache, self.v_cache, self.d_tables,
                               self.d_lens, self.scale, max_len, partition=0, workspace=self.ws)
+
+    def step(self, step_idx):
+        """One decode step; returns a record of what it did (for checking)."""
+        ids = self.seq_ids()
+        set_idx = self.staging.k % len(self.staging.sets)
+        h = self.staging.acquire()
+        self.alloc.pa_prepare_step(ids, 1, self.MB, h["slots"], h["tables"], h["lens"])
+        q, k, v = self.loop.token_kv(step_idx, self.B, self.device)
+        self._qkv = (q, k, v)
+        if self.fixed_plan:
+            self.q_buf.copy_(q)
+            self.k_buf.copy_(k)
+            self.v_buf.copy_(v)
+        max_len = self.max_len if self.fixed_plan else int(h["lens"].max())
+        if self.graph and self.graphs[set_idx] is not None:
+            self.graphs[set_idx].replay()
+        else:
+            self._device_step(h, max_len)
+            if self.graph:  # capture this staging set's step for the steps that reuse it
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    self._device_step(h, max_len)
+                self.graphs[set_idx] = g
+        self.staging.release()
         record = dict(ids=ids, slots=h["slots"].clone(), lens=h["lens"].clone(),
                       tables=h["tables"].clone(), q=q, k=k, v=v, out=self.out, retired=[],
                       admitted=[])
