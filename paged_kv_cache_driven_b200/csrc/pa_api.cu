@@ -197,10 +197,10 @@ bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_ro
 
 // Grouped query heads: one CTA per (partition, KV head, request, chunk of up to
 // 16 query heads), the contraction on the tensor cores.
-template <typename T, typename TO, int D, int S, bool APPEND>
+template <typename T, typename TO, int D, int S, bool APPEND, int NHT>
 pa_status launch_grouped(const pa::DecodeParams& prm, cudaStream_t stream) {
   using Tg = pa::GqaTiling<D>;
-  auto kern = pa::paged_decode_gqa_kernel<T, TO, D, S, APPEND>;
+  auto kern = pa::paged_decode_gqa_kernel<T, TO, D, S, APPEND, NHT>;
   static bool configured[kMaxDevices] = {};
   if (!opt_in_smem(kern, Tg::SMEM, configured)) return PA_ERR_CUDA;
   const int64_t rows = static_cast<int64_t>(prm.NB) * prm.Hkv * S;
@@ -222,7 +222,8 @@ pa_status dispatch_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t
   const bool grouped = prm.H != prm.Hkv;
 #define PA_CASE(DD, SS)                                                            \
   if (D == DD && S == SS)                                                          \
-    return grouped ? launch_grouped<T, TO, DD, SS, APPEND>(prm, st)                \
+    return grouped ? (prm.H / prm.Hkv <= 8 ? launch_grouped<T, TO, DD, SS, APPEND, 1>(prm, st)   \
+                                           : launch_grouped<T, TO, DD, SS, APPEND, 2>(prm, st)) \
                    : launch_decode<T, TO, DD, SS, APPEND>(prm, st);
   PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
   PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)

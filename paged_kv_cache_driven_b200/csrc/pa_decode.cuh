@@ -429,13 +429,13 @@ struct GqaTiling {
   static constexpr int BOX = 16 * 128;          // one swizzled box: 16 rows x 64 elements
   static constexpr int TILE = (D / 64) * BOX;   // one K (or V) unit
   static constexpr int STAGE = 2 * TILE;
-  static constexpr int QPITCH = (D + 8) * 2;    // the Q tile, padded rows
-  static constexpr int SMEM_Q = ROWS * QPITCH;
   static constexpr int NC = 4;                  // consumer warps; unit u goes to warp u % NC
   static constexpr int NS = 2 * NC;             // two stages per consumer
   static constexpr int SMEM_MERGE = NC * ROWS * (D + 2) * 4;  // reuses the stages at the end
   static constexpr int SMEM_STAGES = NS * STAGE > SMEM_MERGE ? NS * STAGE : SMEM_MERGE;
   // + 1024: the stages start on a 1024-byte boundary (the swizzle period)
+  static constexpr int QPITCH = (D + 8) * 2;    // the Q tile (when Q is not kept in registers)
+  static constexpr int SMEM_Q = ROWS * QPITCH;
   static constexpr int SMEM = 1024 + SMEM_STAGES + SMEM_Q + 2 * NS * 8 + NS * 4;
 };
 
@@ -479,6 +479,14 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
                : "r"(smem_u32(p)));
 }
 
+// Transpose of an 8x8 matrix of 16-bit values held one packed pair per lane in
+// the accumulator layout (lane 4g + t: row g, columns 2t, 2t + 1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // Two fp32 -> a packed pair of 16-bit values (low half = first), round to nearest.
 template <typename T>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi);
@@ -498,16 +506,15 @@ __device__ __forceinline__ float2 unpack2(uint32_t x) {
   return Elem<T>::pair(x);
 }
 
-template <typename T, typename TO, int D, int S, bool APPEND>
+template <typename T, typename TO, int D, int S, bool APPEND, int NHT>
 __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
     paged_decode_gqa_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv) {
   using Tg = GqaTiling<D>;
-  constexpr int ROWS = Tg::ROWS, PITCH = Tg::QPITCH, TILE = Tg::TILE, STAGE = Tg::STAGE;
+  constexpr int ROWS = Tg::ROWS, TILE = Tg::TILE, STAGE = Tg::STAGE;
   constexpr int NS = Tg::NS, NC = Tg::NC;
   constexpr int BR = S < 16 ? S : 16;  // rows per box
   constexpr int SLAB = S * D * 2;
-  constexpr int NT = D / 8;   // 8-wide n-tiles of O
   constexpr int KS = D / 16;  // k-steps of S
 
   const int part = blockIdx.x;
@@ -621,21 +628,49 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   }
 
   // ---- consumers ----
-  const int gq = lane >> 2;  // accumulator row (and row + 8)
-  const int tq = lane & 3;   // accumulator column pair
-  // Q tile: rows < gc are query heads hk * G + c0 + row, the rest zero
-  for (int idx = threadIdx.x; idx < ROWS * (D / 8); idx += NC * 32) {
-    const int row = idx / (D / 8), ch = idx % (D / 8);
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (row < gc) {
-      const int64_t hq = static_cast<int64_t>(hk) * G + c0 + row;
-      val = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
-                                            ((static_cast<int64_t>(i) * p.H + hq) * D + ch * 8) * 2);
+  // The unit is worked transposed, tokens as the MMA rows and query heads as
+  // its 8-wide columns, so a group of G <= 8 heads fills the columns instead of
+  // padding 16 rows:  S^T[16 tok x 8 heads] = K[16 x D] . Q^T;  then
+  // O^T[D x 8 heads] += V^T[D x 16 tok] . P^T.
+  const int g = lane >> 2;  // accumulator row (token g and g + 8; d rows of O^T)
+  const int t = lane & 3;   // accumulator column pair (heads 2t, 2t + 1 of a column tile)
+  // Q^T as the B operand: head (column) g of column tile nt, elements 2t, 2t + 1
+  // (b0) and 2t + 8, 2t + 9 (b1) of each k-step. Small groups keep it in
+  // registers, loaded once from global memory; otherwise it is a shared tile
+  // (rows = heads, zero past gc) read with ldmatrix at every k-step.
+  constexpr bool QREG = NHT * KS <= 8;
+  uint32_t qb[QREG ? NHT : 1][QREG ? KS : 1][2];
+  if constexpr (QREG) {
+#pragma unroll
+    for (int nt = 0; nt < NHT; ++nt) {
+      const int row = 8 * nt + g;
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          static_cast<const uint8_t*>(p.q) +
+          ((static_cast<int64_t>(i) * p.H + static_cast<int64_t>(hk) * G + c0 +
+            min(row, gc - 1)) * D) * 2);
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        qb[nt][kk][0] = row < gc ? __ldg(qrow + kk * 8 + t) : 0u;
+        qb[nt][kk][1] = row < gc ? __ldg(qrow + kk * 8 + 4 + t) : 0u;
+      }
     }
-    *reinterpret_cast<uint4*>(qtile + row * PITCH + ch * 16) = val;
+  } else {
+    for (int idx = threadIdx.x; idx < ROWS * (D / 8); idx += NC * 32) {
+      const int row = idx / (D / 8), ch = idx % (D / 8);
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (row < gc) {
+        const int64_t hq = static_cast<int64_t>(hk) * G + c0 + row;
+        val = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
+                                              ((static_cast<int64_t>(i) * p.H + hq) * D + ch * 8) * 2);
+      }
+      *reinterpret_cast<uint4*>(qtile + row * Tg::QPITCH + ch * 16) = val;
+    }
+    // consumers only: the Q tile is complete before anyone reads it
+    asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
   }
-  // consumers only: the Q tile is complete before anyone reads it
-  asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
+  // ldmatrix lane address into the Q tile: head (lane & 7) + 8 (lane >> 4),
+  // 8-column half (lane >> 3) & 1 -> r0, r1 = b0, b1 of heads 0-7, r2, r3 of 8-15
+  const int q_row = (lane & 7) + 8 * (lane >> 4), q_c8 = ((lane >> 3) & 1) * 8;
   // fused append: the new token's rows, one 16-byte chunk per lane; the warp
   // that consumes the new token's unit patches them in
   const int t_new = L - 1;
@@ -659,17 +694,21 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   }
   __syncwarp();
 
-  float o[NT][4];
+  constexpr int MT = D / 16;  // 16-row tiles of O^T
+  float o[MT][NHT][4];
 #pragma unroll
-  for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max of rows gq and gq + 8 (base 2)
-  float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums
-  // ldmatrix lane addresses: A (Q) rows lane % 16, k half lane / 16; B (K) token
-  // (lane & 7) + 8 * (lane >> 4), k half (lane >> 3) & 1; B (V, transposed) token
-  // (lane & 7) + 8 * ((lane >> 3) & 1), d half lane >> 4; K and V through the swizzle
-  const int a_row = lane & 15, a_k8 = (lane >> 4) * 8;
-  const int kb_tok = (lane & 7) + 8 * (lane >> 4), kb_k8 = ((lane >> 3) & 1) * 8;
-  const int vb_tok = (lane & 7) + 8 * ((lane >> 3) & 1), vb_d8 = (lane >> 4) * 8;
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NHT; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+  float m[NHT][2], l[NHT][2];  // per head 8nt + 2t + e: running max (base 2), this lane's sum
+#pragma unroll
+  for (int nt = 0; nt < NHT; ++nt) m[nt][0] = m[nt][1] = -INFINITY, l[nt][0] = l[nt][1] = 0.f;
+  // ldmatrix lane addresses into a token-major 16 x 16 tile, giving the A
+  // fragment (rows g / g + 8, k halves 0-7 / 8-15 in r0 .. r3):
+  //   K (rows = tokens):            token lane & 15, column half lane >> 4
+  //   V^T via .trans (k = tokens):  token (lane & 7) + 8 (lane >> 4), d half (lane >> 3) & 1
+  const int k_tok = lane & 15, k_c8 = (lane >> 4) * 8;
+  const int v_tok = (lane & 7) + 8 * (lane >> 4), v_c8 = ((lane >> 3) & 1) * 8;
 
   for (int k = w; k < nunits; k += NC) {
     const int s = k % NS;
@@ -691,144 +730,142 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
       __syncwarp();
     }
 
-    // S = Q K^T for tokens 0-7 (sacc[0]) and 8-15 (sacc[1]); even and odd
-    // k-steps accumulate in separate registers so two MMA chains run at once
-    float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    float sodd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    // S^T = K Q^T; even and odd k-steps in separate registers (two MMA chains)
+    float sacc[NHT][4], sodd[NHT][4];
+#pragma unroll
+    for (int nt = 0; nt < NHT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = sodd[nt][e] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
-      uint32_t a[4], b[4];
-      ldsm_x4(a, qtile + a_row * PITCH + (kk * 16 + a_k8) * 2);
-      ldsm_x4(b, ktile + swz(kb_tok, (kk * 16 + kb_k8) >> 3));
-      float (&acc0)[4] = (kk & 1) ? sodd[0] : sacc[0];
-      float (&acc1)[4] = (kk & 1) ? sodd[1] : sacc[1];
-      mma16816<T>(acc0, a, b[0], b[1]);
-      mma16816<T>(acc1, a, b[2], b[3]);
+      uint32_t a[4];
+      ldsm_x4(a, ktile + swz(k_tok, (kk * 16 + k_c8) >> 3));
+      if constexpr (QREG) {
+#pragma unroll
+        for (int nt = 0; nt < NHT; ++nt)
+          mma16816<T>((kk & 1) ? sodd[nt] : sacc[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+      } else {
+        uint32_t b[4];
+        ldsm_x4(b, qtile + q_row * Tg::QPITCH + (kk * 16 + q_c8) * 2);
+#pragma unroll
+        for (int nt = 0; nt < NHT; ++nt)
+          mma16816<T>((kk & 1) ? sodd[nt] : sacc[nt], a, b[2 * nt], b[2 * nt + 1]);
+      }
     }
+    // scores (base 2), masked by selection: element e is token g + 8 (e >> 1),
+    // head 8 nt + 2t + (e & 1)
+    const bool tok_lo = (valid >> g) & 1u, tok_hi = (valid >> (g + 8)) & 1u;
+    uint32_t bhi[NHT][2], blo[NHT][2];
+    float al[NHT][2];
+    bool any_rescale = false;
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[j][e] += sodd[j][e];
-    // scores (base 2), masked by selection: accumulator element e of n-tile j is
-    // row gq + 8 * (e >> 1), token 8 * j + 2 * tq + (e & 1)
-    float sc[2][4];
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int nt = 0; nt < NHT; ++nt) {
+      float sc[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int tok = 8 * j + 2 * tq + (e & 1);
-        const bool ok = (valid >> tok) & 1u;
-        sc[j][e] = ok ? sacc[j][e] * p.q_scale : -INFINITY;
-        if (e < 2) mx0 = fmaxf(mx0, sc[j][e]); else mx1 = fmaxf(mx1, sc[j][e]);
+        const bool ok = (e >> 1) ? tok_hi : tok_lo;
+        sc[e] = ok ? (sacc[nt][e] + sodd[nt][e]) * p.q_scale : -INFINITY;
       }
+      float pr[4];
 #pragma unroll
-    for (int off = 1; off <= 2; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, off));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    // a unit with no valid token for a row keeps its max at -inf: guard the exponent
-    const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m0 - mn0);
-    const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
-    float pr[2][4];
-    float ls0 = 0.f, ls1 = 0.f;
+      for (int c = 0; c < 2; ++c) {  // head 8nt + 2t + c: max over the 16 tokens
+        float mx = fmaxf(sc[c], sc[c + 2]);
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float mref = e < 2 ? mn0 : mn1;
-        pr[j][e] = sc[j][e] == -INFINITY ? 0.f : exp2f(sc[j][e] - mref);
-        if (e < 2) ls0 += pr[j][e]; else ls1 += pr[j][e];
+        for (int off = 4; off <= 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
+        const float mn = fmaxf(m[nt][c], mx);
+        // a unit with no valid token for this head keeps its max at -inf
+        al[nt][c] = mn == -INFINITY ? 1.f : exp2f(m[nt][c] - mn);
+        any_rescale |= al[nt][c] != 1.f;
+        pr[c] = sc[c] == -INFINITY ? 0.f : exp2f(sc[c] - mn);
+        pr[c + 2] = sc[c + 2] == -INFINITY ? 0.f : exp2f(sc[c + 2] - mn);
+        l[nt][c] = l[nt][c] * al[nt][c] + pr[c] + pr[c + 2];
+        m[nt][c] = mn;
       }
-    l0 = l0 * al0 + ls0;
-    l1 = l1 * al1 + ls1;
-    m0 = mn0;
-    m1 = mn1;
-    // once the running max settles, most units change no row's max: skip the
-    // rescale of O unless some row of the warp needs it
-    if (__any_sync(kFullMask, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        o[n][0] *= al0;
-        o[n][1] *= al0;
-        o[n][2] *= al1;
-        o[n][3] *= al1;
+      // P^T as the B operand: tokens 2t, 2t + 1 (b0) and 2t + 8, 2t + 9 (b1) of
+      // head g, by transposing the accumulator-layout pairs. bf16 keeps 8 bits,
+      // so P goes in as a hi + lo pair (its rounding drops from 2^-9 to 2^-17);
+      // fp16 keeps 11, within the tolerance on its own.
+      const uint32_t h0 = pack2<T>(pr[0], pr[1]), h1 = pack2<T>(pr[2], pr[3]);
+      bhi[nt][0] = movmatrix_trans(h0);
+      bhi[nt][1] = movmatrix_trans(h1);
+      if (std::is_same<T, __nv_bfloat16>::value) {
+        const float2 f0 = unpack2<T>(h0), f1 = unpack2<T>(h1);
+        blo[nt][0] = movmatrix_trans(pack2<T>(pr[0] - f0.x, pr[1] - f0.y));
+        blo[nt][1] = movmatrix_trans(pack2<T>(pr[2] - f1.x, pr[3] - f1.y));
       }
     }
-    // P as the A operand (16 x 16 tokens). bf16 keeps 8 bits, so P goes in as a
-    // hi + lo pair (its rounding drops from 2^-9 to 2^-17); fp16 keeps 11, within
-    // the tolerance on its own, so only the hi part is used.
-    constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
-    uint32_t ph[4], plo[4];
+    // once the running max settles most units move no head's max
+    if (__any_sync(kFullMask, any_rescale)) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      ph[2 * j] = pack2<T>(pr[j][0], pr[j][1]);      // row gq, tokens 8j + 2tq, +1
-      ph[2 * j + 1] = pack2<T>(pr[j][2], pr[j][3]);  // row gq + 8
-      if (kSplitP) {
-        const float2 h0 = unpack2<T>(ph[2 * j]), h1 = unpack2<T>(ph[2 * j + 1]);
-        plo[2 * j] = pack2<T>(pr[j][0] - h0.x, pr[j][1] - h0.y);
-        plo[2 * j + 1] = pack2<T>(pr[j][2] - h1.x, pr[j][3] - h1.y);
-      }
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NHT; ++nt) {
+          o[mt][nt][0] *= al[nt][0];
+          o[mt][nt][1] *= al[nt][1];
+          o[mt][nt][2] *= al[nt][0];
+          o[mt][nt][3] *= al[nt][1];
+        }
     }
-    // A-fragment order: (row gq, k 0-7), (row gq+8, k 0-7), (row gq, k 8-15), (row gq+8, k 8-15)
-    const uint32_t ahi[4] = {ph[0], ph[1], ph[2], ph[3]};
-    const uint32_t alo[4] = {plo[0], plo[1], plo[2], plo[3]};
-    // V rows that were not copied are zeroed in the B fragments (0 * NaN would be NaN)
+    // V^T as the A operand (ldmatrix.trans of the token-major tile); tokens that
+    // were not copied are zeroed in it (0 * NaN would be NaN)
     const bool partial = valid != 0xffffu;
-    const uint32_t vm0 = (((valid >> (2 * tq)) & 1u) ? 0x0000ffffu : 0u) |
-                         (((valid >> (2 * tq + 1)) & 1u) ? 0xffff0000u : 0u);
-    const uint32_t vm1 = (((valid >> (2 * tq + 8)) & 1u) ? 0x0000ffffu : 0u) |
-                         (((valid >> (2 * tq + 9)) & 1u) ? 0xffff0000u : 0u);
+    const uint32_t vm0 = (((valid >> (2 * t)) & 1u) ? 0x0000ffffu : 0u) |
+                         (((valid >> (2 * t + 1)) & 1u) ? 0xffff0000u : 0u);
+    const uint32_t vm1 = (((valid >> (2 * t + 8)) & 1u) ? 0x0000ffffu : 0u) |
+                         (((valid >> (2 * t + 9)) & 1u) ? 0xffff0000u : 0u);
 #pragma unroll
-    for (int n2 = 0; n2 < NT / 2; ++n2) {
-      uint32_t b[4];
-      ldsm_x4_trans(b, vtile + swz(vb_tok, (n2 * 16 + vb_d8) >> 3));
+    for (int mt = 0; mt < MT; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_trans(a, vtile + swz(v_tok, (mt * 16 + v_c8) >> 3));
       if (partial) {
-        b[0] &= vm0;
-        b[1] &= vm1;
-        b[2] &= vm0;
-        b[3] &= vm1;
+        a[0] &= vm0;
+        a[1] &= vm0;
+        a[2] &= vm1;
+        a[3] &= vm1;
       }
-      mma16816<T>(o[2 * n2], ahi, b[0], b[1]);
-      mma16816<T>(o[2 * n2 + 1], ahi, b[2], b[3]);
-      if (kSplitP) {
-        mma16816<T>(o[2 * n2], alo, b[0], b[1]);
-        mma16816<T>(o[2 * n2 + 1], alo, b[2], b[3]);
+#pragma unroll
+      for (int nt = 0; nt < NHT; ++nt) {
+        mma16816<T>(o[mt][nt], a, bhi[nt][0], bhi[nt][1]);
+        if (std::is_same<T, __nv_bfloat16>::value)
+          mma16816<T>(o[mt][nt], a, blo[nt][0], blo[nt][1]);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
 
-  // row sums over the lane quad
+  // head sums over the 8 lanes that share t
 #pragma unroll
-  for (int off = 1; off <= 2; off <<= 1) {
-    l0 += __shfl_xor_sync(kFullMask, l0, off);
-    l1 += __shfl_xor_sync(kFullMask, l1, off);
-  }
-  // merge the NC consumers' (m, l, O) per row through shared memory (the stages
+  for (int nt = 0; nt < NHT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int off = 4; off <= 16; off <<= 1)
+        l[nt][c] += __shfl_xor_sync(kFullMask, l[nt][c], off);
+  // merge the NC consumers' (m, l, O) per head through shared memory (the stages
   // are free: every unit has been consumed once all consumers pass the barrier)
   asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
-  float* mg = reinterpret_cast<float*>(stages);  // [NC][ROWS][D + 2]: m, l, O
+  float* mg = reinterpret_cast<float*>(stages);  // [NC][ROWS][D + 2]: m, l, O per head
   {
     float* mine = mg + w * ROWS * (D + 2);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float* rowp = mine + (gq + 8 * half) * (D + 2);
-      if (tq == 0) {
-        rowp[0] = half ? m1 : m0;
-        rowp[1] = half ? l1 : l0;
-      }
+    for (int nt = 0; nt < NHT; ++nt)
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        rowp[2 + 8 * n + 2 * tq] = o[n][2 * half];
-        rowp[2 + 8 * n + 2 * tq + 1] = o[n][2 * half + 1];
+      for (int c = 0; c < 2; ++c) {
+        float* rowp = mine + (8 * nt + 2 * t + c) * (D + 2);
+        if (g == 0) {
+          rowp[0] = m[nt][c];
+          rowp[1] = l[nt][c];
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          rowp[2 + 16 * mt + g] = o[mt][nt][c];
+          rowp[2 + 16 * mt + g + 8] = o[mt][nt][c + 2];
+        }
       }
-    }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
-  // consumer w finishes rows w, w + NC, ...: M = max m, out = sum 2^(m - M) O / sum 2^(m - M) l
+  // consumer w finishes heads w, w + NC, ...: M = max m, out = sum 2^(m - M) O / sum 2^(m - M) l
   for (int row = w; row < gc; row += NC) {
     float M = -INFINITY;
 #pragma unroll
