@@ -431,6 +431,10 @@ struct GqaTiling {
   static constexpr int STAGE = 2 * TILE;
   static constexpr int NC = 4;                  // consumer warps; unit u goes to warp u % NC
   static constexpr int NS = 2 * NC;             // two stages per consumer
+  // Consumer w takes units w, w + NC, ...; a stage is reused every NS units, so
+  // with NS a multiple of NC each stage's units belong to one consumer and it
+  // never waits on a stage phase two ahead (which a parity wait cannot tell apart).
+  static_assert(NS % NC == 0, "stages must be a multiple of the consumer count");
   static constexpr int SMEM_MERGE = NC * ROWS * (D + 2) * 4;  // reuses the stages at the end
   static constexpr int SMEM_STAGES = NS * STAGE > SMEM_MERGE ? NS * STAGE : SMEM_MERGE;
   // + 1024: the stages start on a 1024-byte boundary (the swizzle period)
