@@ -155,3 +155,30 @@ def test_prompt_prefill_full_size_sampled():
     got = torch.stack([out[qs[i] + j, h] for i, j, h in picks]).cpu().numpy()
     assert_parity(got, want, "prompt prefill sampled rows")
     assert bool(torch.isfinite(out).all())
+
+
+@pytest.mark.parametrize("dt,Hkv", [(torch.float16, 32), (torch.bfloat16, 8)],
+                         ids=["fp16", "gqa_64q_8kv"])
+def test_chunked_prefill_large_sampled(dt, Hkv):
+    """Chunked prefill at scale: 8 requests with U[0, 6000] cached tokens and
+    U[300, 2500] new ones, head_dim 128, block 16; fp16 with 32 heads, and 64
+    query heads on 8 KV heads (LLaMA-2-70B-shaped groups). Sampled rows against
+    the oracle's decode of the row's prefix."""
+    g = torch.Generator().manual_seed(11)
+    ctx = torch.randint(0, 6001, (8,), generator=g).tolist()
+    new = torch.randint(300, 2501, (8,), generator=g).tolist()
+    H = 32 if Hkv == 32 else 64
+    pc = workloads.prefill_case(ctx, new, H=H, D=128, S=16, dtype=dt, seed=12, device=DEV,
+                                Hkv=Hkv)
+    out = run_prefill(pc)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    picks = []
+    for i in range(8):
+        for j in (0, new[i] - 1, int(torch.randint(0, new[i], (1,), generator=g))):
+            picks.append((i, j, int(torch.randint(0, H, (1,), generator=g))))
+    want = oracle_prefill_rows(pc, picks)
+    qs = pc.q_start.cpu().tolist()
+    got = torch.stack([out[qs[i] + j, h] for i, j, h in picks]).cpu().numpy()
+    assert_parity(got, want, f"chunked prefill {dt} Hkv={Hkv}")
+    assert bool(torch.isfinite(out).all())
