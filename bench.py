@@ -166,11 +166,12 @@ def measured_peak():
 
 
 def kernel_source_hash():
-    """Hash of the decode kernels' source with comments and blank lines removed,
-    so a profile stays attached to the code it measured and nothing else."""
+    """Hash of the headline call's kernels (the partition pass and the reduce,
+    with the device helpers they use), comments and blank lines removed, so a
+    profile stays attached to the kernel code it measured and nothing else."""
     import re
     h = hashlib.sha256()
-    for f in ("pa_decode.cuh", "pa_device.cuh", "pa_api.cu"):
+    for f in ("pa_decode.cuh", "pa_device.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_driven_b200", "csrc", f)) as fh:
             text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
         lines = [re.sub(r"//.*", "", l).rstrip() for l in text.splitlines()]

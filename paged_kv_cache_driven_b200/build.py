@@ -13,7 +13,8 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpagedattn.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("pa_api.cu", "pa_alloc.cpp", "pa_stepper.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_device.cuh", "pa_decode.cuh", "pa_append.cuh",
-                                                      "pa_prefill.cuh", "pa_tcgen05.cuh")] \
+                                                      "pa_gqa.cuh", "pa_prefill.cuh",
+                                                      "pa_tcgen05.cuh")] \
     + [os.path.join(ROOT, "include", "pagedattn.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

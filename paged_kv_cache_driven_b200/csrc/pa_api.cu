@@ -17,6 +17,7 @@
 
 #include "pa_append.cuh"
 #include "pa_decode.cuh"
+#include "pa_gqa.cuh"
 #include "pa_prefill.cuh"
 #include "pagedattn.h"
 
