@@ -184,9 +184,10 @@ pa_status pa_prefill(void* out, pa_dtype out_dt, const void* q, const void* k_ca
  * Grouped-query decode (not on the pages, which have one KV head per query
  * head): the cache holds Hkv KV heads, [NB, Hkv, S, D]; q and out hold H query
  * heads, H a multiple of Hkv, and query head h reads KV head h / (H / Hkv)
- * (consecutive query heads share a KV head). When H / Hkv is even, one CTA
- * serves up to 8 query heads of a KV head from one staged copy of each K/V
- * unit, so every K/V byte is read from HBM once per group. k_new, v_new
+ * (consecutive query heads share a KV head). For H > Hkv one CTA serves up to
+ * 16 query heads of a KV head from one staged copy of each K/V unit (on the
+ * tensor cores), so every K/V byte is read from HBM once per group of up to 16
+ * heads. k_new, v_new
  * ([B, Hkv, D]) are optional together: when given, the step's new token is
  * appended at position seq_lens[i] - 1 first, exactly as pa_decode_append.
  * Everything else (dtypes, D, S, partition, workspace sized by

@@ -1,6 +1,8 @@
 // The device half of the C ABI (pagedattn.h): argument validation, launch
-// planning and kernel dispatch for pa_kv_append and pa_decode, and the device
-// error word. Every check runs on the host before anything is launched.
+// planning, tensor-map encoding and kernel dispatch for pa_kv_append,
+// pa_decode / pa_decode_append / pa_decode_gqa / pa_decode_noalloc,
+// pa_prefill and pa_copy_blocks, and the device error word. Every check runs
+// on the host before anything is launched.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
