@@ -206,9 +206,75 @@ bool valid_problem(const Problem& p) {
          p.Hkv > 0 && p.H % p.Hkv == 0;
 }
 
+// FP8 E4M3 (the OCP 8-bit floating-point format, "fn" variant: no infinities):
+// sign bit 7, exponent bits 6-3 with bias 7, mantissa bits 2-0. Exponent 0 is
+// subnormal (m * 2^-9); exponent 15 with mantissa 7 is NaN; everything else is
+// (1 + m / 8) * 2^(e - 7). Not on the pages: a storage format for the paged cache.
+double decode_e4m3(uint8_t bits) {
+  const int sign = bits >> 7, e = (bits >> 3) & 15, m = bits & 7;
+  double v;
+  if (e == 15 && m == 7) {
+    v = std::numeric_limits<double>::quiet_NaN();
+  } else if (e == 0) {
+    v = std::ldexp(static_cast<double>(m), -9);
+  } else {
+    v = std::ldexp(1.0 + m / 8.0, e - 7);
+  }
+  return sign ? -v : v;
+}
+
 }  // namespace
 
 extern "C" {
+
+double oracle_decode_e4m3(uint8_t bits) { return decode_e4m3(bits); }
+
+// Paged decode over an FP8 E4M3 cache with one scale per tensor: K_t = k_scale *
+// e4m3(k_cache[...]), V_t likewise; q (16-bit, q_dtype 0 = binary16, 1 = bfloat16)
+// [B, H, D]; out[i, h] = softmax_t(scale * q . K_t) V_t over the first seq_lens[i]
+// tokens, two-pass in fp64, exactly as oracle_paged_decode with dequantized K/V.
+int oracle_paged_decode_fp8(const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                            double k_scale, double v_scale, const int32_t* block_tables,
+                            const int32_t* seq_lens, int64_t B, int64_t H, int64_t Hkv,
+                            int64_t D, int64_t S, int64_t NB, int64_t MB, double scale,
+                            int q_dtype, int n_threads, double* out) {
+  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out || B < 0 || H <= 0 ||
+      Hkv <= 0 || H % Hkv || D <= 0 || S <= 0 || NB < 0 || MB < 0 || (q_dtype != 0 && q_dtype != 1))
+    return 1;
+  const int64_t G = H / Hkv;
+  return parallel_for(B * H, n_threads, [&](int64_t k) {
+    const int64_t i = k / H, h = k % H;
+    double* o = out + k * D;
+    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    const int64_t L = seq_lens[i];
+    if (L < 0 || L > MB * S) return 3;
+    if (L == 0) return 0;
+    std::vector<double> sc(static_cast<size_t>(L));
+    std::vector<int64_t> rows(static_cast<size_t>(L));
+    for (int64_t t = 0; t < L; ++t) {
+      const int64_t blk = block_tables[i * MB + t / S];
+      if (blk < 0 || blk >= NB) return 3;
+      const int64_t row = ((blk * Hkv + h / G) * S + t % S) * D;
+      rows[t] = row;
+      double dot = 0.0;
+      for (int64_t d = 0; d < D; ++d) {
+        const uint16_t qb = q[(i * H + h) * D + d];
+        const double qv = q_dtype == 0 ? decode_binary16(qb) : decode_bfloat16(qb);
+        dot += qv * (k_scale * decode_e4m3(k_cache[row + d]));
+      }
+      sc[t] = scale * dot;
+    }
+    double m = -std::numeric_limits<double>::infinity();
+    for (double x : sc) m = std::max(m, x);
+    double z = 0.0;
+    for (double x : sc) z += std::exp(x - m);
+    for (int64_t t = 0; t < L; ++t) {
+      const double w = std::exp(sc[t] - m) / z;
+      for (int64_t d = 0; d < D; ++d) o[d] += w * (v_scale * decode_e4m3(v_cache[rows[t] + d]));
+    }
+    return 0;
+  });
+}
 
 // Decodes one 16-bit element (dtype 0 = binary16, 1 = bfloat16) to double.
 double oracle_decode16(uint16_t bits, int dtype) {
