@@ -10,7 +10,10 @@ value = scale * decode(stored).
 Quantization is round to nearest, ties to the even code, with out-of-range
 magnitudes saturated to 448 (reading: the usual "satfinite" conversion; the
 kernel's append does the same, and the pins check it against torch's own
-float8_e4m3fn conversion wherever that one is defined).
+float8_e4m3fn conversion wherever that one is defined). The quotient x / scale
+is taken in fp32 with one correctly rounded division before it is rounded to a
+code: a quantised code is an integer decided by floating point, so both sides
+take it in the kernel's precision (the inputs are 16-bit, exact in fp32).
 """
 
 import ctypes
@@ -45,9 +48,9 @@ def decode_table():
 
 
 def quantize(x, scale):
-    """Codes (uint8) of x / scale: round to nearest, ties to even code, saturate
-    at 448. x is any float array; NaN inputs give 0x7F."""
-    y = np.asarray(x, dtype=np.float64) / float(scale)
+    """Codes (uint8) of fp32(x / scale): round to nearest, ties to even code,
+    saturate at 448. x is any float array (taken as fp32); NaN gives 0x7F."""
+    y = (np.asarray(x, dtype=np.float32) / np.float32(scale)).astype(np.float64)
     table = decode_table()
     mags = table[:127]  # codes 0 .. 126: the finite non-negative values, increasing
     a = np.minimum(np.abs(y), mags[-1])

@@ -29,7 +29,7 @@ def test_decode_table_matches_torch():
 
 def test_quantize_matches_torch_in_range():
     g = torch.Generator().manual_seed(0)
-    x = torch.cat([torch.randn(20000, generator=g, dtype=torch.float64) * s
+    x = torch.cat([torch.randn(20000, generator=g, dtype=torch.float32) * s
                    for s in (1e-3, 0.1, 1.0, 30.0, 200.0)])
     x = x[x.abs() <= 448]
     want = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
@@ -49,8 +49,11 @@ def test_quantize_rules():
         mid = (table[c] + table[c + 1]) / 2
         q = int(ofp8.quantize(np.array([mid]), 1.0)[0])
         assert q == (c if c % 2 == 0 else c + 1)
-    # the scale divides first
+    # the scale divides first, in fp32
     assert ofp8.quantize(np.array([3.0]), 2.0)[0] == ofp8.quantize(np.array([1.5]), 1.0)[0]
+    x = torch.randn(5000, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).float()
+    want = (x / torch.tensor(0.037)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ofp8.quantize(x.numpy(), 0.037), want)
 
 
 @pytest.mark.parametrize("H,Hkv", [(4, 4), (8, 2)])
