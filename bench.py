@@ -450,6 +450,44 @@ def time_decode_case(case, iters, warmup, partition=0):
     return statistics.median(times), binding.pa_decode_plan(B, Hc, Dc, Sc, maxlen, partition)
 
 
+def time_decode_fp8(seed, iters, warmup):
+    """The LLaMA-2-13B decode shape over an E4M3 cache (filled by pa_kv_append_fp8
+    from the bf16 case): median event-timed pa_decode_fp8 call with L2 flushed
+    before each; returns (ms, KV bytes, plan)."""
+    device = torch.device("cuda", 0)
+    case = workloads.llama13b_decode(seed=seed, device=device)
+    B, Hc, Dc = case.q.shape
+    NB, _, Sc, _ = case.k_cache.shape
+    kc8 = torch.empty((NB, Hc, Sc, Dc), dtype=torch.uint8, device=device)
+    vc8 = torch.empty_like(kc8)
+    slots = torch.arange(NB * Sc, dtype=torch.int64, device=device)
+    binding.pa_kv_append_fp8(case.k_cache.permute(0, 2, 1, 3).reshape(-1, Hc, Dc).contiguous(),
+                             case.v_cache.permute(0, 2, 1, 3).reshape(-1, Hc, Dc).contiguous(),
+                             slots, kc8, vc8, 0.05, 0.08)
+    del case.k_cache, case.v_cache
+    maxlen = max(case.seq_lens_host)
+    out = torch.empty((B, Hc, Dc), dtype=DTYPE, device=device)
+    wsb = binding.pa_decode_workspace_bytes(B, Hc, Dc, Sc, maxlen, 0)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    times = []
+    for k in range(warmup + iters):
+        flush.fill_(k & 0xff)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        binding.pa_decode_fp8(out, case.q, kc8, vc8, 0.05, 0.08, case.block_tables,
+                              case.seq_lens, case.scale, maxlen, partition=0, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        if k >= warmup:
+            times.append(a.elapsed_time(b))
+    if binding.pa_get_device_error():
+        raise SystemExit("device error word set")
+    nbytes = sum(Hc * (2 * L * Dc + 2 * Dc * 2) + 4 * (-(-L // Sc)) for L in case.seq_lens_host) \
+        + 4 * B
+    return statistics.median(times), nbytes, binding.pa_decode_plan(B, Hc, Dc, Sc, maxlen, 0)
+
+
 def run_shape_workloads(args):
     """--workload long_context | sweep: decode-only KV GB/s of the other
     configurations, one JSON line per case (L2 flushed before every call)."""
@@ -458,6 +496,14 @@ def run_shape_workloads(args):
     if args.workload == "long_context":
         cases = [("long_context", lambda: workloads.long_context_decode(seed=args.seed,
                                                                         device=device))]
+    elif args.workload == "llama13b_fp8":
+        ms, nbytes, plan = time_decode_fp8(args.seed, args.steps, args.warmup)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        print(json.dumps({"workload": "llama13b_fp8_e4m3_cache", "ms": round(ms, 4),
+                          "gb_s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 3),
+                          "kv_bytes": nbytes, "tok_s_layer": round(64 / (ms / 1e3), 1),
+                          "partition": {"tokens": plan[0], "num": plan[1]}}), flush=True)
+        return
     elif args.workload == "llama70b":
         cases = [("llama70b_gqa_64q_8kv", lambda: workloads.llama70b_decode(seed=args.seed,
                                                                             device=device))]
@@ -684,8 +730,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="llama13b",
-                    choices=["llama13b", "long_context", "sweep", "llama70b", "prompt_prefill",
-                             "prompt_prefill_small"],
+                    choices=["llama13b", "long_context", "sweep", "llama70b", "llama13b_fp8",
+                             "prompt_prefill", "prompt_prefill_small"],
                     help="llama13b: the headline step (default); the others time decode-only "
                          "calls of the long-context, shape-sweep and LLaMA-2-70B-shaped "
                          "grouped-query configurations, or paged prefill attention over "

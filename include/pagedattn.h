@@ -141,6 +141,35 @@ pa_status pa_decode_append(void* out, pa_dtype out_dt, const void* q, const void
                            void* stream);
 
 /* ---------------------------------------------------------------------------
+ * FP8 E4M3 KV cache (not on the pages, which keep K/V in 16-bit; a storage
+ * extension that halves the bytes decode reads). The caches are [NB, H, S, D]
+ * uint8 arrays of E4M3 codes ("fn" variant: sign bit 7, exponent bits 6-3 with
+ * bias 7, mantissa bits 2-0, no infinities, largest magnitude 448), one fp32
+ * scale per tensor: K = k_scale * e4m3(code), V = v_scale * e4m3(code).
+ *
+ * pa_kv_append_fp8: the slot_mapping scatter of pa_kv_append, storing each
+ * element of k / v ([T, H, D], in_dt F16 or BF16, 16-byte aligned) as the code
+ * of fp32(x / scale) -- one correctly rounded fp32 division, then round to
+ * nearest even, magnitudes past 448 saturated. D a multiple of 16; scales
+ * finite and > 0. Slots and errors as pa_kv_append.
+ * ------------------------------------------------------------------------- */
+pa_status pa_kv_append_fp8(const void* k, const void* v, pa_dtype in_dt,
+                           const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                           float k_scale, float v_scale, int T, int H, int D, int S, int NB,
+                           void* stream);
+
+/* pa_decode over E4M3 caches: q [B, H, D] (q_dt F16 or BF16), out as pa_decode;
+ * out[i, h] = softmax_t(scale * q . K_t) V_t with K_t, V_t dequantized as above
+ * (k_scale is folded into the scores, v_scale into the output). D, S,
+ * partition, workspace (pa_decode_workspace_bytes) and errors as pa_decode; one
+ * KV head per query head; no fused append (append with pa_kv_append_fp8). */
+pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
+                        const void* k_cache, const void* v_cache, float k_scale, float v_scale,
+                        const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
+                        int B, int H, int D, int S, int NB, int partition, int max_seq_len,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Paged prefill attention ("vLLM KV Cache and PagedAttention Explained", Step 6
  * "Prefill and Decode": every prompt token is processed at once, and each one
  * attends to the tokens before it and to itself; the attention formula of its

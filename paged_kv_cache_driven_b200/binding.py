@@ -38,6 +38,14 @@ _SIGNATURES = {
                        _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_decode_noalloc": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32,
                            _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    # k, v, in_dt, slot_mapping, k_cache, v_cache, k_scale, v_scale, T, H, D, S, NB, stream
+    "pa_kv_append_fp8": ([_vp, _vp, _i32, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, _i32,
+                          _i32, _i32, _i32, _i32, _vp], _i32),
+    # out, out_dt, q, q_dt, k_cache, v_cache, k_scale, v_scale, block_tables, MB, seq_lens,
+    # scale, B, H, D, S, NB, partition, max_seq_len, workspace, ws_bytes, stream
+    "pa_decode_fp8": ([_vp, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _i32,
+                       _vp, ctypes.c_float, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz,
+                       _vp], _i32),
     # out, out_dt, q, k_cache, v_cache, block_tables, MB, seq_lens, q_start, scale,
     # B, H, Hkv, D, S, NB, dt, T, max_q_len, stream
     "pa_prefill": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_float, _i32, _i32,
@@ -240,6 +248,48 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, q_start, scale,
                             _ptr(block_tables), MB, _ptr(seq_lens), _ptr(q_start), float(scale),
                             B, H, Hkv, D, S, NB, _DT[q.dtype], T, int(max_q_len),
                             _stream(stream)), "pa_prefill")
+
+
+def pa_kv_append_fp8(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale, stream=None):
+    """Scatter k, v [T, H, D] (fp16/bf16) into uint8 E4M3 caches [NB, H, S, D]
+    as codes of fp32(x / scale), round to nearest even, saturated at 448."""
+    for n, t in (("k", k), ("v", v), ("slot_mapping", slot_mapping), ("k_cache", k_cache),
+                 ("v_cache", v_cache)):
+        _cuda(t, n)
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise ValueError("E4M3 caches are uint8 tensors of codes")
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    T, H, D = k.shape
+    NB, H2, S, D2 = k_cache.shape
+    if (H2, D2) != (H, D) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("shape mismatch")
+    _check(lib().pa_kv_append_fp8(_ptr(k), _ptr(v), _DT[k.dtype], _ptr(slot_mapping), _ptr(k_cache),
+                                  _ptr(v_cache), float(k_scale), float(v_scale), T, H, D, S, NB,
+                                  _stream(stream)), "pa_kv_append_fp8")
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_lens, scale,
+                  max_seq_len, partition=0, workspace=None, stream=None):
+    """Decode over uint8 E4M3 caches [NB, H, S, D] with per-tensor scales."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                 ("block_tables", block_tables), ("seq_lens", seq_lens)):
+        _cuda(t, n)
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise ValueError("E4M3 caches are uint8 tensors of codes")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    B, H, D = q.shape
+    NB, H2, S, _ = k_cache.shape
+    if H2 != H:
+        raise ValueError("the E4M3 decode has one KV head per query head")
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_decode_fp8(_ptr(out), _DT[out.dtype], _ptr(q), _DT[q.dtype], _ptr(k_cache),
+                               _ptr(v_cache), float(k_scale), float(v_scale), _ptr(block_tables),
+                               MB, _ptr(seq_lens), float(scale), B, H, D, S, NB, int(partition),
+                               int(max_seq_len), _ptr(workspace), ws_bytes, _stream(stream)),
+           "pa_decode_fp8")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

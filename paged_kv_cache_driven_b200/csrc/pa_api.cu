@@ -220,6 +220,30 @@ pa_status launch_grouped(const pa::DecodeParams& prm, cudaStream_t stream) {
   return cuda_status();
 }
 
+// E4M3 cache: the multi-head kernel with one-byte cache elements.
+template <typename T, typename TO, int D, int S>
+pa_status launch_decode_fp8(const pa::DecodeParams& prm, cudaStream_t stream) {
+  using Tl = pa::DecodeTiling<D, S, 1>;
+  auto kern = pa::paged_decode_partition_kernel<T, TO, D, S, false, __nv_fp8_e4m3>;
+  static bool configured[kMaxDevices] = {};
+  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
+  const dim3 grid(prm.NP, prm.H, prm.B);
+  kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
+  launch_reduce<TO, D>(prm, stream);
+  return cuda_status();
+}
+
+template <typename T, typename TO>
+pa_status dispatch_fp8_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t st) {
+#define PA_CASE(DD, SS) \
+  if (D == DD && S == SS) return launch_decode_fp8<T, TO, DD, SS>(prm, st);
+  PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
+  PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
+  PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
+#undef PA_CASE
+  return PA_ERR_INVALID;
+}
+
 template <typename T, typename TO, bool APPEND>
 pa_status dispatch_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t st) {
   const bool grouped = prm.H != prm.Hkv;
@@ -414,6 +438,7 @@ pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_n
   prm.block_tables = block_tables;
   prm.seq_lens = seq_lens;
   prm.q_scale = scale * 1.4426950408889634f;  // log2(e)
+  prm.v_scale = 1.f;
   prm.MB = MB;
   prm.B = B;
   prm.H = H;
@@ -519,6 +544,105 @@ pa_status pa_prefill(void* out, pa_dtype out_dt, const void* q, const void* k_ca
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   return dt == PA_BF16 ? dispatch_prefill<__nv_bfloat16>(prm, q, out_dt, D, S, st)
                        : dispatch_prefill<__half>(prm, q, out_dt, D, S, st);
+}
+
+pa_status pa_kv_append_fp8(const void* k, const void* v, pa_dtype in_dt,
+                           const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                           float k_scale, float v_scale, int T, int H, int D, int S, int NB,
+                           void* stream) {
+  if (T < 0 || H <= 0 || D <= 0 || S <= 0 || NB < 0 || !cache_dtype_ok(in_dt)) return PA_ERR_INVALID;
+  if (D % 16 != 0) return PA_ERR_INVALID;  // 8-byte code vectors, 16-byte cache rows
+  if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+    return PA_ERR_INVALID;
+  if (T == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  const int vpr = D / 8;
+  const int64_t total = static_cast<int64_t>(T) * H * vpr;
+  const int64_t n_slots = static_cast<int64_t>(NB) * S;
+  int64_t blocks = ceil_div(total, 256);
+  const int64_t cap = 148LL * 16;
+  if (blocks > cap) blocks = cap;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (in_dt == PA_BF16)
+    pa::kv_append_fp8_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+        static_cast<uint2*>(k_cache), static_cast<uint2*>(v_cache), k_scale, v_scale, total, H,
+        vpr, S, n_slots);
+  else
+    pa::kv_append_fp8_kernel<__half><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+        static_cast<uint2*>(k_cache), static_cast<uint2*>(v_cache), k_scale, v_scale, total, H,
+        vpr, S, n_slots);
+  return cuda_status();
+}
+
+pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
+                        const void* k_cache, const void* v_cache, float k_scale, float v_scale,
+                        const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
+                        int B, int H, int D, int S, int NB, int partition, int max_seq_len,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  if (B < 0 || H <= 0 || NB < 0 || MB < 0) return PA_ERR_INVALID;
+  if (!cache_dtype_ok(q_dt) || !out_dtype_ok(out_dt) || !decode_shape_ok(D, S)) return PA_ERR_INVALID;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID;
+  if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+    return PA_ERR_INVALID;
+  if (B > 65535 || H > 65535) return PA_ERR_INVALID;
+  const int64_t L_max = static_cast<int64_t>(MB) * S;
+  if (L_max > INT_MAX || max_seq_len < 0 || max_seq_len > L_max) return PA_ERR_INVALID;
+  int P, NP;
+  if (!plan(B, H, S, max_seq_len, partition, &P, &NP)) return PA_ERR_INVALID;
+  if (B == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || MB == 0)
+    return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  const size_t need = workspace_for(B, H, D, NP);
+  if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace))) return PA_ERR_INVALID;
+  pa::DecodeParams prm{};
+  prm.out = out;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.block_tables = block_tables;
+  prm.seq_lens = seq_lens;
+  prm.q_scale = scale * k_scale * 1.4426950408889634f;  // K's scale folded into q, log2(e)
+  prm.v_scale = v_scale;
+  prm.MB = MB;
+  prm.B = B;
+  prm.H = H;
+  prm.Hkv = H;
+  prm.NB = NB;
+  if (NP > 1) {
+    const size_t n = static_cast<size_t>(B) * H * NP;
+    prm.ws_m = static_cast<float*>(workspace);
+    prm.ws_l = prm.ws_m + n;
+    prm.ws_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                          align256(n * 2 * sizeof(float)));
+    prm.P = P;
+    prm.NP = NP;
+    prm.L_cap = static_cast<int>(std::min<int64_t>(L_max, static_cast<int64_t>(NP) * P));
+  } else {
+    prm.P = static_cast<int>(L_max > 0 ? L_max : S);
+    prm.NP = 1;
+    prm.L_cap = static_cast<int>(L_max);
+  }
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (q_dt == PA_F16) {
+    switch (out_dt) {
+      case PA_F32: return dispatch_fp8_shape<__half, float>(prm, D, S, st);
+      case PA_F16: return dispatch_fp8_shape<__half, __half>(prm, D, S, st);
+      case PA_BF16: return dispatch_fp8_shape<__half, __nv_bfloat16>(prm, D, S, st);
+    }
+  } else {
+    switch (out_dt) {
+      case PA_F32: return dispatch_fp8_shape<__nv_bfloat16, float>(prm, D, S, st);
+      case PA_F16: return dispatch_fp8_shape<__nv_bfloat16, __half>(prm, D, S, st);
+      case PA_BF16: return dispatch_fp8_shape<__nv_bfloat16, __nv_bfloat16>(prm, D, S, st);
+    }
+  }
+  return PA_ERR_INVALID;
 }
 
 pa_status pa_get_device_error(void* stream, uint32_t* flags) {

@@ -44,6 +44,47 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The same scatter into an FP8 E4M3 cache (a storage extension, not on the
+// pages): each element is stored as the E4M3 code of fp32(x / scale) (one
+// correctly rounded division, then round to nearest even, saturated at 448),
+// K and V with their own per-tensor scale. One thread per 8 elements: a
+// 16-byte vector of 16-bit input becomes an 8-byte vector of codes.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    kv_append_fp8_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                         const int64_t* __restrict__ slots, uint2* __restrict__ k_cache,
+                         uint2* __restrict__ v_cache, float k_scale, float v_scale, int64_t total,
+                         int H, int vpr, int S, int64_t n_slots) {
+  const int64_t per_token = static_cast<int64_t>(H) * vpr;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = idx / per_token;
+    const int64_t rem = idx - t * per_token;
+    const int64_t h = rem / vpr;
+    const int64_t c = rem - h * vpr;
+    const int64_t slot = __ldg(slots + t);
+    if (slot < 0) continue;  // padding
+    if (slot >= n_slots) {
+      raise_error(PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t blk = slot / S;
+    const int64_t off = slot - blk * S;
+    const int64_t dst = ((blk * H + h) * S + off) * vpr + c;
+    float kf[8], vf[8];
+    convert_frag<T>(__ldcs(k + idx), kf);
+    convert_frag<T>(__ldcs(v + idx), vf);
+    uint32_t kw[4], vw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      kw[e] = float2_to_e4m3x2(__fdiv_rn(kf[2 * e], k_scale), __fdiv_rn(kf[2 * e + 1], k_scale));
+      vw[e] = float2_to_e4m3x2(__fdiv_rn(vf[2 * e], v_scale), __fdiv_rn(vf[2 * e + 1], v_scale));
+    }
+    k_cache[dst] = make_uint2(kw[0] | (kw[1] << 16), kw[2] | (kw[3] << 16));
+    v_cache[dst] = make_uint2(vw[0] | (vw[1] << 16), vw[2] | (vw[3] << 16));
+  }
+}
+
 // Copy-on-write, device half ("vLLM KV Cache and PagedAttention Explained",
 // Step 9): copies whole physical blocks, every head, of K and V from src to
 // dst for each (src, dst) pair. One thread per 16-byte vector; the pairs come

@@ -58,25 +58,27 @@ struct DecodeParams {
   int P;     // tokens per partition (multiple of S)
   int NP;    // partitions in the grid
   int L_cap; // lengths are clamped to this (MB*S, or NP*P when split)
+  float v_scale;  // V = v_scale * stored value (1 for 16-bit caches; E4M3 caches)
 };
 
-// Shapes of the partition pass for head_dim D and block_size S.
-//   EPL = 8  elements per lane per row fragment (one 16-byte shared load)
-//   LPR      lanes per row (D / 8: 8, 16 or 32); RPW = 32 / LPR rows per warp-wide load
-//   CR       rows per pipeline unit: CR x D of K and of V (about 4 KB each) is one
+// Shapes of the partition pass for head_dim D, block_size S and EB-byte cache
+// elements (2: fp16 / bf16, 1: E4M3).
+//   EPL      elements per lane per row fragment (one 16-byte shared load): 16 / EB
+//   LPR      lanes per row (D / EPL); RPW = 32 / LPR rows per warp-wide load
+//   CR       rows per pipeline unit: CR x D of K and of V (up to 4 KB each) is one
 //            stage, so the stage size no longer grows with S; a block of S rows
 //            is S / CR units
 //   NS, NW   stages per warp and warps per CTA: about 64 KB of stages per CTA
-template <int D, int S>
+template <int D, int S, int EB = 2>
 struct DecodeTiling {
-  static constexpr int EPL = 8;
+  static constexpr int EPL = 16 / EB;
   static constexpr int LPR = D / EPL;
   static constexpr int RPW = 32 / LPR;
-  static constexpr int CR_RAW = 2048 / D;
+  static constexpr int CR_RAW = 4096 / (D * EB);
   static constexpr int CR = CR_RAW < S ? CR_RAW : S;
   static constexpr int NV = CR / RPW;  // rows per lane per unit
-  static constexpr int SLAB = S * D * 2;     // one (block, head) slab of K or of V
-  static constexpr int UNIT = CR * D * 2;    // one unit of K or of V
+  static constexpr int SLAB = S * D * EB;    // one (block, head) slab of K or of V
+  static constexpr int UNIT = CR * D * EB;   // one unit of K or of V
   static constexpr int STAGE = 2 * UNIT;
   static constexpr int NS = STAGE <= 4096 ? 4 : 2;
   static constexpr int NW_RAW = 65536 / (NS * STAGE);
@@ -129,10 +131,15 @@ struct RawFrag {
 // run holds that token copies the row into its staged unit once the bulk copy
 // has landed (so the scores see it) and stores it to the cache, as
 // pa_kv_append would have before the decode.
-template <typename T, typename TO, int D, int S, bool APPEND>
-__global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
+//
+// TC is the cache element type: T itself, or E4M3 codes with per-tensor
+// scales (K's folded into q_scale, V's applied to the accumulated output).
+template <typename T, typename TO, int D, int S, bool APPEND, typename TC = T>
+__global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
     paged_decode_partition_kernel(const DecodeParams p) {
-  using Tl = DecodeTiling<D, S>;
+  constexpr int EB = sizeof(TC);
+  static_assert(!APPEND || EB == 2, "the fused append copies 16-bit rows");
+  using Tl = DecodeTiling<D, S, EB>;
   constexpr int NW = Tl::NW, NS = Tl::NS, SLAB = Tl::SLAB, UNIT = Tl::UNIT, STAGE = Tl::STAGE;
   constexpr int EPL = Tl::EPL, LPR = Tl::LPR, RPW = Tl::RPW, CR = Tl::CR, NV = Tl::NV;
   constexpr int DUP = LPR / NV;  // lanes of a group holding the same row's score
@@ -143,7 +150,7 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
   const int g = lane / LPR;   // row group
-  const int pl = lane % LPR;  // position in the row: elements pl * 8 .. pl * 8 + 7
+  const int pl = lane % LPR;  // position in the row: elements pl * EPL .. pl * EPL + EPL - 1
 
   int L = __ldg(p.seq_lens + i);
   const bool len_ok = L >= 0 && L <= p.L_cap;
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
       if (ok) {
         mbar_arrive_expect_tx(&bar[s], 2 * UNIT);
         const int64_t off = static_cast<int64_t>(id) * block_stride +
-                            static_cast<int64_t>(t0 % S) * D * 2;
+                            static_cast<int64_t>(t0 % S) * D * EB;
         bulk_g2s(stage0 + s * STAGE, kbase + off, UNIT, &bar[s], policy);
         bulk_g2s(stage0 + s * STAGE + UNIT, vbase + off, UNIT, &bar[s], policy);
       } else {
@@ -292,7 +299,7 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
         float kf[EPL];
-        load_row<T, EPL>(ks + ((v * RPW + g) * D + pl * EPL) * 2, kf);
+        load_cache_row<TC, EPL>(ks + ((v * RPW + g) * D + pl * EPL) * EB, kf);
         float a = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) a = fmaf(qf[e], kf[e], a);
@@ -315,7 +322,7 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
         for (int v = 0; v < NV; ++v) {
           const float pv = __shfl_sync(kFullMask, pr, g * LPR + v * DUP);
           float vf[EPL];
-          load_row<T, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * 2, vf);
+          load_cache_row<TC, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * EB, vf);
 #pragma unroll
           for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pv, vf[e], acc[e]);
         }
@@ -328,7 +335,7 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
             const float pv = __shfl_sync(kFullMask, pr, g * LPR + v * DUP);
             const bool row_ok = v * RPW + g < nvalid;
             float vf[EPL];
-            load_row<T, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * 2, vf);
+            load_cache_row<TC, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * EB, vf);
 #pragma unroll
             for (int e = 0; e < EPL; ++e) acc[e] = row_ok ? fmaf(pv, vf[e], acc[e]) : acc[e];
           }
@@ -378,6 +385,7 @@ __global__ void __launch_bounds__(DecodeTiling<D, S>::NW * 32)
     float a = 0.f;
 #pragma unroll
     for (int u = 0; u < NW; ++u) a = fmaf(wgt[u], acc_s[u * D + d], a);
+    a *= p.v_scale;
     if (direct) {
       const float o = Ltot > 0.f ? a / Ltot : 0.f;
       static_cast<TO*>(p.out)[ih * D + d] = to_out<TO>(o);

@@ -5,6 +5,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "pagedattn.h"
@@ -130,11 +131,20 @@ struct Elem<__nv_bfloat16> {
   }
 };
 
-// DL consecutive 16-bit elements (DL in {2, 4, 8}) from shared or global memory
-// into fp32 registers, with one 4/8/16-byte load.
+// DL consecutive 16-bit elements (DL in {2, 4, 8, 16}) from shared or global
+// memory into fp32 registers, with one 4/8/16-byte load (two for 16).
 template <typename T, int DL>
 __device__ __forceinline__ void load_row(const void* p, float (&f)[DL]) {
-  if constexpr (DL == 2) {
+  if constexpr (DL == 16) {
+    float a[8], b[8];
+    load_row<T, 8>(p, a);
+    load_row<T, 8>(static_cast<const uint8_t*>(p) + 16, b);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      f[k] = a[k];
+      f[8 + k] = b[k];
+    }
+  } else if constexpr (DL == 2) {
     const uint32_t x = *reinterpret_cast<const uint32_t*>(p);
     const float2 a = Elem<T>::pair(x);
     f[0] = a.x;
@@ -156,6 +166,46 @@ __device__ __forceinline__ void load_row(const void* p, float (&f)[DL]) {
       f[2 * k] = a.x;
       f[2 * k + 1] = a.y;
     }
+  }
+}
+
+// FP8 E4M3 (cache storage): two codes (low byte first) -> fp32, exactly, through
+// the hardware conversion to a pair of binary16 values.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t x) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(x));
+  __half2 h;
+  *reinterpret_cast<uint32_t*>(&h) = h2;
+  return __half22float2(h);
+}
+
+// Two fp32 -> two E4M3 codes (lo in the low byte), round to nearest even,
+// saturated at +-448.
+__device__ __forceinline__ uint16_t float2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// One row fragment of the cache (16 bytes in shared memory) -> fp32 registers:
+// 8 elements of a 16-bit cache, or 16 of an E4M3 cache.
+template <typename TC, int EPL>
+__device__ __forceinline__ void load_cache_row(const void* p, float (&f)[EPL]) {
+  if constexpr (sizeof(TC) == 1) {
+    static_assert(EPL == 16, "an E4M3 fragment is 16 codes");
+    const uint4 x = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[k] & 0xffffu));
+      const float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[k] >> 16));
+      f[4 * k] = a.x;
+      f[4 * k + 1] = a.y;
+      f[4 * k + 2] = b.x;
+      f[4 * k + 3] = b.y;
+    }
+  } else {
+    load_row<TC, EPL>(p, f);
   }
 }
 

@@ -1,0 +1,138 @@
+"""FP8 E4M3 KV cache (a storage extension, not on the pages): pa_kv_append_fp8
+bit for bit against the oracle's quantizer, and pa_decode_fp8 against the
+oracle's decode over the same codes, at the decode tolerance, with NaN codes
+poisoning every byte a request does not own; small cases element by element,
+the LLaMA-2-13B decode shape on sampled pairs."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import MAX_ABS, REL_L2, assert_parity, sample_pairs
+from oracle import fp8 as ofp8
+from paged_kv_cache_driven_b200 import binding, workloads
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+NAN_CODE = 0x7F
+
+
+def fp8_case(lens, H, D, S, in_dt, seed, k_scale=0.05, v_scale=0.08):
+    """A decode case whose caches are filled through pa_kv_append_fp8 from the
+    16-bit case's K/V rows; unused bytes are NaN codes. Returns (case, kc8, vc8)."""
+    case = workloads.decode_case(lens, H=H, D=D, S=S, dtype=in_dt, seed=seed, device=DEV,
+                                 poison=False)
+    NB = case.k_cache.shape[0]
+    kc8 = torch.full((NB, H, S, D), NAN_CODE, dtype=torch.uint8, device=DEV)
+    vc8 = torch.full_like(kc8, NAN_CODE)
+    for i, L in enumerate(case.seq_lens_host):
+        if L == 0:
+            continue
+        blocks = torch.tensor(case.tables_host[i], device=DEV)
+        k = case.k_cache[blocks].permute(0, 2, 1, 3).reshape(-1, H, D)[:L].contiguous()
+        v = case.v_cache[blocks].permute(0, 2, 1, 3).reshape(-1, H, D)[:L].contiguous()
+        slots = (blocks.repeat_interleave(S) * S + torch.arange(S, device=DEV).repeat(len(blocks)))[:L]
+        binding.pa_kv_append_fp8(k, v, slots.to(torch.int64), kc8, vc8, k_scale, v_scale)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    return case, kc8, vc8
+
+
+@pytest.mark.parametrize("in_dt", [torch.bfloat16, torch.float16])
+def test_append_fp8_bit_exact(in_dt):
+    g = torch.Generator().manual_seed(1)
+    T, H, D, S, NB = 300, 4, 128, 16, 40
+    k = (torch.randn(T, H, D, generator=g) * 3).to(in_dt)
+    v = (torch.randn(T, H, D, generator=g) * 3).to(in_dt)
+    k[0, 0, :4] = torch.tensor([500.0, -1e4, 0.0, -0.0]).to(in_dt)  # saturation and zeros
+    slots = torch.randperm(NB * S, generator=g)[:T].to(torch.int64)
+    slots[5] = -1  # padding: skipped
+    kc8 = torch.full((NB, H, S, D), NAN_CODE, dtype=torch.uint8, device=DEV)
+    vc8 = torch.full_like(kc8, NAN_CODE)
+    binding.pa_kv_append_fp8(k.to(DEV), v.to(DEV), slots.to(DEV), kc8, vc8, 0.05, 0.08)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    want_k = np.full((NB, H, S, D), NAN_CODE, np.uint8)
+    want_v = want_k.copy()
+    kq = ofp8.quantize(k.float().numpy(), 0.05)
+    vq = ofp8.quantize(v.float().numpy(), 0.08)
+    for t, s in enumerate(slots.tolist()):
+        if s >= 0:
+            want_k[s // S, :, s % S, :] = kq[t]
+            want_v[s // S, :, s % S, :] = vq[t]
+    assert np.array_equal(kc8.cpu().numpy(), want_k)
+    assert np.array_equal(vc8.cpu().numpy(), want_v)
+    # a slot past the pool is flagged and skipped
+    bad = torch.tensor([NB * S + 3], dtype=torch.int64, device=DEV)
+    binding.pa_kv_append_fp8(k[:1].to(DEV), v[:1].to(DEV), bad, kc8, vc8, 0.05, 0.08)
+    assert binding.pa_get_device_error() & binding.PA_DEVERR_SLOT
+
+
+def run_fp8(case, kc8, vc8, out_dt=torch.float32, partition=0, k_scale=0.05, v_scale=0.08):
+    B, H, D = case.q.shape
+    S = kc8.shape[2]
+    maxlen = max(case.seq_lens_host + [0])
+    out = torch.empty((B, H, D), dtype=out_dt, device=DEV)
+    wsb = binding.pa_decode_workspace_bytes(B, H, D, S, maxlen, partition)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=DEV)
+    binding.pa_decode_fp8(out, case.q, kc8, vc8, k_scale, v_scale, case.block_tables,
+                          case.seq_lens, case.scale, maxlen, partition=partition, workspace=ws)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    return out
+
+
+@pytest.mark.parametrize("D,S", [(64, 8), (128, 16), (128, 32), (256, 16)])
+@pytest.mark.parametrize("partition", [0, -1])
+def test_decode_fp8_small(D, S, partition):
+    lens = [0, 1, S - 1, S, 3 * S + 5, 700]
+    case, kc8, vc8 = fp8_case(lens, H=3, D=D, S=S, in_dt=torch.bfloat16, seed=D + S)
+    out = run_fp8(case, kc8, vc8, partition=partition)
+    want = ofp8.paged_decode_fp8(case.q.cpu(), kc8.cpu(), vc8.cpu(), 0.05, 0.08,
+                                 case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
+    assert_parity(out.cpu().numpy(), want, f"fp8 D={D} S={S} p={partition}")
+    assert np.all(out[0].cpu().numpy() == 0)  # L = 0
+
+
+@pytest.mark.parametrize("q_dt,out_dt", [(torch.float16, torch.float16),
+                                         (torch.bfloat16, torch.bfloat16)])
+def test_decode_fp8_dtypes(q_dt, out_dt):
+    case, kc8, vc8 = fp8_case([50, 333, 1000], H=4, D=128, S=16, in_dt=q_dt, seed=3)
+    out = run_fp8(case, kc8, vc8, out_dt=out_dt)
+    want = ofp8.paged_decode_fp8(case.q.cpu(), kc8.cpu(), vc8.cpu(), 0.05, 0.08,
+                                 case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
+    got = out.float().cpu().numpy()
+    ulp = 2.0 ** -8 if out_dt == torch.bfloat16 else 2.0 ** -11
+    assert np.abs(got - want).max() <= MAX_ABS + ulp * np.abs(want).max()
+
+
+def test_decode_fp8_llama13b_shape_sampled():
+    """40 heads, head_dim 128, block 16, batch 64, L ~ U[1, 2048]: the bench's
+    decode shape with an E4M3 cache, in its launch configuration."""
+    lens = workloads.uniform_lengths(64, 1, 2048, 0)
+    case, kc8, vc8 = fp8_case(lens, H=40, D=128, S=16, in_dt=torch.bfloat16, seed=0)
+    out = run_fp8(case, kc8, vc8)
+    pairs = sample_pairs(case, 24)
+    # the oracle on the sampled (request, head) pairs: a one-head sub-problem each
+    qs, ks, vs, tabs, Ls = [], [], [], [], []
+    off = 0
+    for i, h in pairs:
+        L = case.seq_lens_host[i]
+        blocks = torch.tensor(case.tables_host[i], device=DEV)
+        ks.append(kc8[blocks, h].unsqueeze(1).cpu())
+        vs.append(vc8[blocks, h].unsqueeze(1).cpu())
+        qs.append(case.q[i, h].view(1, 1, -1).cpu())
+        tabs.append(list(range(off, off + len(blocks))))
+        Ls.append(L)
+        off += len(blocks)
+    MB = max(len(t) for t in tabs)
+    bt = torch.full((len(pairs), MB), -1, dtype=torch.int32)
+    for r, t in enumerate(tabs):
+        bt[r, :len(t)] = torch.tensor(t, dtype=torch.int32)
+    want = ofp8.paged_decode_fp8(torch.cat(qs), torch.cat(ks), torch.cat(vs), 0.05, 0.08, bt,
+                                 torch.tensor(Ls, dtype=torch.int32), case.scale)[:, 0]
+    got = torch.stack([out[i, h] for i, h in pairs]).cpu().numpy()
+    assert_parity(got, want, "fp8 13B shape")
+    assert bool(torch.isfinite(out).all())
