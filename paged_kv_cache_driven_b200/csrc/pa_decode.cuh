@@ -80,7 +80,9 @@ struct DecodeTiling {
   static constexpr int SLAB = S * D * EB;    // one (block, head) slab of K or of V
   static constexpr int UNIT = CR * D * EB;   // one unit of K or of V
   static constexpr int STAGE = 2 * UNIT;
-  static constexpr int NS = STAGE <= 4096 ? 4 : 2;
+  // E4M3 units carry twice the elements per byte, so more warps (two stages
+  // each) keep the same bytes in flight with twice the threads to convert them
+  static constexpr int NS = (STAGE <= 4096 && EB == 2) ? 4 : 2;
   static constexpr int NW_RAW = 65536 / (NS * STAGE);
   static constexpr int NW = NW_RAW < 1 ? 1 : (NW_RAW > 8 ? 8 : NW_RAW);
   static constexpr int SMEM_PIPE = NW * NS * STAGE;
@@ -300,10 +302,18 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
       for (int v = 0; v < NV; ++v) {
         float kf[EPL];
         load_cache_row<TC, EPL>(ks + ((v * RPW + g) * D + pl * EPL) * EB, kf);
-        float a = 0.f;
+        if constexpr (EB == 1) {  // twice the elements per byte: packed pairs
+          float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) a = fmaf(qf[e], kf[e], a);
-        dot[v] = a;
+          for (int e = 0; e < EPL; e += 2)
+            a2 = ffma2(make_float2(qf[e], qf[e + 1]), make_float2(kf[e], kf[e + 1]), a2);
+          dot[v] = a2.x + a2.y;
+        } else {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) a = fmaf(qf[e], kf[e], a);
+          dot[v] = a;
+        }
       }
       const float score = transpose_reduce<NV, LPR>(dot, lane);
       const bool valid = my_row < nvalid;
@@ -323,8 +333,18 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
           const float pv = __shfl_sync(kFullMask, pr, g * LPR + v * DUP);
           float vf[EPL];
           load_cache_row<TC, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * EB, vf);
+          if constexpr (EB == 1) {
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pv, vf[e], acc[e]);
+            for (int e = 0; e < EPL; e += 2) {
+              const float2 r = ffma2(make_float2(pv, pv), make_float2(vf[e], vf[e + 1]),
+                                     make_float2(acc[e], acc[e + 1]));
+              acc[e] = r.x;
+              acc[e + 1] = r.y;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pv, vf[e], acc[e]);
+          }
         }
       } else {
         // the request's last unit: rows past nvalid may hold anything (NaN);

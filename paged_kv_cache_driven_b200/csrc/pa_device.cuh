@@ -103,6 +103,26 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// Packed pairs of fp32 (one 64-bit register pair, two lanes of work per
+// instruction).
+__device__ __forceinline__ uint64_t as_u64(float2 a) {
+  return static_cast<uint64_t>(__float_as_uint(a.x)) |
+         (static_cast<uint64_t>(__float_as_uint(a.y)) << 32);
+}
+__device__ __forceinline__ float2 as_f2(uint64_t u) {
+  return make_float2(__uint_as_float(static_cast<uint32_t>(u)),
+                     __uint_as_float(static_cast<uint32_t>(u >> 32)));
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(as_u64(a)), "l"(as_u64(b)), "l"(as_u64(c)));
+  return as_f2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(as_u64(a)), "l"(as_u64(b)));
+  return as_f2(d);
+}
 // ---- 16-bit element conversions -------------------------------------------------
 
 template <typename T>

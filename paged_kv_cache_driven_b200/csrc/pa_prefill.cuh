@@ -117,26 +117,7 @@ __device__ __forceinline__ uint32_t pack_pair<__half>(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Packed pairs of fp32 (one 64-bit register pair, two lanes of work per
-// instruction) and the three-input max.
-__device__ __forceinline__ uint64_t as_u64(float2 a) {
-  return static_cast<uint64_t>(__float_as_uint(a.x)) |
-         (static_cast<uint64_t>(__float_as_uint(a.y)) << 32);
-}
-__device__ __forceinline__ float2 as_f2(uint64_t u) {
-  return make_float2(__uint_as_float(static_cast<uint32_t>(u)),
-                     __uint_as_float(static_cast<uint32_t>(u >> 32)));
-}
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(as_u64(a)), "l"(as_u64(b)), "l"(as_u64(c)));
-  return as_f2(d);
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(as_u64(a)), "l"(as_u64(b)));
-  return as_f2(d);
-}
+// The three-input max.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
