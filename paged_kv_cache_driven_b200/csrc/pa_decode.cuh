@@ -325,8 +325,10 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
       const float alpha = exp2f(m - m_new);
       const float pr = valid ? exp2f(sc - m_new) : 0.f;
       lsum = lsum * alpha + ((pl % DUP) == 0 ? pr : 0.f);
+      if (m_new != m) {  // warp-uniform; otherwise alpha is exactly 1
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
+        for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
+      }
       if (nvalid == CR) {
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
