@@ -61,7 +61,7 @@ struct PrefillTiling {
   static constexpr int BN = 128;              // keys per tile
   // K runs further ahead than V: S needs K(j + 1) right after P(j) is ready,
   // V(j + 1) only after the next softmax
-  static constexpr int KST = D == 128 ? 3 : 4;  // K stages
+  static constexpr int KST = D == 128 ? 2 : 4;  // K stages
   static constexpr int VST = D == 128 ? 2 : 4;  // V stages
   static constexpr int COLB = D / 64;         // 64-element (128-byte) column blocks
   static constexpr int CB_BYTES = 128 * 128;  // one column block of 128 rows
@@ -69,11 +69,13 @@ struct PrefillTiling {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int OFF_K = NQT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int OFF_XCH = OFF_V + VST * KV_BYTES;  // row-max exchange between halves
+  static constexpr int XCH_BYTES = NQT * 2 * 2 * BM * 4;  // [tile][phase parity][half][row]
+  static constexpr int OFF_BAR = OFF_XCH + XCH_BYTES;
   // + alignment slack and barriers; at least 120 KB, so that one CTA holds an
   // SM (it allocates all 512 tensor-memory columns)
   static constexpr int SMEM = 1024 + OFF_BAR + 256 > 120 * 1024 ? 1024 + OFF_BAR + 256 : 120 * 1024;
-  static constexpr int THREADS = NQT * 128 + 64;
+  static constexpr int THREADS = NQT * 256 + 64;  // two softmax warpgroups per tile
   static constexpr uint32_t TMEM_COLS = 512;  // per tile: S/P 128 columns, O 128
   static_assert(D == 64 || D == 128, "head size 64 or 128");
   static_assert(SMEM <= 232448, "shared memory per CTA");
@@ -170,7 +172,7 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity,
 }
 
 template <typename T, typename TO, int D, int S>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
     paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmq,
                          const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv) {
@@ -220,7 +222,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* s_full = v_empty + Tl::VST;       // [NQT]
   uint64_t* p_full = s_full + Tl::NQT;        // [NQT]
   uint64_t* o_done = p_full + Tl::NQT;        // [NQT]
-  uint64_t* mma_done = o_done + Tl::NQT;
+  uint64_t* xch_bar = o_done + Tl::NQT;       // [NQT]: the tile's two halves have posted
+  uint64_t* mma_done = xch_bar + Tl::NQT;
+  float* xch = reinterpret_cast<float*>(sm + Tl::OFF_XCH);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -237,14 +241,16 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int t = 0; t < Tl::NQT; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&p_full[t], 256);
       mbar_init(&o_done[t], 1);
+      mbar_init(&xch_bar[t], 256);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  constexpr int kProducer = 4 * Tl::NQT * 2, kIssuer = kProducer + 1;  // warps 16, 17
+  if (warp == kIssuer) {
     __syncwarp();
     tc::tmem_alloc(tmem_slot, Tl::TMEM_COLS);
     tc::tmem_relinquish();
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__(320, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == kProducer) {
     // ---------------- producer: lane b loads cache block b of each key tile ----------------
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, nq * Tl::Q_BYTES);
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     (void)ok;
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == kIssuer) {
     // ---------------- MMA issuer (lane 0), V tail zeroing (whole warp) ----------------
     constexpr int fmt = LO ? 1 : 0;
     constexpr uint32_t idesc_s = tc::instr_desc_f16(fmt, 0, 0, Tl::BM, Tl::BN);
@@ -404,89 +410,93 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- softmax (warps 4t .. 4t + 3: tile t, thread r = row r) ----------------
-    const int t = warp >> 2;
+    // ---------------- softmax: warps 8t .. 8t + 7 serve query tile t; warpgroup
+    // half hw of them takes keys 64 hw .. 64 hw + 63 of each key tile and output
+    // columns hw D / 2 .. of each row; thread r of a warpgroup owns row r ----------------
+    constexpr int HK = Tl::BN / 2;  // keys per half
+    constexpr int HD = D / 2;       // output columns per half
+    const int t = warp >> 3;
+    const int hw = (warp >> 2) & 1;
     const int r = threadIdx.x & 127;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + t * 256 + lane_base, tO = tS + 128;
+    const uint32_t tT = tmem + t * 256 + lane_base;
+    const uint32_t tS = tT + hw * HK, tO = tT + 128 + hw * HD;
     const int qrow = row0 + t * Tl::BM + r;
     const int lim = min(ctx + qrow, L - 1);  // last key this row sees
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // l: this half's share of the running sum
     bool ok = nk[t] > 0;
+    auto slot = [&](int j, int half) { return xch + ((t * 2 + (j & 1)) * 2 + half) * Tl::BM; };
     for (int j = 0; ok && j < nk[t]; ++j) {
       ok = wait_warp(&s_full[t], j & 1, abort_flag);
       if (!ok) break;
       tc::fence_after_sync();
-      const int kb = j * Tl::BN;
+      const int kb = j * Tl::BN + hw * HK;
       // keys past this row's last one count as -inf (scale > 0, so the order of
       // raw scores is the order of scaled ones)
-      const bool diag = kb + Tl::BN - 1 > lim;
-      // the row's 128 scores in two halves: the second half's loads are in
-      // flight while the first half's max is taken
-      float x[Tl::BN];
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      const bool diag = kb + HK - 1 > lim;
+      float x[HK];
       {
-        uint32_t u[Tl::BN];
-        constexpr int HALF = Tl::BN / 2;
+        uint32_t u[HK];
 #pragma unroll
-        for (int c4 = 0; c4 < HALF / 32; ++c4)
+        for (int c4 = 0; c4 < HK / 32; ++c4)
           tc::tmem_ld32(tS + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c4 * 32]));
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int c4 = HALF / 32; c4 < Tl::BN / 32; ++c4)
-          tc::tmem_ld32(tS + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c4 * 32]));
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          if (hf == 1) tc::tmem_wait_ld();
-#pragma unroll
-          for (int c = hf * HALF; c < (hf + 1) * HALF; ++c)
-            x[c] = diag && kb + c > lim ? -INFINITY : __uint_as_float(u[c]);
-#pragma unroll
-          for (int c = hf * HALF; c < (hf + 1) * HALF; c += 2)
-            mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], x[c], x[c + 1]);
-        }
+        for (int c = 0; c < HK; ++c) x[c] = diag && kb + c > lim ? -INFINITY : __uint_as_float(u[c]);
       }
-      const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * p.scale_log2;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < HK; c += 2) mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], x[c], x[c + 1]);
+      const float hmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
+      // the row's max over both halves: post this half's, read the other's
+      // (slots alternate with the key tile, so a half never overwrites a value
+      // the other has not read yet)
+      slot(j, hw)[r] = hmax;
+      mbar_arrive(&xch_bar[t]);
+      ok = wait_warp(&xch_bar[t], j & 1, abort_flag);
+      if (!ok) break;
+      const float tmax = fmaxf(hmax, slot(j, hw ^ 1)[r]) * p.scale_log2;
       // The reference max only moves when the tile max exceeds it by more than
-      // 2^8 in weight; the weights stay <= 256, exact in the final ratio.
+      // 2^8 in weight; the weights stay <= 256, exact in the final ratio. Both
+      // halves see the same tile max, so they take the same decision.
       const float m_new = fmaxf(m, tmax);
       const bool grow = m_new > m + 8.f;
       const float m_use = grow ? m_new : m;
       const float alpha = grow ? fast_exp2(m - m_use) : 1.f;
       m = m_use;
-      // P over the scores, 8 keys at a time: keys 2k, 2k+1 of chunk q (32 keys)
-      // as one 16-bit pair in column 32q + k, and for bf16 the rounding residue
-      // p - bf16(p), itself rounded, in column 32q + 16 + k
+      // P over this half's scores, 8 keys at a time: keys 2k, 2k+1 of a 32-key
+      // chunk q of the tile as one 16-bit pair in column 32q + k, and for bf16
+      // the rounding residue p - bf16(p), itself rounded, in column 32q + 16 + k
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
       const float2 nm2 = make_float2(-m_use, -m_use);
       float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int g = 0; g < Tl::BN / 8; ++g) {  // 8 keys: 4 columns of P (and 4 of residues)
+      for (int g = 0; g < HK / 8; ++g) {
         float* v = &x[8 * g];
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 t = ffma2(make_float2(v[2 * e], v[2 * e + 1]), sc2, nm2);
-          const float2 pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          const float2 tt = ffma2(make_float2(v[2 * e], v[2 * e + 1]), sc2, nm2);
+          const float2 pe = make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
           acc[e & 1] = fadd2(acc[e & 1], pe);
           hi[e] = pack_pair<T>(pe.x, pe.y);
           if constexpr (LO) {
             // bf16 pair -> the two fp32 values it holds: exact bit moves
-            const float2 h = make_float2(__uint_as_float(hi[e] << 16),
-                                         __uint_as_float(hi[e] & 0xffff0000u));
-            const float2 r = make_float2(pe.x - h.x, pe.y - h.y);
-            lo[e] = pack_pair<T>(r.x, r.y);
+            const float2 hh = make_float2(__uint_as_float(hi[e] << 16),
+                                          __uint_as_float(hi[e] & 0xffff0000u));
+            lo[e] = pack_pair<T>(pe.x - hh.x, pe.y - hh.y);
           }
         }
-        const uint32_t col = 32 * (g >> 2) + 4 * (g & 3);
+        const uint32_t col = 32 * (g >> 2) + 4 * (g & 3);  // within this half's 64 columns
         tc::tmem_st4(tS + col, hi);
         if constexpr (LO) tc::tmem_st4(tS + col + 16, lo);
       }
       // The product of the previous key tile has completed (the commit that
-      // released these scores covers it): rescale the rows whose max moved.
+      // released these scores covers it): rescale this half's output columns
+      // of the rows whose max moved.
       if (j > 0 && __any_sync(kFullMask, grow)) {
 #pragma unroll 1
-        for (int c4 = 0; c4 < D / 32; ++c4) {
+        for (int c4 = 0; c4 < HD / 32; ++c4) {
           uint32_t u[32];
           tc::tmem_ld32(tO + c4 * 32, u);
           tc::tmem_wait_ld();
@@ -500,14 +510,19 @@ __global__ void __launch_bounds__(320, 1)
       tc::fence_before_sync();
       mbar_arrive(&p_full[t]);
     }
-    // epilogue: O / l -> out
+    // epilogue: the row's sum over both halves, then O / l -> out (this half's columns)
+    if (ok) {
+      slot(nk[t], hw)[r] = l;
+      mbar_arrive(&xch_bar[t]);
+      ok = wait_warp(&xch_bar[t], nk[t] & 1, abort_flag);
+    }
     if (ok) ok = wait_warp(&o_done[t], 0, abort_flag);
     if (ok) {
       tc::fence_after_sync();
-      const float inv = 1.f / l;
-      TO* dst = reinterpret_cast<TO*>(p.out) + (static_cast<int64_t>(q0 + qrow) * p.H + h) * D;
+      const float inv = 1.f / (l + slot(nk[t], hw ^ 1)[r]);
+      TO* dst = reinterpret_cast<TO*>(p.out) + (static_cast<int64_t>(q0 + qrow) * p.H + h) * D + hw * HD;
 #pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
+      for (int c4 = 0; c4 < HD / 32; ++c4) {
         uint32_t u[32];
         tc::tmem_ld32(tO + c4 * 32, u);
         tc::tmem_wait_ld();
@@ -520,7 +535,7 @@ __global__ void __launch_bounds__(320, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kIssuer) {
     __syncwarp();
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, Tl::TMEM_COLS);
