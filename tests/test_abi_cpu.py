@@ -116,3 +116,78 @@ def test_stepper_rejects_bad_arguments_on_host(lib):
         assert lib.pa_stepper_create(*args) == binding.PA_ERR_INVALID, idx
     assert lib.pa_stepper_step(NULL, P, P, NULL, NULL) == binding.PA_ERR_INVALID
     assert lib.pa_stepper_output(NULL, 0, ctypes.byref(h)) == binding.PA_ERR_INVALID
+
+
+def prefill_args(**kw):
+    a = dict(out=P, out_dt=binding.PA_F32, q=P, k=P, v=P, bt=P, MB=8, sl=P, qs=P, scale=0.1, B=2,
+             H=4, Hkv=4, D=128, S=16, NB=16, dt=binding.PA_BF16, T=100, max_q_len=64, stream=NULL)
+    a.update(kw)
+    return [a[k] for k in ("out", "out_dt", "q", "k", "v", "bt", "MB", "sl", "qs", "scale", "B",
+                           "H", "Hkv", "D", "S", "NB", "dt", "T", "max_q_len", "stream")]
+
+
+@pytest.mark.parametrize("bad", [
+    dict(D=96), dict(D=256), dict(S=4), dict(S=256), dict(dt=binding.PA_F32), dict(out_dt=9),
+    dict(scale=0.0), dict(scale=-1.0), dict(scale=float("nan")), dict(Hkv=3), dict(Hkv=0),
+    dict(q=NULL), dict(qs=NULL), dict(bt=NULL), dict(out=ctypes.c_void_p(16 * 1024 + 4)),
+    dict(NB=0), dict(NB=1 << 28), dict(T=-1), dict(max_q_len=-1), dict(B=-1),
+])
+def test_prefill_rejects_bad_arguments_on_host(lib, bad):
+    assert lib.pa_prefill(*prefill_args(**bad)) == binding.PA_ERR_INVALID
+
+
+def test_prefill_nothing_to_do_is_noop(lib):
+    for kw in (dict(B=0), dict(T=0), dict(max_q_len=0)):
+        assert lib.pa_prefill(*prefill_args(q=NULL, out=NULL, **kw)) == binding.PA_OK
+
+
+def fp8_decode_args(**kw):
+    a = dict(out=P, out_dt=binding.PA_F32, q=P, q_dt=binding.PA_BF16, k=P, v=P, ks=0.05, vs=0.08,
+             bt=P, MB=8, sl=P, scale=0.1, B=2, H=4, D=128, S=16, NB=16, partition=0,
+             max_seq_len=100, ws=NULL, ws_bytes=0, stream=NULL)
+    a.update(kw)
+    return [a[k] for k in ("out", "out_dt", "q", "q_dt", "k", "v", "ks", "vs", "bt", "MB", "sl",
+                           "scale", "B", "H", "D", "S", "NB", "partition", "max_seq_len", "ws",
+                           "ws_bytes", "stream")]
+
+
+@pytest.mark.parametrize("bad", [
+    dict(ks=0.0), dict(vs=-1.0), dict(ks=float("inf")), dict(vs=float("nan")), dict(D=96),
+    dict(q_dt=binding.PA_F32), dict(S=4), dict(k=NULL), dict(q=ctypes.c_void_p(16 * 1024 + 8)),
+    dict(max_seq_len=100, partition=16),  # needs a workspace, none given
+])
+def test_decode_fp8_rejects_bad_arguments_on_host(lib, bad):
+    assert lib.pa_decode_fp8(*fp8_decode_args(**bad)) == binding.PA_ERR_INVALID
+
+
+def test_decode_fp8_zero_batch_is_noop(lib):
+    assert lib.pa_decode_fp8(*fp8_decode_args(B=0, q=NULL, out=NULL)) == binding.PA_OK
+
+
+def fp8_append_args(**kw):
+    a = dict(k=P, v=P, in_dt=binding.PA_BF16, slots=P, kc=P, vc=P, ks=0.05, vs=0.08, T=4, H=2,
+             D=64, S=16, NB=8, stream=NULL)
+    a.update(kw)
+    return [a[k] for k in ("k", "v", "in_dt", "slots", "kc", "vc", "ks", "vs", "T", "H", "D", "S",
+                           "NB", "stream")]
+
+
+@pytest.mark.parametrize("bad", [
+    dict(D=8), dict(D=72), dict(ks=0.0), dict(vs=float("nan")), dict(in_dt=binding.PA_F32),
+    dict(T=-1), dict(slots=NULL), dict(kc=ctypes.c_void_p(16 * 1024 + 8)),
+])
+def test_append_fp8_rejects_bad_arguments_on_host(lib, bad):
+    assert lib.pa_kv_append_fp8(*fp8_append_args(**bad)) == binding.PA_ERR_INVALID
+
+
+def test_append_fp8_zero_tokens_is_noop(lib):
+    assert lib.pa_kv_append_fp8(*fp8_append_args(T=0, k=NULL, v=NULL)) == binding.PA_OK
+
+
+def test_gqa_rejects_heads_not_a_multiple(lib):
+    args = decode_args(H=6)
+    # pa_decode_gqa(out, out_dt, q, k_new, v_new, k_cache, v_cache, bt, MB, sl, scale, B, H, Hkv,
+    #               D, S, NB, dt, partition, max_seq_len, ws, ws_bytes, stream)
+    out, out_dt, q, k, v, bt, MB, sl, scale, B, H, D, S, NB, dt, part, msl, ws, wsb, st = args
+    assert lib.pa_decode_gqa(out, out_dt, q, NULL, NULL, k, v, bt, MB, sl, scale, B, H, 4, D, S,
+                             NB, dt, part, msl, ws, wsb, st) == binding.PA_ERR_INVALID
