@@ -9,21 +9,23 @@
 // K_t / V_t read through the block table (token t in block
 // block_tables[i][t / S], slot t % S), query head h reading KV head h / (H / Hkv).
 //
-// One CTA per (256 query rows = two 128-row tiles, query head, request), 320
+// One CTA per (256 query rows = two 128-row tiles, query head, request), 576
 // threads in four roles:
-//   warps 0-3, 4-7  softmax for query tile 0 / 1: thread r owns row r of its
-//              tile (tensor-memory lane r); reads the tile's scores from tensor
-//              memory (the whole row, read in two overlapped halves), keeps the running max / sum
-//              in fp32, writes the weights P back over the scores as 16-bit
+//   warps 0-7, 8-15  softmax for query tile 0 / 1, two warpgroups per tile:
+//              warpgroup half h takes keys 64 h .. 64 h + 63 of each key tile
+//              and output columns h D / 2 .. of each row; thread r owns row r
+//              of its tile (tensor-memory lane r). It reads its half of the
+//              scores from tensor memory, meets the other half on an mbarrier
+//              to share the row max, keeps the running max / its share of the
+//              sum in fp32, writes the weights P back over the scores as 16-bit
 //              pairs (bf16 as hi + lo halves, so the weights keep ~16 bits), and
-//              rescales the tile's output accumulator when its reference max
-//              moves;
-//   warp 8     producer: TMA loads of the two Q tiles and of 128-key K / V
-//              tiles, one box per (cache block, 64-column block); K runs up to
-//              three tiles ahead, V two (four each for head size 64);
-//              lane b reads the table entry of block b of a tile and issues its
-//              boxes, so a tile's boxes go out in parallel;
-//   warp 9     MMA issuer (lane 0) and tensor-memory owner, also zeroing V rows
+//              rescales its output columns when the reference max moves;
+//   warp 16    producer: TMA loads of the two Q tiles and of 128-key K / V
+//              tiles, one box per (cache block, 64-column block); K and V run
+//              two tiles ahead (four for head size 64); lane b reads the table
+//              entry of block b of a tile and issues its boxes, so a tile's
+//              boxes go out in parallel;
+//   warp 17    MMA issuer (lane 0) and tensor-memory owner, also zeroing V rows
 //              past the end of the request in the last key tile:
 //              S_t = Q_t K^T (both operands K-major in shared memory) and
 //              O_t += P_t V (P_t from tensor memory, V an MN-major operand),
@@ -59,7 +61,7 @@ struct PrefillTiling {
   static constexpr int BM = 128;              // query rows per tile (MMA M)
   static constexpr int NQT = 2;               // query tiles per CTA
   static constexpr int BN = 128;              // keys per tile
-  // K runs further ahead than V: S needs K(j + 1) right after P(j) is ready,
+  // separate K and V rings: S needs K(j + 1) right after P(j) is ready,
   // V(j + 1) only after the next softmax
   static constexpr int KST = D == 128 ? 2 : 4;  // K stages
   static constexpr int VST = D == 128 ? 2 : 4;  // V stages
