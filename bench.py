@@ -20,6 +20,12 @@ cached tokens (pa_decode: partition pass + log-sum-exp reduce).
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 For N > 1 launch under torch.distributed.run; every rank decodes its own batch
 (weak scaling, no data-path collective).
+
+Other workloads (--workload, one GPU, one JSON line each): long_context and
+sweep (decode-only calls of the other decode configurations), llama70b
+(grouped-query decode), llama13b_fp8 (the headline decode shape over an FP8
+E4M3 cache) and prompt_prefill (causal paged prefill attention, TFLOP/s against
+the measured bf16 tensor peak).
 """
 
 import argparse
