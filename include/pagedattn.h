@@ -337,6 +337,15 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst, i
 pa_status pa_build_slot_mapping(const pa_alloc* a, const int64_t* seq_ids, const int* start_pos,
                                 const int* n_tok, int n_seq, int64_t* dst);
 
+/* Host-side check of a slot mapping before pa_kv_append / pa_kv_append_fp8
+ * (which do not detect duplicates; with two tokens on one slot one write
+ * wins): slots [T] host int64, n_slots = NB * S. Returns PA_OK if every
+ * non-negative slot is below n_slots and no slot appears twice (negative
+ * entries are padding); PA_ERR_OUT_OF_RANGE for a slot >= n_slots,
+ * PA_ERR_INVALID for a repeated slot or bad arguments; *first_bad (optional)
+ * receives the index of the offending entry (for a repeat, the later one). */
+pa_status pa_check_slots(const int64_t* slots, int64_t T, int64_t n_slots, int64_t* first_bad);
+
 /* Host block tables [n_seq, MB] int32, padded with -1. PA_ERR_OUT_OF_RANGE if
  * a table has more than MB blocks. */
 pa_status pa_build_block_tables(const pa_alloc* a, const int64_t* seq_ids, int n_seq, int MB,

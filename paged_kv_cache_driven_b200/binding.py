@@ -32,6 +32,7 @@ _SIGNATURES = {
     "pa_decode": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32, _i32,
                    _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_get_device_error": ([_vp, _vp], _i32),
+    "pa_check_slots": ([_vp, _i64, _i64, _vp], _i32),
     "pa_decode_append": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32,
                           _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_decode_gqa": ([_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32,
@@ -225,6 +226,19 @@ def pa_decode_gqa(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_s
                                _ptr(seq_lens), float(scale), B, H, Hkv, D, S, NB, _DT[q.dtype],
                                int(partition), int(max_seq_len), _ptr(workspace), ws_bytes,
                                _stream(stream)), "pa_decode_gqa")
+
+
+def pa_check_slots(slots, n_slots):
+    """Host check of a slot mapping (a CPU int64 tensor): raises PagedAttnError
+    (PA_ERR_OUT_OF_RANGE or PA_ERR_INVALID, with the offending index) if a slot
+    is past n_slots or appears twice; negative slots are padding."""
+    if slots.is_cuda or slots.dtype != torch.int64:
+        raise ValueError("slots must be a CPU int64 tensor")
+    s = slots.contiguous()
+    bad = ctypes.c_int64(-1)
+    st = lib().pa_check_slots(_ptr(s), s.numel(), int(n_slots), ctypes.byref(bad))
+    if st != PA_OK:
+        raise PagedAttnError(st, f"pa_check_slots: entry {bad.value}")
 
 
 def pa_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, q_start, scale, max_q_len,

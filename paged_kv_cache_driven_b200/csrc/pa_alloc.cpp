@@ -221,6 +221,27 @@ pa_status pa_build_slot_mapping(const pa_alloc* a, const int64_t* seq_ids, const
   return PA_OK;
 }
 
+pa_status pa_check_slots(const int64_t* slots, int64_t T, int64_t n_slots, int64_t* first_bad) {
+  if (T < 0 || n_slots < 0 || (T > 0 && !slots)) return PA_ERR_INVALID;
+  std::vector<std::pair<int64_t, int64_t>> seen;  // (slot, index) of the non-padding entries
+  seen.reserve(static_cast<size_t>(T));
+  for (int64_t t = 0; t < T; ++t) {
+    if (slots[t] < 0) continue;  // padding
+    if (slots[t] >= n_slots) {
+      if (first_bad) *first_bad = t;
+      return PA_ERR_OUT_OF_RANGE;
+    }
+    seen.emplace_back(slots[t], t);
+  }
+  std::sort(seen.begin(), seen.end());
+  for (size_t k = 1; k < seen.size(); ++k)
+    if (seen[k].first == seen[k - 1].first) {
+      if (first_bad) *first_bad = seen[k].second;  // the later of two entries naming one slot
+      return PA_ERR_INVALID;
+    }
+  return PA_OK;
+}
+
 pa_status pa_build_block_tables(const pa_alloc* a, const int64_t* seq_ids, int n_seq, int MB,
                                 int32_t* dst) {
   if (!a || n_seq < 0 || MB < 0 || (n_seq > 0 && (!seq_ids || !dst))) return PA_ERR_INVALID;

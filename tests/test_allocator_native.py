@@ -255,3 +255,23 @@ def test_random_walk_with_forks_bit_exact(seed):
             assert counts == m.refs
             assert sorted(set(b for t in m.tables.values() for b in t) | set(m.dump())) == \
                 list(range(NB))
+
+
+def test_check_slots_host():
+    """The host-side slot check: duplicates and slots past the pool are refused
+    (the append kernels do not detect duplicates), padding is allowed, and every
+    slot mapping the allocator builds passes."""
+    ok = torch.tensor([5, -1, 7, 0, -1, 63], dtype=torch.int64)
+    binding.pa_check_slots(ok, 64)
+    binding.pa_check_slots(torch.empty(0, dtype=torch.int64), 64)
+    with pytest.raises(PagedAttnError) as e:
+        binding.pa_check_slots(torch.tensor([5, 9, 5], dtype=torch.int64), 64)
+    assert e.value.code == binding.PA_ERR_INVALID and "entry 2" in str(e.value)
+    with pytest.raises(PagedAttnError) as e:
+        binding.pa_check_slots(torch.tensor([5, 64], dtype=torch.int64), 64)
+    assert e.value.code == binding.PA_ERR_OUT_OF_RANGE and "entry 1" in str(e.value)
+    a = BlockAllocator(64, 16)
+    for sid, L in enumerate([6, 50, 8, 100]):
+        a.pa_seq_grow(sid, L)
+    slots = a.pa_build_slot_mapping([0, 1, 2, 3], [0, 0, 0, 0], [6, 50, 8, 100])
+    binding.pa_check_slots(slots, 64 * 16)
