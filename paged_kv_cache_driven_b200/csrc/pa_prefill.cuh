@@ -444,7 +444,11 @@ __global__ void __launch_bounds__(576, 1)
           tc::tmem_ld32(tS + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c4 * 32]));
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < HK; ++c) x[c] = diag && kb + c > lim ? -INFINITY : __uint_as_float(u[c]);
+        for (int c = 0; c < HK; ++c) x[c] = __uint_as_float(u[c]);
+        if (diag) {  // only tiles that reach past the row's last key pay for the mask
+#pragma unroll
+          for (int c = 0; c < HK; ++c) x[c] = kb + c > lim ? -INFINITY : x[c];
+        }
       }
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
