@@ -19,7 +19,10 @@ One step, in this order (the order is part of the contract the tests check):
      prompt K/V through slot_mapping (the prefill write of Step 6 "Prefill").
 
 Random draws (lengths, budgets, token values, the shuffled free list) come from
-``workloads.BatchingLoop``; everything else runs in the library.
+``workloads.BatchingLoop``; everything else runs in the library. The host time
+spent in allocator calls (grow, slot mapping, tables, free) is summed in
+``host_s`` and reported per step in the step's record, with the device slot
+mappings of the step's admissions.
 
 With ``graph=True`` the device part of step 2-3 (the three uploads from the
 pinned staging set and the append + decode launches) is a CUDA graph: the
@@ -32,6 +35,7 @@ give the same bits.
 """
 
 import math
+import time
 
 import torch
 
@@ -97,6 +101,8 @@ class ContinuousBatching:
         self.v_buf = torch.empty_like(self.q_buf)
         self.graphs = [None] * len(self.staging.sets)
         self.events = []  # (kind, seq_id, serial, prompt_len) for admissions / retirements
+        self.host_s = 0.0  # seconds spent in allocator calls (grow, slots, tables, free)
+        self.prompt_slots = []  # device slot mappings of the admissions since the last step
         for b in range(B):
             self.slots.append(self._admit(loop.initial_lens[b], loop.budgets[b]))
 
@@ -104,10 +110,14 @@ class ContinuousBatching:
         """Creates a request, allocates its prompt blocks and appends its prompt K/V."""
         sid = self.serial
         self.serial += 1
+        t = time.perf_counter()
         self.alloc.pa_seq_grow(sid, prompt_len)
+        h_slots = self.alloc.pa_build_slot_mapping([sid], [0], [prompt_len])
+        self.host_s += time.perf_counter() - t
         k, v = self.loop.prompt_kv(sid, prompt_len, self.device)
-        slots = self.alloc.pa_build_slot_mapping([sid], [0], [prompt_len]).to(self.device)
+        slots = h_slots.to(self.device)
         binding.pa_kv_append(k, v, slots, self.k_cache, self.v_cache)
+        self.prompt_slots.append(slots)
         self.events.append(("admit", sid, prompt_len))
         return [sid, max(1, int(budget))]
 
@@ -130,11 +140,15 @@ class ContinuousBatching:
                               self.d_lens, self.scale, max_len, partition=0, workspace=self.ws)
 
     def step(self, step_idx):
-        """One decode step; returns a record of what it did (for checking)."""
+        """One decode step; returns a record of what it did (for checking and timing)."""
         ids = self.seq_ids()
         set_idx = self.staging.k % len(self.staging.sets)
         h = self.staging.acquire()
+        host0 = self.host_s
+        self.prompt_slots = []
+        t = time.perf_counter()
         self.alloc.pa_prepare_step(ids, 1, self.MB, h["slots"], h["tables"], h["lens"])
+        self.host_s += time.perf_counter() - t
         q, k, v = self.loop.token_kv(step_idx, self.B, self.device)
         self._qkv = (q, k, v)
         if self.fixed_plan:
@@ -159,10 +173,14 @@ class ContinuousBatching:
             self.slots[b][1] -= 1
             if self.slots[b][1] <= 0:
                 old = self.slots[b][0]
+                t = time.perf_counter()
                 self.alloc.pa_seq_free(old)
+                self.host_s += time.perf_counter() - t
                 self.events.append(("retire", old, 0))
                 L, budget = self.loop.arrival()
                 self.slots[b] = self._admit(L, budget)
                 record["retired"].append(old)
                 record["admitted"].append((self.slots[b][0], L, self.slots[b][1]))
+        record["host_s"] = self.host_s - host0
+        record["prompt_slots"] = self.prompt_slots
         return record
