@@ -50,6 +50,7 @@ H, D, S, BATCH, MAX_LEN = 40, 128, 16, 64, 2048
 DTYPE = torch.bfloat16
 ELEM = 2
 METRIC = "paged decode attention KV GB/s"
+E2E_MIN_STEPS = 200
 WORKLOAD = "llama2-13b-shaped single-layer decode: 40 heads, head_dim 128, block 16, bf16, " \
            "batch 64, seq_lens U[1,2048], permuted pool"
 
@@ -1018,7 +1019,10 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    extra = args.warmup + args.steps + 8
+    # the end-to-end leg runs at least E2E_MIN_STEPS steps, so that its one pipeline
+    # fill and drain weigh the same whatever --steps is
+    e2e_steps = max(args.steps, E2E_MIN_STEPS)
+    extra = args.warmup + e2e_steps + 8
     wl = Workload(seed=args.seed + 1000 * rank, device=device, extra_tokens=extra)
     stream = torch.cuda.current_stream()
 
@@ -1076,16 +1080,16 @@ def main():
     torch.cuda.synchronize()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
-    for _ in range(args.steps):
+    for _ in range(e2e_steps):
         wl.e2e_step()
     wl.e2e_drain()  # the last result copies are inside the timed region
     e_end.record(stream)
     torch.cuda.synchronize()
     # every e2e step grew each request by one token: timed step j decoded L + W + j + 1
     e2e_bytes = sum(decode_bytes([L + args.warmup + j + 1 for L in wl.lens])
-                    + append_bytes(BATCH, slots=False) for j in range(args.steps))
+                    + append_bytes(BATCH, slots=False) for j in range(e2e_steps))
     assert [wl.alloc.pa_seq_len(i) for i in wl.seq_ids] == \
-        [L + args.warmup + args.steps for L in wl.lens]
+        [L + args.warmup + e2e_steps for L in wl.lens]
     barrier(world)
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device)
     e2e_total = sum_over_ranks(e2e_bytes, world, device)
@@ -1132,7 +1136,7 @@ def main():
                     "api": "pa_stepper_step (host allocator step, uploads, pa_decode_append, "
                            "download; every request grows by one token per step)",
                     "h2d_bytes_per_step": wl.h2d_bytes(), "d2h_bytes_per_step": wl.d2h_bytes(),
-                    "ms_per_step": round(e2e_ms / args.steps, 4)},
+                    "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4)},
             "gpu_launches": wl.launches_per_step(fused=True) * args.steps,
             "clocks": clk.summary(),
         }

@@ -101,8 +101,11 @@ pa_status pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping
  *   max_seq_len   a host-side upper bound on seq_lens (sizes the grid); must be
  *                 <= MB * S. Requests longer than it are clamped and flagged
  *   workspace     device scratch of ws_bytes >= pa_decode_workspace_bytes(...)
- *                 for the same arguments; may be NULL when that size is 0. The
- *                 library keeps no pointer to it after the call's work ends
+ *                 for the same arguments; may be NULL when that size is 0. It
+ *                 needs no initialisation and may be reused by later calls of
+ *                 any shape, but calls whose work overlaps on the GPU need
+ *                 workspaces of their own. The library keeps no pointer to it
+ *                 after the call's work ends
  * Requires 16-byte aligned q, k_cache, v_cache, out and workspace.
  * ------------------------------------------------------------------------- */
 size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, int partition);
@@ -230,12 +233,16 @@ pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k
                         int max_seq_len, void* workspace, size_t ws_bytes, void* stream);
 
 /* Split-KV workspace layout, for tests that inspect the partition pass
- * (NP = number of partitions, all fp32, offsets in bytes from `workspace`):
+ * (NP = number of partitions, n = B*H*NP, all fp32, offsets in bytes from
+ * `workspace`):
  *   m   [B, H, NP] at 0                 max of scale * q.k * log2(e) (base-2 units)
- *   l   [B, H, NP] at B*H*NP*4          sum of 2^(s - m) over the partition
- *   acc [B, H, NP, D] at align256(B*H*NP*8)   sum of 2^(s - m) * V, unnormalised
+ *   l   [B, H, NP] at n*4               sum of 2^(s - m) over the partition
+ *   acc [B, H, NP, D] at align256(n*8)  sum of 2^(s - m) * V, unnormalised
  * Only partitions p < ceil(seq_lens[i] / partition) of requests with more than
- * one partition are written. */
+ * one partition are written; a second kernel, launched so that it can start
+ * while the first finishes, merges them by log-sum-exp ([card] "헷갈리기 쉬운
+ * 구분"). Everything the merge reads is written by the same call, so the
+ * workspace needs no initialisation. */
 
 /* ---------------------------------------------------------------------------
  * Decode without any caller-provided scratch. This entry point has no
@@ -248,9 +255,12 @@ pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k
  * the workspace: the split-KV partials go to a static device array of
  * PA_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads it,
  * until the process exits. The call allocates nothing.
- *   - The first call on a device looks up that array's device address
- *     (cudaGetSymbolAddress) with the device current; make that first call
- *     before any stream capture on the device.
+ *   - The first call on a device that needs the array looks up its device
+ *     address (cudaGetSymbolAddress) with the device current, and again
+ *     whenever the device's context has changed (after a cudaDeviceReset);
+ *     make that first call before any stream capture on the device.
+ *   - Arguments are checked as pa_decode checks them, first: a bad argument
+ *     returns PA_ERR_INVALID whatever the size of the split.
  *   - A call whose split needs more scratch than the array holds (see
  *     pa_decode_workspace_bytes) returns PA_ERR_OOM and launches nothing.
  *   - Every call shares the one array and leaves its partials there; nothing
@@ -259,6 +269,9 @@ pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k
  *     race on the array: order them on one stream or serialise them.
  * ------------------------------------------------------------------------- */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* The size of that array in this build of the library (PA_NOALLOC_SCRATCH_BYTES). */
+size_t pa_noalloc_scratch_bytes(void);
 
 pa_status pa_decode_noalloc(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
                             const void* v_cache, const int32_t* block_tables, int MB,

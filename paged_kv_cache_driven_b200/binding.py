@@ -39,6 +39,7 @@ _SIGNATURES = {
                        _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_decode_noalloc": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32,
                            _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "pa_noalloc_scratch_bytes": ([], _sz),
     # k, v, in_dt, slot_mapping, k_cache, v_cache, k_scale, v_scale, T, H, D, S, NB, stream
     "pa_kv_append_fp8": ([_vp, _vp, _i32, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, _i32,
                           _i32, _i32, _i32, _i32, _vp], _i32),
@@ -325,7 +326,9 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, m
                                    int(max_seq_len), _stream(stream)), "pa_decode_noalloc")
 
 
-PA_NOALLOC_SCRATCH_BYTES = 16 << 20
+def pa_noalloc_scratch_bytes():
+    """Size of the library's static scratch array that pa_decode_noalloc uses."""
+    return int(lib().pa_noalloc_scratch_bytes())
 
 
 def pa_copy_blocks(k_cache, v_cache, src_dst, stream=None):

@@ -1,8 +1,8 @@
-// The device half of the C ABI (pagedattn.h): argument validation, launch
-// planning, tensor-map encoding and kernel dispatch for pa_kv_append,
-// pa_decode / pa_decode_append / pa_decode_gqa / pa_decode_noalloc,
-// pa_prefill and pa_copy_blocks, and the device error word. Every check runs
-// on the host before anything is launched.
+// The C-ABI layer (pagedattn.h): argument validation, launch planning, the
+// split-KV workspace layout, tensor-map encoding and dispatch to the launchers
+// of the translation units that hold the kernels (pa_k_*.cu), the device
+// error words, and pa_decode_noalloc's static scratch. Every check runs on the
+// host before anything is launched.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -15,18 +15,16 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
-#include <type_traits>
 
-#include "pa_append.cuh"
-#include "pa_decode.cuh"
-#include "pa_gqa.cuh"
-#include "pa_prefill.cuh"
+#include "pa_launch.h"
 #include "pagedattn.h"
+
+using pa::host::ceil_div;
+using pa::host::kMaxDevices;
 
 namespace {
 
 constexpr int kDefaultPartition = 512;  // tokens per split-KV partition when splitting
-constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -37,8 +35,6 @@ bool out_dtype_ok(pa_dtype dt) { return dt == PA_F16 || dt == PA_BF16 || dt == P
 bool decode_shape_ok(int D, int S) {
   return (D == 64 || D == 128 || D == 256) && (S == 8 || S == 16 || S == 32);
 }
-
-int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -57,9 +53,12 @@ int sm_count() {
 //   -1      never split: one partition covering any length up to MB * S
 //   > 0     that many tokens (a multiple of S)
 //   0       automatic: 512-token partitions, halved (down to 64 tokens, staying a
-//           multiple of S) while the grid would hold fewer than about four
-//           waves of CTAs (three CTAs per SM), so that small batches still
-//           spread over every SM; no split if one partition covers every request
+//           multiple of S) while the grid would hold fewer CTAs than the device
+//           has SMs, so that small batches still spread over every SM; no split
+//           if one partition covers every request. (Measured at batch 1, 32
+//           heads, 1.3K tokens: 256-token partitions, 192 CTAs, are fastest for
+//           head sizes 64 to 256; 64-token ones, 672 CTAs, are 40 % slower,
+//           each CTA's fixed start and end costing more than its short stream.)
 bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* NP_out) {
   if (max_seq_len < 0 || S <= 0) return false;
   int P;
@@ -73,7 +72,7 @@ bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* 
     P = partition;
   } else {
     P = kDefaultPartition;
-    const int64_t target = 4LL * 3 * sm_count();
+    const int64_t target = sm_count();
     const int64_t pairs = static_cast<int64_t>(B > 0 ? B : 1) * (H > 0 ? H : 1);
     while (P > 64 && (P / 2) % S == 0 && pairs * ceil_div(max_seq_len, P) < target) P /= 2;
   }
@@ -89,51 +88,26 @@ bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* 
   return true;
 }
 
+// Split-KV workspace: m and l [B, H, NP], then (256-byte aligned) acc [B, H, NP, D].
+size_t acc_offset(size_t n) { return align256(n * 2 * sizeof(float)); }
+
 size_t workspace_for(int B, int H, int D, int NP) {
   if (NP <= 1) return 0;
   const size_t n = static_cast<size_t>(B) * H * NP;
-  return align256(n * 2 * sizeof(float)) + n * D * sizeof(float);
+  return acc_offset(n) + n * D * sizeof(float);
 }
 
-pa_status cuda_status() {
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
-// The shared-memory opt-in is a per-device property of a kernel function.
-template <typename K>
-bool opt_in_smem(K kern, int bytes, bool (&configured)[kMaxDevices]) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  if (!configured[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-        cudaSuccess)
-      return false;
-    configured[dev] = true;
-  }
-  return true;
-}
-
-template <typename TO, int D>
-void launch_reduce(const pa::DecodeParams& prm, cudaStream_t stream) {
-  if (prm.NP > 1) {
-    const int64_t pairs = static_cast<int64_t>(prm.B) * prm.H;
-    pa::splitkv_reduce_kernel<TO, D>
-        <<<static_cast<unsigned>((pairs + 3) / 4), 128, 0, stream>>>(prm);
-  }
-}
-
-// One KV head per query head (or an odd group size): the multi-head kernel,
-// each CTA reading its query head's KV head.
-template <typename T, typename TO, int D, int S, bool APPEND>
-pa_status launch_decode(const pa::DecodeParams& prm, cudaStream_t stream) {
-  using Tl = pa::DecodeTiling<D, S>;
-  auto kern = pa::paged_decode_partition_kernel<T, TO, D, S, APPEND>;
-  static bool configured[kMaxDevices] = {};
-  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
-  const dim3 grid(prm.NP, prm.H, prm.B);
-  kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
-  launch_reduce<TO, D>(prm, stream);
-  return cuda_status();
+// Points the kernel parameters at the workspace parts for NP > 1 partitions.
+void set_split(pa::DecodeParams& prm, void* workspace, int B, int H, int P, int NP,
+               int64_t L_max) {
+  const size_t n = static_cast<size_t>(B) * H * NP;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  prm.ws_m = reinterpret_cast<float*>(base);
+  prm.ws_l = prm.ws_m + n;
+  prm.ws_acc = reinterpret_cast<float*>(base + acc_offset(n));
+  prm.P = P;
+  prm.NP = NP;
+  prm.L_cap = static_cast<int>(std::min<int64_t>(L_max, static_cast<int64_t>(NP) * P));
 }
 
 // ---- tensor maps of the caches, for the tiled TMA loads ---------------------
@@ -166,12 +140,20 @@ struct RowMapKey {
   }
 };
 
-bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows, pa_dtype dt) {
+}  // namespace
+
+namespace pa {
+namespace host {
+
+// kind: 0 = f16, 1 = bf16; boxes of 64 elements, so every box row is 128 bytes,
+// the 128-byte swizzle's width.
+static bool row_map_kind(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows,
+                         int kind) {
   static std::mutex mu;
   static RowMapKey keys[16];
   static CUtensorMap maps[16];
   static int used = 0, next = 0;
-  const RowMapKey key{base, rows, D, box_rows, static_cast<int>(dt)};
+  const RowMapKey key{base, rows, D, box_rows, kind};
   std::lock_guard<std::mutex> lock(mu);
   for (int k = 0; k < used; ++k)
     if (keys[k] == key) {
@@ -180,15 +162,17 @@ bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_ro
     }
   auto fn = encode_fn();
   if (!fn) return false;
+  const cuuint64_t esize = 2;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * esize};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType type =
+      kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap map;
-  if (fn(&map, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-         2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  if (fn(&map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   const int slot = used < 16 ? used++ : next;
   next = (slot + 1) % 16;
@@ -198,76 +182,8 @@ bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_ro
   return true;
 }
 
-// Grouped query heads: one CTA per (partition, KV head, request, chunk of up to
-// 16 query heads), the contraction on the tensor cores.
-template <typename T, typename TO, int D, int S, bool APPEND, int NHT>
-pa_status launch_grouped(const pa::DecodeParams& prm, cudaStream_t stream) {
-  using Tg = pa::GqaTiling<D>;
-  auto kern = pa::paged_decode_gqa_kernel<T, TO, D, S, APPEND, NHT>;
-  static bool configured[kMaxDevices] = {};
-  if (!opt_in_smem(kern, Tg::SMEM, configured)) return PA_ERR_CUDA;
-  const int64_t rows = static_cast<int64_t>(prm.NB) * prm.Hkv * S;
-  if (rows <= 0 || rows > INT_MAX) return PA_ERR_INVALID;  // TMA row coordinates are int32
-  const pa_dtype dt = std::is_same<T, __half>::value ? PA_F16 : PA_BF16;
-  CUtensorMap tmk, tmv;
-  if (!row_map(&tmk, prm.k_cache, rows, D, S < 16 ? S : 16, dt) ||
-      !row_map(&tmv, prm.v_cache, rows, D, S < 16 ? S : 16, dt))
-    return PA_ERR_CUDA;
-  const int G = prm.H / prm.Hkv;
-  const dim3 grid(prm.NP, prm.Hkv * ((G + 15) / 16), prm.B);
-  kern<<<grid, (Tg::NC + 1) * 32, Tg::SMEM, stream>>>(prm, tmk, tmv);
-  launch_reduce<TO, D>(prm, stream);
-  return cuda_status();
-}
-
-// E4M3 cache: the multi-head kernel with one-byte cache elements.
-template <typename T, typename TO, int D, int S>
-pa_status launch_decode_fp8(const pa::DecodeParams& prm, cudaStream_t stream) {
-  using Tl = pa::DecodeTiling<D, S, 1>;
-  auto kern = pa::paged_decode_partition_kernel<T, TO, D, S, false, __nv_fp8_e4m3>;
-  static bool configured[kMaxDevices] = {};
-  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
-  const dim3 grid(prm.NP, prm.H, prm.B);
-  kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
-  launch_reduce<TO, D>(prm, stream);
-  return cuda_status();
-}
-
-template <typename T, typename TO>
-pa_status dispatch_fp8_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t st) {
-#define PA_CASE(DD, SS) \
-  if (D == DD && S == SS) return launch_decode_fp8<T, TO, DD, SS>(prm, st);
-  PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
-  PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
-  PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
-#undef PA_CASE
-  return PA_ERR_INVALID;
-}
-
-template <typename T, typename TO, bool APPEND>
-pa_status dispatch_shape(const pa::DecodeParams& prm, int D, int S, cudaStream_t st) {
-  const bool grouped = prm.H != prm.Hkv;
-#define PA_CASE(DD, SS)                                                            \
-  if (D == DD && S == SS)                                                          \
-    return grouped ? (prm.H / prm.Hkv <= 8 ? launch_grouped<T, TO, DD, SS, APPEND, 1>(prm, st)   \
-                                           : launch_grouped<T, TO, DD, SS, APPEND, 2>(prm, st)) \
-                   : launch_decode<T, TO, DD, SS, APPEND>(prm, st);
-  PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
-  PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
-  PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
-#undef PA_CASE
-  return PA_ERR_INVALID;
-}
-
-template <typename T, bool APPEND>
-pa_status dispatch_out(const pa::DecodeParams& prm, pa_dtype out_dt, int D, int S,
-                       cudaStream_t st) {
-  switch (out_dt) {
-    case PA_F32: return dispatch_shape<T, float, APPEND>(prm, D, S, st);
-    case PA_F16: return dispatch_shape<T, __half, APPEND>(prm, D, S, st);
-    case PA_BF16: return dispatch_shape<T, __nv_bfloat16, APPEND>(prm, D, S, st);
-  }
-  return PA_ERR_INVALID;
+bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows, pa_dtype dt) {
+  return row_map_kind(out, base, rows, D, box_rows, dt == PA_BF16 ? 1 : 0);
 }
 
 // ---- paged prefill -------------------------------------------------------------
@@ -289,46 +205,8 @@ bool query_map(CUtensorMap* out, const void* q, int64_t T, int H, int D, pa_dtyp
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, typename TO, int D, int S>
-pa_status launch_prefill(const pa::PrefillParams& prm, const void* q, cudaStream_t stream) {
-  using Tl = pa::PrefillTiling<D, std::is_same<T, __nv_bfloat16>::value>;
-  auto kern = pa::paged_prefill_kernel<T, TO, D, S>;
-  static bool configured[kMaxDevices] = {};
-  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
-  const pa_dtype dt = std::is_same<T, __half>::value ? PA_F16 : PA_BF16;
-  const int64_t rows = static_cast<int64_t>(prm.NB) * prm.Hkv * S;
-  CUtensorMap tmq, tmk, tmv;
-  if (!query_map(&tmq, q, prm.T, prm.H, D, dt) || !row_map(&tmk, prm.k_cache, rows, D, S, dt) ||
-      !row_map(&tmv, prm.v_cache, rows, D, S, dt))
-    return PA_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>(ceil_div(prm.max_q_len, Tl::NQT * Tl::BM)), prm.H, prm.B);
-  kern<<<grid, Tl::THREADS, Tl::SMEM, stream>>>(prm, tmq, tmk, tmv);
-  return cuda_status();
-}
-
-template <typename T, typename TO>
-pa_status dispatch_prefill_shape(const pa::PrefillParams& prm, const void* q, int D, int S,
-                                 cudaStream_t st) {
-#define PA_CASE(DD, SS) \
-  if (D == DD && S == SS) return launch_prefill<T, TO, DD, SS>(prm, q, st);
-  PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32) PA_CASE(64, 64) PA_CASE(64, 128)
-  PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32) PA_CASE(128, 64) PA_CASE(128, 128)
-#undef PA_CASE
-  return PA_ERR_INVALID;
-}
-
-template <typename T>
-pa_status dispatch_prefill(const pa::PrefillParams& prm, const void* q, pa_dtype out_dt, int D,
-                           int S, cudaStream_t st) {
-  switch (out_dt) {
-    case PA_F32: return dispatch_prefill_shape<T, float>(prm, q, D, S, st);
-    case PA_F16: return dispatch_prefill_shape<T, __half>(prm, q, D, S, st);
-    case PA_BF16: return dispatch_prefill_shape<T, __nv_bfloat16>(prm, q, D, S, st);
-  }
-  return PA_ERR_INVALID;
-}
-
-}  // namespace
+}  // namespace host
+}  // namespace pa
 
 extern "C" {
 
@@ -354,17 +232,8 @@ pa_status pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping
   if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
-  const int vpr = D / 8;
-  const int64_t total = static_cast<int64_t>(T) * H * vpr;
-  const int64_t n_slots = static_cast<int64_t>(NB) * S;
-  int64_t blocks = ceil_div(total, 256);
-  const int64_t cap = 148LL * 16;  // grid-stride beyond ~16 CTAs per SM
-  if (blocks > cap) blocks = cap;
-  pa::kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0,
-                         static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total, H, vpr, S, n_slots);
-  return cuda_status();
+  return pa::host::launch_kv_append(k, v, slot_mapping, k_cache, v_cache, T, H, D, S, NB,
+                                    static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst, int n, int H,
@@ -374,14 +243,8 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst, i
   if (n == 0) return PA_OK;
   if (!k_cache || !v_cache || !src_dst || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
-  const int64_t vpb = static_cast<int64_t>(H) * S * D / 8;  // 16-byte vectors per block
-  const int64_t total = vpb * n;
-  int64_t blocks = ceil_div(total, 256);
-  if (blocks > 148LL * 16) blocks = 148LL * 16;
-  pa::copy_blocks_kernel<<<static_cast<unsigned>(blocks), 256, 0,
-                           static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), src_dst, total, vpb, NB);
-  return cuda_status();
+  return pa::host::launch_copy_blocks(k_cache, v_cache, src_dst, n, H, S, D, NB,
+                                      static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partition,
@@ -407,12 +270,14 @@ size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, in
 
 namespace {
 
-// pa_decode and pa_decode_append: k_new / v_new null = plain decode.
-pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_new,
-                      const void* v_new, const void* k_cache, const void* v_cache,
-                      const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
-                      int B, int H, int Hkv, int D, int S, int NB, pa_dtype dt, int partition,
-                      int max_seq_len, void* workspace, size_t ws_bytes, void* stream) {
+// The host checks of pa_decode's arguments, workspace aside (shared by its
+// variants). On PA_OK, *P / *NP hold the plan and *noop is set for B == 0.
+pa_status decode_check(const void* out, pa_dtype out_dt, const void* q, const void* k_cache,
+                       const void* v_cache, const int32_t* block_tables, int MB,
+                       const int32_t* seq_lens, float scale, int B, int H, int Hkv, int D, int S,
+                       int NB, pa_dtype dt, int partition, int max_seq_len, int* P, int* NP,
+                       bool* noop) {
+  *noop = false;
   if (B < 0 || H <= 0 || NB < 0 || MB < 0) return PA_ERR_INVALID;
   if (Hkv <= 0 || H % Hkv != 0) return PA_ERR_INVALID;
   if (!cache_dtype_ok(dt) || !out_dtype_ok(out_dt) || !decode_shape_ok(D, S)) return PA_ERR_INVALID;
@@ -420,13 +285,31 @@ pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_n
   if (B > 65535 || H > 65535) return PA_ERR_INVALID;  // grid y / z limits
   const int64_t L_max = static_cast<int64_t>(MB) * S;
   if (L_max > INT_MAX || max_seq_len < 0 || max_seq_len > L_max) return PA_ERR_INVALID;
-  int P, NP;
-  if (!plan(B, H, S, max_seq_len, partition, &P, &NP)) return PA_ERR_INVALID;
-  if (B == 0) return PA_OK;
+  if (!plan(B, H, S, max_seq_len, partition, P, NP)) return PA_ERR_INVALID;
+  if (B == 0) {
+    *noop = true;
+    return PA_OK;
+  }
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || MB == 0)
     return PA_ERR_INVALID;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
+  return PA_OK;
+}
+
+// pa_decode and pa_decode_append: k_new / v_new null = plain decode.
+pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_new,
+                      const void* v_new, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
+                      int B, int H, int Hkv, int D, int S, int NB, pa_dtype dt, int partition,
+                      int max_seq_len, void* workspace, size_t ws_bytes, void* stream) {
+  int P, NP;
+  bool noop;
+  const pa_status chk = decode_check(out, out_dt, q, k_cache, v_cache, block_tables, MB, seq_lens,
+                                     scale, B, H, Hkv, D, S, NB, dt, partition, max_seq_len, &P,
+                                     &NP, &noop);
+  if (chk != PA_OK || noop) return chk;
+  const int64_t L_max = static_cast<int64_t>(MB) * S;
   const size_t need = workspace_for(B, H, D, NP);
   if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace))) return PA_ERR_INVALID;
 
@@ -445,28 +328,17 @@ pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_n
   prm.Hkv = Hkv;
   prm.NB = NB;
   if (NP > 1) {
-    const size_t n = static_cast<size_t>(B) * H * NP;
-    prm.ws_m = static_cast<float*>(workspace);
-    prm.ws_l = prm.ws_m + n;
-    prm.ws_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                          align256(n * 2 * sizeof(float)));
-    prm.P = P;
-    prm.NP = NP;
-    prm.L_cap = static_cast<int>(std::min<int64_t>(L_max, static_cast<int64_t>(NP) * P));
+    set_split(prm, workspace, B, H, P, NP, L_max);
   } else {
     prm.P = static_cast<int>(L_max > 0 ? L_max : S);  // one partition covers every block
     prm.NP = 1;
     prm.L_cap = static_cast<int>(L_max);
   }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
   prm.k_new = k_new;
   prm.v_new = v_new;
-  if (k_new) {
-    if (dt == PA_F16) return dispatch_out<__half, true>(prm, out_dt, D, S, st);
-    return dispatch_out<__nv_bfloat16, true>(prm, out_dt, D, S, st);
-  }
-  if (dt == PA_F16) return dispatch_out<__half, false>(prm, out_dt, D, S, st);
-  return dispatch_out<__nv_bfloat16, false>(prm, out_dt, D, S, st);
+  if (H != Hkv) return pa::host::launch_grouped(prm, dt, out_dt, D, S, k_new != nullptr, st);
+  return pa::host::launch_decode16(prm, dt, out_dt, D, S, k_new != nullptr, st);
 }
 
 }  // namespace
@@ -541,9 +413,7 @@ pa_status pa_prefill(void* out, pa_dtype out_dt, const void* q, const void* k_ca
   prm.NB = NB;
   prm.T = T;
   prm.max_q_len = max_q_len;
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dt == PA_BF16 ? dispatch_prefill<__nv_bfloat16>(prm, q, out_dt, D, S, st)
-                       : dispatch_prefill<__half>(prm, q, out_dt, D, S, st);
+  return pa::host::launch_prefill(prm, q, dt, out_dt, D, S, static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_kv_append_fp8(const void* k, const void* v, pa_dtype in_dt,
@@ -558,24 +428,8 @@ pa_status pa_kv_append_fp8(const void* k, const void* v, pa_dtype in_dt,
   if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
-  const int vpr = D / 8;
-  const int64_t total = static_cast<int64_t>(T) * H * vpr;
-  const int64_t n_slots = static_cast<int64_t>(NB) * S;
-  int64_t blocks = ceil_div(total, 256);
-  const int64_t cap = 148LL * 16;
-  if (blocks > cap) blocks = cap;
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (in_dt == PA_BF16)
-    pa::kv_append_fp8_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
-        static_cast<uint2*>(k_cache), static_cast<uint2*>(v_cache), k_scale, v_scale, total, H,
-        vpr, S, n_slots);
-  else
-    pa::kv_append_fp8_kernel<__half><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
-        static_cast<uint2*>(k_cache), static_cast<uint2*>(v_cache), k_scale, v_scale, total, H,
-        vpr, S, n_slots);
-  return cuda_status();
+  return pa::host::launch_kv_append_fp8(k, v, in_dt, slot_mapping, k_cache, v_cache, k_scale,
+                                        v_scale, T, H, D, S, NB, static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
@@ -615,43 +469,23 @@ pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt
   prm.Hkv = H;
   prm.NB = NB;
   if (NP > 1) {
-    const size_t n = static_cast<size_t>(B) * H * NP;
-    prm.ws_m = static_cast<float*>(workspace);
-    prm.ws_l = prm.ws_m + n;
-    prm.ws_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                          align256(n * 2 * sizeof(float)));
-    prm.P = P;
-    prm.NP = NP;
-    prm.L_cap = static_cast<int>(std::min<int64_t>(L_max, static_cast<int64_t>(NP) * P));
+    set_split(prm, workspace, B, H, P, NP, L_max);
   } else {
     prm.P = static_cast<int>(L_max > 0 ? L_max : S);
     prm.NP = 1;
     prm.L_cap = static_cast<int>(L_max);
   }
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (q_dt == PA_F16) {
-    switch (out_dt) {
-      case PA_F32: return dispatch_fp8_shape<__half, float>(prm, D, S, st);
-      case PA_F16: return dispatch_fp8_shape<__half, __half>(prm, D, S, st);
-      case PA_BF16: return dispatch_fp8_shape<__half, __nv_bfloat16>(prm, D, S, st);
-    }
-  } else {
-    switch (out_dt) {
-      case PA_F32: return dispatch_fp8_shape<__nv_bfloat16, float>(prm, D, S, st);
-      case PA_F16: return dispatch_fp8_shape<__nv_bfloat16, __half>(prm, D, S, st);
-      case PA_BF16: return dispatch_fp8_shape<__nv_bfloat16, __nv_bfloat16>(prm, D, S, st);
-    }
-  }
-  return PA_ERR_INVALID;
+  return pa::host::launch_decode_fp8(prm, q_dt, out_dt, D, S, static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_get_device_error(void* stream, uint32_t* flags) {
   if (!flags) return PA_ERR_INVALID;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, pa::g_error_word, sizeof(v)) != cudaSuccess) return PA_ERR_CUDA;
-  const unsigned int zero = 0;
-  if (cudaMemcpyToSymbol(pa::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return PA_ERR_CUDA;
+  using namespace pa::host;
+  if (!take_error_append(&v) || !take_error_decode16(&v) || !take_error_grouped(&v) ||
+      !take_error_fp8(&v) || !take_error_prefill(&v))
+    return PA_ERR_CUDA;
   *flags = v;
   return PA_OK;
 }
@@ -668,12 +502,48 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch per device, looked up on the first call
-// made with that device current. The host-side name of the array is only a
-// stand-in for the symbol, never a usable device address.
-std::atomic<void*> g_noalloc_scratch_addr[kMaxDevices];
+// Device address of g_noalloc_scratch per device, looked up with the device
+// current and keyed by the context it was looked up in: a context that is torn
+// down and created again (cudaDeviceReset, for one) loads the module again, and
+// the array can move. The host-side name of the array is only a stand-in for
+// the symbol, never a usable device address.
+struct ScratchAddr {
+  unsigned long long ctx_id = 0;  // cuCtxGetId of the context the address belongs to
+  void* addr = nullptr;
+};
+std::mutex g_noalloc_mu;
+ScratchAddr g_noalloc_addr[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The unique id of the current context (0 if the driver does not give one).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 }  // namespace
+
+extern "C" size_t pa_noalloc_scratch_bytes(void) { return PA_NOALLOC_SCRATCH_BYTES; }
 
 extern "C" pa_status pa_decode_noalloc(void* out, pa_dtype out_dt, const void* q,
                                        const void* k_cache, const void* v_cache,
@@ -681,18 +551,29 @@ extern "C" pa_status pa_decode_noalloc(void* out, pa_dtype out_dt, const void* q
                                        const int32_t* seq_lens, float scale, int B, int H, int D,
                                        int S, int NB, pa_dtype dt, int partition, int max_seq_len,
                                        void* stream) {
+  // pa_decode's own checks first, so a bad argument is PA_ERR_INVALID, never PA_ERR_OOM
   int P, NP;
-  if (B < 0 || H <= 0 || !decode_shape_ok(D, S) || !plan(B, H, S, max_seq_len, partition, &P, &NP))
-    return PA_ERR_INVALID;
+  bool noop;
+  const pa_status st = decode_check(out, out_dt, q, k_cache, v_cache, block_tables, MB, seq_lens,
+                                    scale, B, H, H, D, S, NB, dt, partition, max_seq_len, &P, &NP,
+                                    &noop);
+  if (st != PA_OK || noop) return st;
   const size_t need = workspace_for(B, H, D, NP);
   if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_OOM;  // larger than the static array
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
-  void* scratch = g_noalloc_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!scratch) {
-    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch)
-      return PA_ERR_CUDA;
-    g_noalloc_scratch_addr[dev].store(scratch, std::memory_order_release);
+  void* scratch = nullptr;
+  if (need > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+    const unsigned long long ctx = current_context_id();
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    ScratchAddr& a = g_noalloc_addr[dev];
+    if (!a.addr || a.ctx_id != ctx || ctx == 0) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return PA_ERR_CUDA;
+      a.addr = p;
+      a.ctx_id = ctx;
+    }
+    scratch = a.addr;
   }
   return pa_decode(out, out_dt, q, k_cache, v_cache, block_tables, MB, seq_lens, scale, B, H, D, S,
                    NB, dt, partition, max_seq_len, scratch, PA_NOALLOC_SCRATCH_BYTES, stream);

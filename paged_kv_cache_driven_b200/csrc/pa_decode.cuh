@@ -37,29 +37,10 @@
 #include <type_traits>
 
 #include "pa_device.cuh"
+#include "pa_launch.h"
 
 namespace pa {
 
-struct DecodeParams {
-  void* out;                   // [B, H, D] final output (dtype TO)
-  const void* q;               // [B, H, D]
-  const void* k_cache;         // [NB, H, S, D]
-  const void* v_cache;         // [NB, H, S, D]
-  const int32_t* block_tables; // [B, MB]
-  const int32_t* seq_lens;     // [B]
-  float* ws_m;                 // [B, H, NP]
-  float* ws_l;                 // [B, H, NP]
-  float* ws_acc;               // [B, H, NP, D]
-  const void* k_new;           // [B, H, D] fused append: the new token's K (or null)
-  const void* v_new;           // [B, H, D] fused append: the new token's V (or null)
-  float q_scale;               // scale * log2(e)
-  int MB, B, H, NB;
-  int Hkv;   // KV heads in the cache; query head h reads KV head h / (H / Hkv)
-  int P;     // tokens per partition (multiple of S)
-  int NP;    // partitions in the grid
-  int L_cap; // lengths are clamped to this (MB*S, or NP*P when split)
-  float v_scale;  // V = v_scale * stored value (1 for 16-bit caches; E4M3 caches)
-};
 
 // Shapes of the partition pass for head_dim D, block_size S and EB-byte cache
 // elements (2: fp16 / bf16, 1: E4M3).
@@ -146,6 +127,7 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
   constexpr int EPL = Tl::EPL, LPR = Tl::LPR, RPW = Tl::RPW, CR = Tl::CR, NV = Tl::NV;
   constexpr int DUP = LPR / NV;  // lanes of a group holding the same row's score
 
+  grid_dependents_launch();  // the merge of split requests may be scheduled early
   const int part = blockIdx.x;
   const int h = blockIdx.y;
   const int i = blockIdx.z;
@@ -429,6 +411,10 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
 template <typename TO, int D>
 __global__ void __launch_bounds__(128) splitkv_reduce_kernel(const DecodeParams p) {
   constexpr int DL = D / 32;
+  // Launched as a programmatic dependent of the partition pass: its CTAs may be
+  // resident before that pass ends; this waits until the pass has completed
+  // and its partials are visible.
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int64_t ih = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   if (ih >= static_cast<int64_t>(p.B) * p.H) return;
@@ -472,6 +458,26 @@ __global__ void __launch_bounds__(128) splitkv_reduce_kernel(const DecodeParams 
   TO* o = static_cast<TO*>(p.out) + ih * D + lane * DL;
 #pragma unroll
   for (int e = 0; e < DL; ++e) o[e] = to_out<TO>(lsum > 0.f ? a[e] / lsum : 0.f);
+}
+
+// Launches the merge of split requests (no-op without a split) on `stream` as a
+// programmatic dependent of the partition pass launched just before it, so its
+// launch overlaps that pass's last wave instead of following it.
+template <typename TO, int D>
+inline cudaError_t launch_splitkv_reduce(const DecodeParams& p, cudaStream_t stream) {
+  if (p.NP <= 1) return cudaSuccess;
+  const int64_t pairs = static_cast<int64_t>(p.B) * p.H;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((pairs + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, splitkv_reduce_kernel<TO, D>, p);
 }
 
 }  // namespace pa

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cstdint>
@@ -12,12 +13,22 @@
 
 namespace pa {
 
-// One word per device; kernels OR PA_DEVERR_* bits into it, the host reads and
-// clears it through pa_get_device_error(). All device code is compiled as one
-// translation unit (pa_api.cu), which is the only includer of this header.
-__device__ unsigned int g_error_word = 0;
+// One word per device and per translation unit that holds kernels; kernels OR
+// PA_DEVERR_* bits into it. take_error_word() (host) reads and clears this
+// unit's word; pa_get_device_error() gathers every unit's.
+static __device__ unsigned int g_error_word = 0;
 
 __device__ __forceinline__ void raise_error(unsigned int bits) { atomicOr(&g_error_word, bits); }
+
+// Host: ORs this translation unit's error word into *bits and clears it.
+static inline bool take_error_word(unsigned int* bits) {
+  unsigned int v = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v)) != cudaSuccess) return false;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return false;
+  *bits |= v;
+  return true;
+}
 
 constexpr unsigned kFullMask = 0xffffffffu;
 
@@ -69,6 +80,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (clock64() - t0 > kWaitLimitCycles) return false;
   }
   return true;
+}
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the kernel before it on the
+// stream still runs; grid_dependency_wait() blocks until that kernel has
+// completed and its memory operations are visible. grid_dependents_launch()
+// lets the dependent grid be scheduled once every CTA of this grid has issued
+// it (or exited).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // L2 policy for data read exactly once per step (the KV slabs).

@@ -126,6 +126,7 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   constexpr int SLAB = S * D * 2;
   constexpr int KS = D / 16;  // k-steps of S
 
+  grid_dependents_launch();  // the merge of split requests may be scheduled early
   const int part = blockIdx.x;
   const int G = p.H / p.Hkv;
   const int chunks = (G + 15) / 16;

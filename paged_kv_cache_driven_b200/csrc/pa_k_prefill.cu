@@ -1,0 +1,64 @@
+// Kernels of pa_prefill: causal paged prefill attention on the fifth-generation
+// tensor cores, for both 16-bit cache dtypes, every output dtype, head size 64
+// and 128 and block sizes 8 .. 128, and their launcher.
+
+#include <type_traits>
+
+#include "pa_launch.h"
+#include "pa_prefill.cuh"
+
+namespace pa {
+namespace host {
+namespace {
+
+// One CTA per (256 query rows, query head, request).
+template <typename T, typename TO, int D, int S>
+pa_status launch(const PrefillParams& prm, const void* q, cudaStream_t stream) {
+  using Tl = PrefillTiling<D, std::is_same<T, __nv_bfloat16>::value>;
+  auto kern = paged_prefill_kernel<T, TO, D, S>;
+  static bool configured[kMaxDevices] = {};
+  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
+  const pa_dtype dt = std::is_same<T, __half>::value ? PA_F16 : PA_BF16;
+  const int64_t rows = static_cast<int64_t>(prm.NB) * prm.Hkv * S;
+  CUtensorMap tmq, tmk, tmv;
+  if (!query_map(&tmq, q, prm.T, prm.H, D, dt) || !row_map(&tmk, prm.k_cache, rows, D, S, dt) ||
+      !row_map(&tmv, prm.v_cache, rows, D, S, dt))
+    return PA_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(ceil_div(prm.max_q_len, Tl::NQT * Tl::BM)), prm.H, prm.B);
+  kern<<<grid, Tl::THREADS, Tl::SMEM, stream>>>(prm, tmq, tmk, tmv);
+  return cuda_status();
+}
+
+template <typename T, typename TO>
+pa_status by_shape(const PrefillParams& prm, const void* q, int D, int S, cudaStream_t st) {
+#define PA_CASE(DD, SS) \
+  if (D == DD && S == SS) return launch<T, TO, DD, SS>(prm, q, st);
+  PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32) PA_CASE(64, 64) PA_CASE(64, 128)
+  PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32) PA_CASE(128, 64) PA_CASE(128, 128)
+#undef PA_CASE
+  return PA_ERR_INVALID;
+}
+
+template <typename T>
+pa_status by_out(const PrefillParams& prm, const void* q, pa_dtype out_dt, int D, int S,
+                 cudaStream_t st) {
+  switch (out_dt) {
+    case PA_F32: return by_shape<T, float>(prm, q, D, S, st);
+    case PA_F16: return by_shape<T, __half>(prm, q, D, S, st);
+    case PA_BF16: return by_shape<T, __nv_bfloat16>(prm, q, D, S, st);
+  }
+  return PA_ERR_INVALID;
+}
+
+}  // namespace
+
+pa_status launch_prefill(const PrefillParams& prm, const void* q, pa_dtype dt, pa_dtype out_dt,
+                         int D, int S, cudaStream_t stream) {
+  return dt == PA_BF16 ? by_out<__nv_bfloat16>(prm, q, out_dt, D, S, stream)
+                       : by_out<__half>(prm, q, out_dt, D, S, stream);
+}
+
+bool take_error_prefill(unsigned int* bits) { return take_error_word(bits); }
+
+}  // namespace host
+}  // namespace pa

@@ -41,20 +41,11 @@
 #include <cuda.h>
 
 #include "pa_device.cuh"
+#include "pa_launch.h"
 #include "pa_tcgen05.cuh"
 
 namespace pa {
 
-struct PrefillParams {
-  void* out;                    // [T, H, D] TO
-  const void* k_cache;          // [NB, Hkv, S, D] T
-  const void* v_cache;
-  const int32_t* block_tables;  // [B, MB]
-  const int32_t* seq_lens;      // [B] tokens in the cache, new ones included
-  const int32_t* q_start;       // [B + 1] first query row of each request
-  float scale_log2;             // scale * log2(e)
-  int MB, B, H, Hkv, NB, T, max_q_len;
-};
 
 template <int D, bool LO>
 struct PrefillTiling {

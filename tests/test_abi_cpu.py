@@ -78,6 +78,11 @@ def test_workspace_and_plan(lib):
     assert binding.pa_decode_plan(64, 40, 128, 16, 2048) == (512, 4)
     assert binding.pa_decode_plan(64, 40, 128, 16, 2048, partition=-1) == (0, 1)
     assert binding.pa_decode_plan(64, 40, 128, 16, 2048, partition=256) == (256, 8)
+    # small grids: partitions halve while the grid has fewer CTAs than SMs (148
+    # without a device): one request of 1332 tokens on 32 heads -> 256 x 6
+    assert binding.pa_decode_plan(1, 32, 128, 16, 1332) == (256, 6)
+    assert binding.pa_decode_plan(1, 1, 128, 16, 8192) == (64, 128)
+    assert binding.pa_decode_plan(1, 32, 128, 8, 100) == (64, 2)
     n = 64 * 40 * 4
     want = ((n * 8 + 255) // 256) * 256 + n * 128 * 4
     assert binding.pa_decode_workspace_bytes(64, 40, 128, 16, 2048) == want
@@ -191,3 +196,37 @@ def test_gqa_rejects_heads_not_a_multiple(lib):
     out, out_dt, q, k, v, bt, MB, sl, scale, B, H, D, S, NB, dt, part, msl, ws, wsb, st = args
     assert lib.pa_decode_gqa(out, out_dt, q, NULL, NULL, k, v, bt, MB, sl, scale, B, H, 4, D, S,
                              NB, dt, part, msl, ws, wsb, st) == binding.PA_ERR_INVALID
+
+
+def noalloc_args(**kw):
+    """pa_decode_noalloc's arguments: pa_decode's without the workspace."""
+    a = decode_args(**kw)
+    return a[:17] + [a[19]]
+
+
+@pytest.mark.parametrize("bad", [
+    dict(D=96), dict(S=4), dict(dt=binding.PA_F32), dict(q=NULL), dict(out=NULL), dict(bt=NULL),
+    dict(MB=0), dict(H=0), dict(B=70000), dict(partition=24), dict(scale=float("nan")),
+    dict(max_seq_len=8 * 16 + 1),
+    # bad arguments whose split would also be far larger than the static array:
+    # the argument check comes first, so these are PA_ERR_INVALID, not PA_ERR_OOM
+    dict(B=64, H=40, MB=8192, max_seq_len=8192 * 16 + 1, partition=512),
+    dict(B=64, H=40, MB=8192, max_seq_len=131072, partition=512, q=NULL),
+    dict(B=64, H=70000, MB=8192, max_seq_len=131072, partition=512),
+])
+def test_noalloc_rejects_bad_arguments_before_the_size_check(lib, bad):
+    assert lib.pa_decode_noalloc(*noalloc_args(**bad)) == binding.PA_ERR_INVALID
+
+
+def test_noalloc_size_check_and_exported_limit(lib):
+    limit = binding.pa_noalloc_scratch_bytes()
+    # the header's #define and the library agree
+    text = open(os.path.join(ROOT, "include", "pagedattn.h")).read()
+    m = re.search(r"#define PA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and limit == int(m.group(1)) << int(m.group(2))
+    # a valid call whose split needs more than the array is PA_ERR_OOM
+    big = dict(B=64, H=40, MB=8192, max_seq_len=131072, partition=512)
+    need = binding.pa_decode_workspace_bytes(64, 40, 128, 16, 131072, 512)
+    assert need > limit
+    assert lib.pa_decode_noalloc(*noalloc_args(**big)) == binding.PA_ERR_OOM
+    assert lib.pa_decode_noalloc(*noalloc_args(B=0, q=NULL, out=NULL)) == binding.PA_OK

@@ -84,7 +84,8 @@ def run_fp8(case, kc8, vc8, out_dt=torch.float32, partition=0, k_scale=0.05, v_s
     return out
 
 
-@pytest.mark.parametrize("D,S", [(64, 8), (128, 16), (128, 32), (256, 16)])
+@pytest.mark.parametrize("D,S", [(64, 8), (64, 16), (64, 32), (128, 8), (128, 16), (128, 32),
+                                 (256, 8), (256, 16), (256, 32)])
 @pytest.mark.parametrize("partition", [0, -1])
 def test_decode_fp8_small(D, S, partition):
     lens = [0, 1, S - 1, S, 3 * S + 5, 700]
@@ -136,3 +137,36 @@ def test_decode_fp8_llama13b_shape_sampled():
     got = torch.stack([out[i, h] for i, h in pairs]).cpu().numpy()
     assert_parity(got, want, "fp8 13B shape")
     assert bool(torch.isfinite(out).all())
+
+
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("q_mag", [1e-3, 1.0, 3e3])
+def test_decode_fp8_query_magnitude(D, q_mag):
+    """Tiny, unit and large queries all match the oracle (a 3e3 query times
+    codes up to 448 would overflow an f16 product), including a split into
+    32-token partitions."""
+    lens = [5, 40, 333]
+    case, kc8, vc8 = fp8_case(lens, H=2, D=D, S=16, in_dt=torch.bfloat16, seed=7)
+    case.q.mul_(q_mag)
+    for partition in (0, 32):
+        out = run_fp8(case, kc8, vc8, partition=partition)
+        want = ofp8.paged_decode_fp8(case.q.cpu(), kc8.cpu(), vc8.cpu(), 0.05, 0.08,
+                                     case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
+        assert_parity(out.cpu().numpy(), want, f"fp8 D={D} |q|~{q_mag} p={partition}")
+
+
+def test_decode_fp8_bad_block_id_is_skipped_and_flagged():
+    """A table entry outside the pool is never loaded: the kernel flags it and
+    leaves that block's tokens out; the other requests are unaffected."""
+    case, kc8, vc8 = fp8_case([64, 48], H=2, D=128, S=16, in_dt=torch.bfloat16, seed=9)
+    want = ofp8.paged_decode_fp8(case.q.cpu(), kc8.cpu(), vc8.cpu(), 0.05, 0.08,
+                                 case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
+    bt = case.block_tables.clone()
+    bt[0, 1] = kc8.shape[0] + 7
+    B, H, D = case.q.shape
+    out = torch.empty((B, H, D), dtype=torch.float32, device=DEV)
+    binding.pa_decode_fp8(out, case.q, kc8, vc8, 0.05, 0.08, bt, case.seq_lens, case.scale, 64,
+                          partition=-1)
+    assert binding.pa_get_device_error() & binding.PA_DEVERR_BLOCK_ID
+    assert_parity(out[1:].cpu().numpy(), want[1:], "fp8 neighbour of a bad id")
+    assert bool(torch.isfinite(out[0]).all())

@@ -65,7 +65,7 @@ def test_long_context_reduced():
     case = workloads.long_context_decode(seed=1, device=DEV, batch=2, lo=32768, hi=40000, H=4)
     out, _ = run_decode(case)
     P, NP = binding.pa_decode_plan(2, 4, 128, 16, max(case.seq_lens_host))
-    assert NP > 1 and P % 16 == 0  # split (a small grid gets partitions below 512 tokens)
+    assert NP > 1 and P % 16 == 0  # split
     assert_parity(out.cpu().numpy(), oracle_full(case), "long context reduced")
 
 
@@ -77,4 +77,40 @@ def test_long_context_full_size_sampled():
     pairs = sample_pairs(case, 16)
     got = np.stack([out[i, h].cpu().numpy() for i, h in pairs])
     assert_parity(got, oracle_pairs(case, pairs), "long context full size")
+    assert binding.pa_get_device_error() == 0
+
+
+@pytest.mark.parametrize("fill", ["zeros", "ones", "random", "nan"])
+def test_any_workspace_contents(fill):
+    """The result does not depend on what the workspace held before (every
+    partial the merge reads is written by the same call), and one workspace
+    serves calls of other partition sizes and of a grouped-query shape."""
+    case = workloads.llama13b_decode(seed=3, device=DEV, batch=6)
+    B, H, D = case.q.shape
+    S, maxlen = 16, max(case.seq_lens_host)
+    want = oracle_full(case)
+    gq = workloads.llama70b_decode(seed=4, device=DEV, batch=3)
+    Bg, Hg, _ = gq.q.shape
+    gmax = max(gq.seq_lens_host)
+    size = max([binding.pa_decode_workspace_bytes(B, H, D, S, maxlen, P) for P in (16, 64, 512)]
+               + [binding.pa_decode_workspace_bytes(Bg, Hg, D, S, gmax, 64)])
+    ws = torch.empty(size, dtype=torch.uint8, device=DEV)
+    if fill == "zeros":
+        ws.zero_()
+    elif fill == "ones":
+        ws.fill_(0xFF)
+    elif fill == "random":
+        ws.copy_(torch.randint(0, 256, (size,), dtype=torch.uint8, generator=torch.Generator()
+                               .manual_seed(5)).to(DEV))
+    else:
+        ws.view(torch.float32)[: size // 4].fill_(float("nan"))
+    for P in (64, 16, 512, 64):
+        out = torch.empty((B, H, D), dtype=torch.float32, device=DEV)
+        binding.pa_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables,
+                          case.seq_lens, case.scale, maxlen, partition=P, workspace=ws)
+        assert_parity(out.cpu().numpy(), want, f"{fill} P={P}")
+    out = torch.empty((Bg, Hg, D), dtype=torch.float32, device=DEV)
+    binding.pa_decode_gqa(out, gq.q, gq.k_cache, gq.v_cache, gq.block_tables, gq.seq_lens,
+                          gq.scale, gmax, partition=64, workspace=ws)
+    assert_parity(out.cpu().numpy(), oracle_full(gq), f"{fill} grouped heads")
     assert binding.pa_get_device_error() == 0

@@ -39,7 +39,7 @@ def test_noalloc_matches_pa_decode_twice_in_a_row(partition):
         B, H, D = case.q.shape
         S = case.k_cache.shape[2]
         need = binding.pa_decode_workspace_bytes(B, H, D, S, max(case.seq_lens_host), partition)
-        assert 0 < need <= binding.PA_NOALLOC_SCRATCH_BYTES  # the split really uses the array
+        assert 0 < need <= binding.pa_noalloc_scratch_bytes()  # the split really uses the array
         want, _ = run_decode(case, partition=partition)
         got = noalloc(case, partition)
         torch.cuda.synchronize()
@@ -53,7 +53,7 @@ def test_noalloc_rejects_a_split_larger_than_the_array():
     host with PA_ERR_OOM before anything is launched."""
     B, H, D, S = 64, 40, 128, 16
     big = binding.pa_decode_workspace_bytes(B, H, D, S, 131072, 512)
-    assert big > binding.PA_NOALLOC_SCRATCH_BYTES
+    assert big > binding.pa_noalloc_scratch_bytes()
     q = torch.zeros((B, H, D), dtype=torch.bfloat16, device=DEV)
     out = torch.empty((B, H, D), dtype=torch.float32, device=DEV)
     tables = torch.full((B, 8192), -1, dtype=torch.int32, device=DEV)
