@@ -560,6 +560,10 @@ def run_shape_workloads(args):
     # the oracle is timed on one case of each configuration (the long-context
     # case, one mid-size point of the sweep)
     cpu_cases = {"long_context", "S16_D128_B32_bf16"}
+    if args.case:
+        cases = [(n, m) for n, m in cases if n == args.case]
+        if not cases:
+            raise SystemExit(f"no case named {args.case}")
     rows = []
     for name, make in cases:
         case = make()
@@ -619,7 +623,10 @@ def run_append_workload(args):
     with L2 flushed (a 256 MB write) before each."""
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    case = workloads.prefill_append(seed=args.seed, device=device)
+    if args.workload == "prefill_append_small":  # a profiling-sized case: 4 x 4096 tokens
+        case = workloads.prefill_append(seed=args.seed, device=device, n_req=4, lo=4096, hi=4096)
+    else:
+        case = workloads.prefill_append(seed=args.seed, device=device)
     T, Hc, Dc = case.k.shape
     NB, _, Sc, _ = case.k_cache.shape
     alloc = binding.BlockAllocator(NB, Sc, initial_order=case.block_order)
@@ -649,7 +656,9 @@ def run_append_workload(args):
     ms = statistics.median(times)
     peak, peak_kind = measured_peak()
     gbs = nbytes / (ms / 1e3) / 1e9
-    print(json.dumps({"workload": APPEND_WORKLOAD, "tokens": T, "ms": round(ms, 4),
+    print(json.dumps({"workload": APPEND_WORKLOAD if args.workload == "prefill_append" else
+                      "prefill-scale append, profiling size: 4 requests of 4096 tokens",
+                      "tokens": T, "ms": round(ms, 4),
                       "gb_s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 3),
                       "peak": peak, "peak_kind": peak_kind, "bytes_per_call": nbytes,
                       "kernel": "kv_append_kernel (one launch)", "calls": args.steps,
@@ -984,10 +993,12 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="with --workload sweep: time only this case (e.g. S16_D128_B1_bf16)")
     ap.add_argument("--workload", default="llama13b",
                     choices=["llama13b", "long_context", "sweep", "llama70b", "llama13b_fp8",
                              "prompt_prefill", "prompt_prefill_small", "worked_example",
-                             "prefill_append", "batching"],
+                             "prefill_append", "prefill_append_small", "batching"],
                     help="llama13b: the headline step (default); the others time decode-only "
                          "calls of the long-context, shape-sweep and LLaMA-2-70B-shaped "
                          "grouped-query configurations, paged prefill attention over "
@@ -1004,7 +1015,7 @@ def main():
         run_prefill_workload(args)
         return
     extra = {"worked_example": run_worked_example, "prefill_append": run_append_workload,
-             "batching": run_batching_workload}
+             "prefill_append_small": run_append_workload, "batching": run_batching_workload}
     if args.workload in extra:
         binding.lib()
         extra[args.workload](args)

@@ -170,13 +170,39 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
   const int wt1 = min(we * S, L);
   const int nunits = wt1 > wt0 ? (wt1 - wt0 + CR - 1) / CR : 0;
 
-  // q fragment, pre-scaled so that scores come out in base-2 units.
+  // q fragment, pre-scaled so that scores come out in base-2 units. E4M3 caches
+  // take q as f16 pairs instead, exactly scaled by 2^qe so that its largest
+  // element is below 2^15 (qe undone on the score): the dot products then run
+  // as fp32 accumulations of exact f16 x f16 products straight from the
+  // codes' f16 conversion.
   float qf[EPL];
+  uint32_t qh[EB == 1 ? EPL / 2 : 1];
+  float score_scale = 1.f;
   {
     const T* qp = static_cast<const T*>(p.q) + (static_cast<int64_t>(i) * p.H + h) * D + pl * EPL;
     load_row<T, EPL>(qp, qf);
+    if constexpr (EB == 1) {
+      float mx = 0.f;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) qf[e] *= p.q_scale;
+      for (int e = 0; e < EPL; ++e) mx = fmaxf(mx, fabsf(qf[e]));
+#pragma unroll
+      for (int off = 1; off < LPR; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
+      int qe = 0;
+      if (mx > 0.f && mx < INFINITY) {
+        frexpf(mx, &qe);                      // mx = f * 2^qe, f in [0.5, 1)
+        qe = max(-100, min(100, 15 - qe));    // max |q| * 2^qe < 2^15
+      }
+      const float up = ldexpf(1.f, qe);
+      score_scale = p.q_scale * ldexpf(1.f, -qe);
+#pragma unroll
+      for (int e = 0; e < EPL; e += 2) {
+        const __half2 q2 = __floats2half2_rn(qf[e] * up, qf[e + 1] * up);
+        qh[e / 2] = *reinterpret_cast<const uint32_t*>(&q2);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) qf[e] *= p.q_scale;
+    }
   }
 
   uint64_t* bar = bars + w * NS;
@@ -282,22 +308,24 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
       float dot[NV];
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        float kf[EPL];
-        load_cache_row<TC, EPL>(ks + ((v * RPW + g) * D + pl * EPL) * EB, kf);
-        if constexpr (EB == 1) {  // twice the elements per byte: packed pairs
-          float2 a2 = make_float2(0.f, 0.f);
+        if constexpr (EB == 1) {  // f16 codes x f16 q, fp32 sums
+          uint32_t kh[EPL / 2];
+          e4m3x16_to_h2(ks + ((v * RPW + g) * D + pl * EPL), kh);
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-          for (int e = 0; e < EPL; e += 2)
-            a2 = ffma2(make_float2(qf[e], qf[e + 1]), make_float2(kf[e], kf[e + 1]), a2);
-          dot[v] = a2.x + a2.y;
+          for (int e = 0; e < EPL / 2; ++e) fma_f16pair_f32(qh[e], kh[e], a0, a1);
+          dot[v] = a0 + a1;
         } else {
+          float kf[EPL];
+          load_cache_row<TC, EPL>(ks + ((v * RPW + g) * D + pl * EPL) * EB, kf);
           float a = 0.f;
 #pragma unroll
           for (int e = 0; e < EPL; ++e) a = fmaf(qf[e], kf[e], a);
           dot[v] = a;
         }
       }
-      const float score = transpose_reduce<NV, LPR>(dot, lane);
+      float score = transpose_reduce<NV, LPR>(dot, lane);
+      if constexpr (EB == 1) score *= score_scale;
       const bool valid = my_row < nvalid;
       const float sc = valid ? score : -INFINITY;
       float mb = sc;
@@ -315,17 +343,16 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
           const float pv = __shfl_sync(kFullMask, pr, g * LPR + v * DUP);
-          float vf[EPL];
-          load_cache_row<TC, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * EB, vf);
-          if constexpr (EB == 1) {
+          if constexpr (EB == 1) {  // the weight as f16 (2^-12 relative), fp32 sums
+            uint32_t vh[EPL / 2];
+            e4m3x16_to_h2(vs + ((v * RPW + g) * D + pl * EPL), vh);
+            const __half2 p2 = __float2half2_rn(pv);
+            const uint32_t ph = *reinterpret_cast<const uint32_t*>(&p2);
 #pragma unroll
-            for (int e = 0; e < EPL; e += 2) {
-              const float2 r = ffma2(make_float2(pv, pv), make_float2(vf[e], vf[e + 1]),
-                                     make_float2(acc[e], acc[e + 1]));
-              acc[e] = r.x;
-              acc[e + 1] = r.y;
-            }
+            for (int e = 0; e < EPL / 2; ++e) fma_f16pair_f32(ph, vh[e], acc[2 * e], acc[2 * e + 1]);
           } else {
+            float vf[EPL];
+            load_cache_row<TC, EPL>(vs + ((v * RPW + g) * D + pl * EPL) * EB, vf);
 #pragma unroll
             for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pv, vf[e], acc[e]);
           }

@@ -231,6 +231,30 @@ __device__ __forceinline__ uint16_t float2_to_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// 16 E4M3 codes (one 16-byte fragment) -> 8 f16 pairs, exactly (E4M3 values are
+// f16 values).
+__device__ __forceinline__ void e4m3x16_to_h2(const void* p, uint32_t (&h)[8]) {
+  const uint4 x = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * k]) : "h"(static_cast<uint16_t>(w[k] & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * k + 1]) : "h"(static_cast<uint16_t>(w[k] >> 16)));
+  }
+}
+
+// c0 += lo(a) * lo(b), c1 += hi(a) * hi(b): fp32 accumulation of products of
+// f16 values (the products are exact in fp32), one mixed-precision FMA each.
+__device__ __forceinline__ void fma_f16pair_f32(uint32_t a, uint32_t b, float& c0, float& c1) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %2;\n\t"
+      "mov.b32 {bl, bh}, %3;\n\t"
+      "fma.rn.f32.f16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.f16 %1, ah, bh, %1;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "r"(a), "r"(b));
+}
+
 // One row fragment of the cache (16 bytes in shared memory) -> fp32 registers:
 // 8 elements of a 16-bit cache, or 16 of an E4M3 cache.
 template <typename TC, int EPL>

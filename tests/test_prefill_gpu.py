@@ -182,3 +182,40 @@ def test_chunked_prefill_large_sampled(dt, Hkv):
     got = torch.stack([out[qs[i] + j, h] for i, j, h in picks]).cpu().numpy()
     assert_parity(got, want, f"chunked prefill {dt} Hkv={Hkv}")
     assert bool(torch.isfinite(out).all())
+
+
+@pytest.mark.parametrize("v_scale", [1.0, 2.0 ** 20, 2.0 ** -8, 2.0 ** 30, 2.0 ** -14])
+def test_bf16_value_magnitudes(v_scale):
+    """bf16 caches with V from 2^-14 to 2^30 times N(0, 1): every scale matches
+    the oracle relative to the scale of V (the output is linear in V),
+    including context, ragged tiles and a key tile past the end."""
+    pc = workloads.prefill_case([0, 37, 300], [140, 200, 66], H=2, D=128, S=16,
+                                dtype=torch.bfloat16, seed=11, device=DEV)
+    c = pc.cache
+    c.v_cache.copy_((c.v_cache.float() * v_scale).to(torch.bfloat16))
+    out = run_prefill(pc)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    want = oracle_prefill_full(pc)
+    assert_parity(out.cpu().numpy() / v_scale, want / v_scale, f"V x {v_scale}")
+
+
+def test_bf16_mixed_tile_modes():
+    """One request whose V tiles (128 tokens each) alternate between 2^18 and
+    2^28 times N(0, 1), so that rows mix key tiles of very different
+    magnitude."""
+    pc = workloads.prefill_case([0], [600], H=2, D=128, S=16, dtype=torch.bfloat16, seed=12,
+                                device=DEV)
+    c = pc.cache
+    S = c.k_cache.shape[2]
+    table = c.tables_host[0]
+    c.v_cache.copy_((c.v_cache.float() * 2.0 ** 18).to(torch.bfloat16))
+    for j in range(0, 600, 256):  # tokens j .. j + 127 of every other key tile: x 2^10 more
+        for blk in table[j // S:(j + 128) // S]:
+            c.v_cache[blk] = (c.v_cache[blk].float() * 2.0 ** 10).to(torch.bfloat16)
+    out = run_prefill(pc)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    want = oracle_prefill_full(pc)
+    scale = float(np.abs(want).max())
+    assert_parity(out.cpu().numpy() / scale, want / scale, "mixed tile modes")
