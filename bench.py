@@ -712,7 +712,7 @@ def run_batching_workload(args):
     def run(fused, graph, keep=False):
         loop = make_loop()
         cb = ContinuousBatching(loop, device, max_steps=64 + W, poison=False, fused=fused,
-                                graph=graph)
+                                graph=graph, keep_records=keep)
         for k in range(W):
             cb.step(k)
         torch.cuda.synchronize()

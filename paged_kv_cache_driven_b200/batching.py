@@ -34,24 +34,32 @@ maximum; the eager path does the same when ``fixed_plan`` is set, so the two
 give the same bits.
 """
 
+import ctypes
 import math
 import time
 
+import numpy as np
 import torch
 
 from . import binding
 
 
 class StagingRing:
-    """Pinned host buffers for each step's slots, block tables and lengths, ``depth``
-    sets deep. The host fills set k while the copies of earlier sets may still be
-    in flight; before a set is refilled, the event recorded after its copies is
-    waited on, so the host never rewrites memory a pending copy still reads."""
+    """Pinned host buffers for each step's slots, block tables and lengths (and
+    the slot mappings of the step's admitted prompts), ``depth`` sets deep. The
+    host fills set k while the copies of earlier sets may still be in flight;
+    before a set is refilled, the event recorded after its copies is waited on,
+    so the host never rewrites memory a pending copy still reads. (A copy from
+    pageable memory would instead make the host wait for the whole stream.)"""
+
+    PROMPT_SLOTS = 1 << 16  # admitted prompt tokens per step that fit the pinned slab
 
     def __init__(self, n_seq, max_blocks, n_new=1, depth=2):
         self.sets = [dict(slots=torch.empty(n_seq * n_new, dtype=torch.int64).pin_memory(),
                           tables=torch.empty((n_seq, max_blocks), dtype=torch.int32).pin_memory(),
-                          lens=torch.empty(n_seq, dtype=torch.int32).pin_memory())
+                          lens=torch.empty(n_seq, dtype=torch.int32).pin_memory(),
+                          prompt=torch.empty(self.PROMPT_SLOTS, dtype=torch.int64).pin_memory(),
+                          prompt_used=0)
                      for _ in range(depth)]
         self.events = [None] * depth
         self.k = 0
@@ -60,6 +68,7 @@ class StagingRing:
         i = self.k % len(self.sets)
         if self.events[i] is not None:
             self.events[i].synchronize()
+        self.sets[i]["prompt_used"] = 0
         return self.sets[i]
 
     def release(self, stream=None):
@@ -71,7 +80,7 @@ class StagingRing:
 
 class ContinuousBatching:
     def __init__(self, loop, device, max_steps=64, poison=True, fused=False, graph=False,
-                 fixed_plan=False):
+                 fixed_plan=False, keep_records=True):
         self.loop = loop
         self.fused = fused  # pa_decode_append instead of pa_kv_append + pa_decode
         self.graph = graph
@@ -88,7 +97,10 @@ class ContinuousBatching:
         self.alloc = binding.BlockAllocator(NB, S, initial_order=loop.block_order)
         self.scale = 1.0 / math.sqrt(D)
         self.serial = 0
-        self.slots = []  # per batch slot: [seq_id, remaining budget]
+        self.keep_records = keep_records  # step records carry copies of slots, tables, lengths
+        self.sid = []  # per batch slot: its sequence id
+        self.ids_c = (ctypes.c_int64 * B)()  # the same, as the allocator takes it
+        self.budget = np.zeros(B, dtype=np.int64)  # per batch slot: tokens left to decode
         self.staging = StagingRing(B, self.MB)
         self.d_slots = torch.empty(B, dtype=torch.int64, device=device)
         self.d_tables = torch.empty((B, self.MB), dtype=torch.int32, device=device)
@@ -104,25 +116,39 @@ class ContinuousBatching:
         self.host_s = 0.0  # seconds spent in allocator calls (grow, slots, tables, free)
         self.prompt_slots = []  # device slot mappings of the admissions since the last step
         for b in range(B):
-            self.slots.append(self._admit(loop.initial_lens[b], loop.budgets[b]))
+            self._admit(b, loop.initial_lens[b], loop.budgets[b])
 
-    def _admit(self, prompt_len, budget):
-        """Creates a request, allocates its prompt blocks and appends its prompt K/V."""
+    def _admit(self, b, prompt_len, budget, h=None):
+        """Creates a request in batch slot b, allocates its prompt blocks and
+        appends its prompt K/V. During a step (h: the step's staging set) the
+        slot mapping goes up from the set's pinned slab, asynchronously."""
         sid = self.serial
         self.serial += 1
+        pinned = h is not None and h["prompt_used"] + prompt_len <= StagingRing.PROMPT_SLOTS
         t = time.perf_counter()
         self.alloc.pa_seq_grow(sid, prompt_len)
-        h_slots = self.alloc.pa_build_slot_mapping([sid], [0], [prompt_len])
+        if pinned:
+            off = h["prompt_used"]
+            h_slots = self.alloc.pa_build_slot_mapping(
+                [sid], [0], [prompt_len], out=h["prompt"][off:off + prompt_len])
+            h["prompt_used"] = off + prompt_len
+        else:
+            h_slots = self.alloc.pa_build_slot_mapping([sid], [0], [prompt_len])
         self.host_s += time.perf_counter() - t
         k, v = self.loop.prompt_kv(sid, prompt_len, self.device)
-        slots = h_slots.to(self.device)
+        slots = h_slots.to(self.device, non_blocking=pinned)
         binding.pa_kv_append(k, v, slots, self.k_cache, self.v_cache)
         self.prompt_slots.append(slots)
         self.events.append(("admit", sid, prompt_len))
-        return [sid, max(1, int(budget))]
+        if b < len(self.sid):
+            self.sid[b] = sid
+        else:
+            self.sid.append(sid)
+        self.ids_c[b] = sid
+        self.budget[b] = max(1, int(budget))
 
     def seq_ids(self):
-        return [s[0] for s in self.slots]
+        return list(self.sid)
 
     def _device_step(self, h, max_len):
         """Uploads from staging set h, then append + decode (eager or under capture)."""
@@ -147,7 +173,7 @@ class ContinuousBatching:
         host0 = self.host_s
         self.prompt_slots = []
         t = time.perf_counter()
-        self.alloc.pa_prepare_step(ids, 1, self.MB, h["slots"], h["tables"], h["lens"])
+        self.alloc.pa_prepare_step(self.ids_c, 1, self.MB, h["slots"], h["tables"], h["lens"])
         self.host_s += time.perf_counter() - t
         q, k, v = self.loop.token_kv(step_idx, self.B, self.device)
         self._qkv = (q, k, v)
@@ -165,22 +191,24 @@ class ContinuousBatching:
                 with torch.cuda.graph(g):
                     self._device_step(h, max_len)
                 self.graphs[set_idx] = g
+        if self.keep_records:
+            record = dict(ids=ids, slots=h["slots"].clone(), lens=h["lens"].clone(),
+                          tables=h["tables"].clone(), q=q, k=k, v=v, out=self.out, retired=[],
+                          admitted=[])
+        else:
+            record = dict(ids=ids, retired=[], admitted=[])
+        self.budget -= 1
+        for b in np.flatnonzero(self.budget <= 0).tolist():  # batch slots in index order
+            old = self.sid[b]
+            t = time.perf_counter()
+            self.alloc.pa_seq_free(old)
+            self.host_s += time.perf_counter() - t
+            self.events.append(("retire", old, 0))
+            L, budget = self.loop.arrival()
+            self._admit(b, L, budget, h)
+            record["retired"].append(old)
+            record["admitted"].append((self.sid[b], L, int(self.budget[b])))
         self.staging.release()
-        record = dict(ids=ids, slots=h["slots"].clone(), lens=h["lens"].clone(),
-                      tables=h["tables"].clone(), q=q, k=k, v=v, out=self.out, retired=[],
-                      admitted=[])
-        for b in range(self.B):
-            self.slots[b][1] -= 1
-            if self.slots[b][1] <= 0:
-                old = self.slots[b][0]
-                t = time.perf_counter()
-                self.alloc.pa_seq_free(old)
-                self.host_s += time.perf_counter() - t
-                self.events.append(("retire", old, 0))
-                L, budget = self.loop.arrival()
-                self.slots[b] = self._admit(L, budget)
-                record["retired"].append(old)
-                record["admitted"].append((self.slots[b][0], L, self.slots[b][1]))
         record["host_s"] = self.host_s - host0
         record["prompt_slots"] = self.prompt_slots
         return record
