@@ -173,9 +173,9 @@ def measured_peak():
 
 
 def kernel_source_hash():
-    """Hash of the headline call's kernels (the partition pass with its fused merge,
-    with the device helpers they use), comments and blank lines removed, so a
-    profile stays attached to the kernel code it measured and nothing else."""
+    """Hash of the headline call's kernels (the partition pass and the split-KV
+    merge, with the device helpers they use), comments and blank lines removed,
+    so a profile stays attached to the kernel code it measured and nothing else."""
     import re
     h = hashlib.sha256()
     for f in ("pa_decode.cuh", "pa_device.cuh"):
@@ -460,18 +460,40 @@ def decode_bytes_case(case):
                for L in case.seq_lens_host) + 4 * B
 
 
+L2_FLUSHED = "flushed before each call: 256 MB write, then 256 MB read"
+
+
+class L2Flush:
+    """Empties L2 (126 MB) before a timed call: a 256 MB write, then a 256 MB
+    read. The read evicts the write's dirty lines, so L2 holds neither the
+    call's inputs nor dirty lines whose write-back the timed call would pay for
+    (after a write alone, a call that reads more than L2 writes about 126 MB
+    back to HBM while it runs)."""
+
+    def __init__(self, device):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=device)
+        self.sink = torch.empty((), dtype=torch.float32, device=device)
+        self.k = 0
+
+    def __call__(self):
+        self.k += 1
+        self.w.fill_(self.k & 0xff)
+        torch.sum(self.r, dim=0, out=self.sink)
+
+
 def time_decode_case(case, iters, warmup, partition=0):
-    """Median event-timed pa_decode call with L2 flushed (a 256 MB write) before each."""
+    """Median event-timed pa_decode call with L2 flushed (L2Flush) before each."""
     B, Hc, Dc = case.q.shape
     Sc = case.k_cache.shape[2]
     maxlen = max(case.seq_lens_host)
     out = torch.empty((B, Hc, Dc), dtype=case.q.dtype, device=case.q.device)
     wsb = binding.pa_decode_workspace_bytes(B, Hc, Dc, Sc, maxlen, partition)
     ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=case.q.device)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=case.q.device)
+    flush = L2Flush(case.q.device)
     times = []
     for k in range(warmup + iters):
-        flush.fill_(k & 0xff)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         if case.k_cache.shape[1] != Hc:
@@ -510,10 +532,10 @@ def time_decode_fp8(seed, iters, warmup):
     out = torch.empty((B, Hc, Dc), dtype=DTYPE, device=device)
     wsb = binding.pa_decode_workspace_bytes(B, Hc, Dc, Sc, maxlen, 0)
     ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     times = []
     for k in range(warmup + iters):
-        flush.fill_(k & 0xff)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         binding.pa_decode_fp8(out, case.q, kc8, vc8, 0.05, 0.08, case.block_tables,
@@ -527,6 +549,37 @@ def time_decode_fp8(seed, iters, warmup):
     nbytes = sum(Hc * (2 * L * Dc + 2 * Dc * 2) + 4 * (-(-L // Sc)) for L in case.seq_lens_host) \
         + 4 * B
     return statistics.median(times), nbytes, binding.pa_decode_plan(B, Hc, Dc, Sc, maxlen, 0)
+
+
+def latency_floors(device, iters, warmup):
+    """The small-batch floor, timed like the sweep's calls (L2 flushed, events
+    around the call): a launch of a one-element fill (a kernel that does
+    nothing measurable), and a decode of a single CTA (one request of 16
+    tokens, one head, head_dim 128: one length, one table entry and one 8 KB
+    K/V block to load)."""
+    flush = L2Flush(device)
+    x = torch.empty(1, dtype=torch.float32, device=device)
+    case = workloads.decode_case([16], H=1, D=128, S=16, dtype=torch.bfloat16, seed=0,
+                                 device=device)
+    out = torch.empty((1, 1, 128), dtype=torch.bfloat16, device=device)
+
+    def med(fn):
+        ts = []
+        for k in range(warmup + iters):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if k >= warmup:
+                ts.append(a.elapsed_time(b) * 1e3)
+        return round(statistics.median(ts), 2)
+
+    return {"empty_launch": med(lambda: x.fill_(0.0)),
+            "single_cta_decode": med(lambda: binding.pa_decode(
+                out, case.q, case.k_cache, case.v_cache, case.block_tables, case.seq_lens,
+                case.scale, 16, partition=0, workspace=None))}
 
 
 def run_shape_workloads(args):
@@ -543,7 +596,8 @@ def run_shape_workloads(args):
         print(json.dumps({"workload": "llama13b_fp8_e4m3_cache", "ms": round(ms, 4),
                           "gb_s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 3),
                           "kv_bytes": nbytes, "tok_s_layer": round(64 / (ms / 1e3), 1),
-                          "partition": {"tokens": plan[0], "num": plan[1]}}), flush=True)
+                          "partition": {"tokens": plan[0], "num": plan[1]},
+                          "l2": L2_FLUSHED}), flush=True)
         return
     elif args.workload == "llama70b":
         cases = [("llama70b_gqa_64q_8kv", lambda: workloads.llama70b_decode(seed=args.seed,
@@ -573,7 +627,7 @@ def run_shape_workloads(args):
         row = {"workload": name, "ms": round(ms, 4), "gb_s": round(gbs, 1),
                "frac_of_peak": round(gbs / peak, 3), "kv_bytes": nbytes,
                "tok_s_layer": round(case.q.shape[0] / (ms / 1e3), 1),
-               "partition": {"tokens": plan[0], "num": plan[1]}}
+               "partition": {"tokens": plan[0], "num": plan[1]}, "l2": L2_FLUSHED}
         if name in cpu_cases and not args.no_cpu_baseline:
             row["cpu_baseline"] = cpu_baseline_legs(case.q, case.k_cache, case.v_cache,
                                                     case.tables_host, case.seq_lens_host,
@@ -583,8 +637,9 @@ def run_shape_workloads(args):
         del case
         torch.cuda.empty_cache()
     big = [r for r in rows if r["kv_bytes"] > 1 << 30]
+    floors = latency_floors(device, args.steps, args.warmup) if args.workload == "sweep" else None
     summary = {"metric": METRIC + " (decode only)", "workload": args.workload,
-               "peak": peak, "peak_kind": peak_kind, "cases": len(rows),
+               "peak": peak, "peak_kind": peak_kind, "cases": len(rows), "latency_floors_us": floors,
                "min_frac_over_1GB": min((r["frac_of_peak"] for r in big), default=None),
                "median_frac_over_1GB": statistics.median([r["frac_of_peak"] for r in big])
                if big else None}
@@ -593,16 +648,17 @@ def run_shape_workloads(args):
 
 def run_worked_example(args):
     """--workload worked_example: the pages' four requests of 6/50/8/100 tokens
-    (4 heads, head_dim 64, fp16). The whole cache is 256 KB, so it sits in L2:
-    the GPU time is a launch-latency figure, not a bandwidth one. The line's
-    point is the oracle leg on the same inputs (all threads and one)."""
+    (4 heads, head_dim 64, fp16). The whole cache is 256 KB: even with L2
+    flushed before each call the GPU time is a launch- and latency-bound
+    figure, not a bandwidth one. The line's point is the oracle leg on the same
+    inputs (all threads and one)."""
     device = torch.device("cuda", 0)
     case = workloads.worked_example(seed=args.seed, device=device)
     ms, plan = time_decode_case(case, args.steps, args.warmup)
     nbytes = decode_bytes_case(case)
     row = {"workload": "worked_example_6_50_8_100", "ms": round(ms, 4),
            "gb_s": round(nbytes / (ms / 1e3) / 1e9, 2), "kv_bytes": nbytes,
-           "note": "L2-resident (256 KB cache); launch-bound",
+           "note": "256 KB cache; launch- and latency-bound", "l2": L2_FLUSHED,
            "partition": {"tokens": plan[0], "num": plan[1]}}
     if not args.no_cpu_baseline:
         row["cpu_baseline"] = cpu_baseline_legs(case.q, case.k_cache, case.v_cache,
@@ -620,7 +676,7 @@ def run_append_workload(args):
     tokens through slot_mapping (the shape sweep's append), KV GB/s against the
     measured HBM copy bandwidth. Algorithmic bytes: the new tokens' K and V read
     and written plus the int64 slots, T*H*D*e*4 + 8T. Median of event-timed calls
-    with L2 flushed (a 256 MB write) before each."""
+    with L2 flushed (L2Flush) before each."""
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     if args.workload == "prefill_append_small":  # a profiling-sized case: 4 x 4096 tokens
@@ -637,12 +693,12 @@ def run_append_workload(args):
     alloc.close()
     e = case.k.element_size()
     nbytes = T * Hc * Dc * e * 4 + 8 * T
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     times = []
     with ClockSampler(0) as clk:
         clk.mark_start()
         for k in range(args.warmup + args.steps):
-            flush.fill_(k & 0xff)
+            flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             binding.pa_kv_append(case.k, case.v, slots, case.k_cache, case.v_cache)
@@ -662,7 +718,7 @@ def run_append_workload(args):
                       "gb_s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 3),
                       "peak": peak, "peak_kind": peak_kind, "bytes_per_call": nbytes,
                       "kernel": "kv_append_kernel (one launch)", "calls": args.steps,
-                      "clocks": clk.summary()}), flush=True)
+                      "l2": L2_FLUSHED, "clocks": clk.summary()}), flush=True)
 
 
 BATCHING_WORKLOAD = "continuous batching: 40 heads, head_dim 128, block 16, bf16, batch 256, " \
@@ -1140,7 +1196,8 @@ def main():
                          "frac_of_copy_bw": round(dec_gbs / peak, 4),
                          "frac_of_nominal_8000": round(dec_gbs / 8000.0, 4),
                          "kernel": "pa_decode_append call: paged_decode_partition_kernel<APPEND> "
-                                   "(split-KV merge fused into the same launch)",
+                                   "+ splitkv_reduce_kernel (launched as a programmatic "
+                                   "dependent); timed together as one call",
                          "call_ms": round(dec_ms, 4),
                          "algorithmic_bytes_per_launch": step_bytes},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",

@@ -107,6 +107,14 @@ pa_status pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping
  *                 workspaces of their own. The library keeps no pointer to it
  *                 after the call's work ends
  * Requires 16-byte aligned q, k_cache, v_cache, out and workspace.
+ * How a split is merged: an automatic split (partition = 0) into 2, 4 or 8
+ * partitions whose grid (B * H * partitions CTAs) fits within two CTAs per SM
+ * runs as thread-block clusters, one per (request, head), and partition 0
+ * merges the others' results through distributed shared memory: the workspace
+ * is still required but left untouched. Every other split leaves per-partition
+ * results in the workspace (layout below) for a merge kernel. Both merges do
+ * the same arithmetic in the same order: the output bits do not depend on
+ * which one ran.
  * ------------------------------------------------------------------------- */
 size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, int partition);
 
@@ -114,7 +122,11 @@ size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, in
  * for these arguments on the current device; *partition_tokens = 0 and
  * *num_partitions = 1 mean a single pass with no workspace. The automatic choice
  * (partition = 0) depends on B * H and the device's SM count: call this and
- * pa_decode_workspace_bytes with the device current that pa_decode will run on. */
+ * pa_decode_workspace_bytes with the device current that pa_decode will run on.
+ * Automatic: 512-token partitions, halved (down to 64 tokens) while the grid
+ * has fewer CTAs than the device has SMs; a resulting count of 3, 5, 6 or 7 is
+ * then re-cut to the next (else the previous) power of two when that grid fits
+ * within two CTAs per SM, so that the split merges inside clusters. */
 pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partition,
                          int* partition_tokens, int* num_partitions);
 
@@ -242,7 +254,8 @@ pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k
  * one partition are written; a second kernel, launched so that it can start
  * while the first finishes, merges them by log-sum-exp ([card] "헷갈리기 쉬운
  * 구분"). Everything the merge reads is written by the same call, so the
- * workspace needs no initialisation. */
+ * workspace needs no initialisation. (A split merged inside clusters, see
+ * pa_decode, writes none of it.) */
 
 /* ---------------------------------------------------------------------------
  * Decode without any caller-provided scratch. This entry point has no

@@ -59,6 +59,10 @@ int sm_count() {
 //           heads, 1.3K tokens: 256-token partitions, 192 CTAs, are fastest for
 //           head sizes 64 to 256; 64-token ones, 672 CTAs, are 40 % slower,
 //           each CTA's fixed start and end costing more than its short stream.)
+//           A small grid then has a partition count of 3, 5, 6 or 7 rounded
+//           to a power of two (the next, else the previous; partitions re-cut
+//           evenly in whole blocks) when the grid stays within two CTAs per SM,
+//           so that its split can merge inside a cluster (cluster_merge).
 bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* NP_out) {
   if (max_seq_len < 0 || S <= 0) return false;
   int P;
@@ -75,6 +79,18 @@ bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* 
     const int64_t target = sm_count();
     const int64_t pairs = static_cast<int64_t>(B > 0 ? B : 1) * (H > 0 ? H : 1);
     while (P > 64 && (P / 2) % S == 0 && pairs * ceil_div(max_seq_len, P) < target) P /= 2;
+    const int64_t n = ceil_div(max_seq_len, P);
+    if (n > 2 && n < 8 && (n & (n - 1)) != 0) {
+      const int64_t up = n < 4 ? 4 : 8;
+      for (const int64_t c : {up, up / 2}) {
+        if (pairs * c > 2 * target) continue;
+        // c partitions of a whole number of blocks; where blocks do not divide
+        // evenly the last one or two hold no token (they only join the merge)
+        *P_out = static_cast<int>(ceil_div(ceil_div(max_seq_len, c), S) * S);
+        *NP_out = static_cast<int>(c);
+        return true;
+      }
+    }
   }
   const int64_t np = ceil_div(max_seq_len, P);
   if (np <= 1) {
@@ -86,6 +102,18 @@ bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* 
   *P_out = P;
   *NP_out = static_cast<int>(np);
   return true;
+}
+
+// Whether an automatic split of NP partitions over B x H (request, head) pairs
+// merges inside clusters instead of through the workspace and the merge
+// kernel: NP is a portable cluster size (2, 4 or 8; the cluster spans the
+// grid's x dimension, the partitions of one pair), and the grid fits within two
+// CTAs per SM, so that it is resident at once and the CTAs that wait at their
+// cluster's barrier hold no SM another CTA is queued for. Large grids keep the
+// merge kernel, which overlaps their last wave.
+bool cluster_merge(int B, int H, int NP) {
+  if (NP != 2 && NP != 4 && NP != 8) return false;
+  return static_cast<int64_t>(B) * H * NP <= 2 * static_cast<int64_t>(sm_count());
 }
 
 // Split-KV workspace: m and l [B, H, NP], then (256-byte aligned) acc [B, H, NP, D].
@@ -337,8 +365,10 @@ pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_n
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   prm.k_new = k_new;
   prm.v_new = v_new;
-  if (H != Hkv) return pa::host::launch_grouped(prm, dt, out_dt, D, S, k_new != nullptr, st);
-  return pa::host::launch_decode16(prm, dt, out_dt, D, S, k_new != nullptr, st);
+  if (H != Hkv)  // (the grouped-query kernel always merges through the workspace)
+    return pa::host::launch_grouped(prm, dt, out_dt, D, S, k_new != nullptr, st);
+  const bool cluster = partition == 0 && cluster_merge(B, H, prm.NP);
+  return pa::host::launch_decode16(prm, dt, out_dt, D, S, k_new != nullptr, cluster, st);
 }
 
 }  // namespace
@@ -475,7 +505,9 @@ pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt
     prm.NP = 1;
     prm.L_cap = static_cast<int>(L_max);
   }
-  return pa::host::launch_decode_fp8(prm, q_dt, out_dt, D, S, static_cast<cudaStream_t>(stream));
+  const bool cluster = partition == 0 && cluster_merge(B, H, prm.NP);
+  return pa::host::launch_decode_fp8(prm, q_dt, out_dt, D, S, cluster,
+                                     static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_get_device_error(void* stream, uint32_t* flags) {

@@ -70,6 +70,10 @@ struct DecodeTiling {
   static constexpr int SMEM_BARS = NW * NS * 8;
   static constexpr int SMEM_MERGE = NW * (D + 2) * 4;
   static constexpr int SMEM = SMEM_PIPE + SMEM_BARS + SMEM_MERGE;
+  // Launched in clusters: partition 0's slots for the (acc, m, l) of up to 8
+  // partitions, written by the other CTAs of its cluster.
+  static constexpr int SMEM_XCH = 8 * (D + 2) * 4;
+  static constexpr int SMEM_CL = SMEM + SMEM_XCH;
   static_assert(S % CR == 0 && CR % RPW == 0 && NV >= 1 && NV <= LPR, "bad tiling");
   static_assert(UNIT % 16 == 0, "bulk copies move multiples of 16 bytes");
 };
@@ -117,7 +121,13 @@ struct RawFrag {
 //
 // TC is the cache element type: T itself, or E4M3 codes with per-tensor
 // scales (K's folded into q_scale, V's applied to the accumulated output).
-template <typename T, typename TO, int D, int S, bool APPEND, typename TC = T>
+//
+// CLUSTER = true: launched in clusters of p.NP CTAs, one per (request, head); partition 0 merges the others' results, which they store
+// into its shared memory, instead of the merge kernel reading them from the
+// workspace. (A template parameter, so that the plain form's code is not
+// touched by it.)
+template <typename T, typename TO, int D, int S, bool APPEND, typename TC = T,
+          bool CLUSTER = false>
 __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
     paged_decode_partition_kernel(const DecodeParams p) {
   constexpr int EB = sizeof(TC);
@@ -128,7 +138,13 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
   constexpr int DUP = LPR / NV;  // lanes of a group holding the same row's score
 
   grid_dependents_launch();  // the merge of split requests may be scheduled early
-  const int part = blockIdx.x;
+  // In a cluster launch every thread takes two cluster barriers, whichever
+  // path it follows: the first (arrived at here) guarantees that every CTA of
+  // the cluster has started before partition 0's shared memory is written, the
+  // second that the writes have landed before partition 0 reads them.
+  constexpr bool clustered = CLUSTER;
+  if constexpr (clustered) cluster_arrive_relaxed();
+  const int part = blockIdx.x;  // in a cluster launch, also the CTA's rank
   const int h = blockIdx.y;
   const int i = blockIdx.z;
   const int lane = threadIdx.x & 31;
@@ -143,8 +159,15 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
     L = L < 0 ? 0 : p.L_cap;
   }
   const int nparts = (L + p.P - 1) / p.P;
-  if (part > 0 && part >= nparts) return;  // nothing here (part 0 writes the L == 0 zeros)
-  const bool direct = nparts <= 1;          // the only partition: write the final output
+  if (part > 0 && part >= nparts) {  // nothing here (part 0 writes the L == 0 zeros)
+    if constexpr (clustered) {
+      cluster_wait_acquire();
+      cluster_arrive_release();
+      cluster_wait_acquire();
+    }
+    return;
+  }
+  const bool direct = nparts <= 1;  // the only partition: write the final output
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tl::SMEM_PIPE);
@@ -412,6 +435,15 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
     Ltot = fmaf(wgt[u], l_s[u], Ltot);
   }
   const int64_t ih = static_cast<int64_t>(i) * p.H + h;
+  // Cluster launch: this partition's (acc, m, l) go to its slot in partition
+  // 0's shared memory (every CTA of the cluster has started once the first
+  // barrier is passed).
+  float* xch = reinterpret_cast<float*>(smem + Tl::SMEM);
+  uint32_t xrem = 0;
+  if constexpr (clustered) {
+    cluster_wait_acquire();
+    xrem = cluster_map(smem_u32(xch + part * (D + 2)), 0);
+  }
   for (int d = threadIdx.x; d < D; d += NW * 32) {
     float a = 0.f;
 #pragma unroll
@@ -420,13 +452,44 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
     if (direct) {
       const float o = Ltot > 0.f ? a / Ltot : 0.f;
       static_cast<TO*>(p.out)[ih * D + d] = to_out<TO>(o);
+    } else if constexpr (clustered) {
+      st_cluster_f32(xrem + d * 4, a);
     } else {
       p.ws_acc[(ih * p.NP + part) * D + d] = a;
     }
   }
   if (!direct && threadIdx.x == 0) {
-    p.ws_m[ih * p.NP + part] = M;
-    p.ws_l[ih * p.NP + part] = Ltot;
+    if constexpr (clustered) {
+      st_cluster_f32(xrem + D * 4, M);
+      st_cluster_f32(xrem + (D + 1) * 4, Ltot);
+    } else {
+      p.ws_m[ih * p.NP + part] = M;
+      p.ws_l[ih * p.NP + part] = Ltot;
+    }
+  }
+  if constexpr (clustered) {
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    if (part != 0 || direct) return;
+    // Partition 0 merges, with the arithmetic of splitkv_reduce_kernel and in
+    // its order, so both ways of merging give the same bits: weights
+    // 2^(m_r - M), the weighted l summed as that kernel's shuffle tree sums
+    // them, the weighted acc summed over r in order.
+    float Mx = -INFINITY;
+    for (int r = 0; r < nparts; ++r) Mx = fmaxf(Mx, xch[r * (D + 2) + D]);
+    float wr[8], lw[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      wr[r] = r < nparts ? exp2f(xch[r * (D + 2) + D] - Mx) : 0.f;
+      lw[r] = r < nparts ? fmaf(wr[r], xch[r * (D + 2) + D + 1], 0.f) : 0.f;
+    }
+    const float lw_sum =
+        ((lw[0] + lw[4]) + (lw[2] + lw[6])) + ((lw[1] + lw[5]) + (lw[3] + lw[7]));
+    for (int d = threadIdx.x; d < D; d += NW * 32) {
+      float a = 0.f;
+      for (int r = 0; r < nparts; ++r) a = fmaf(wr[r], xch[r * (D + 2) + d], a);
+      static_cast<TO*>(p.out)[ih * D + d] = to_out<TO>(lw_sum > 0.f ? a / lw_sum : 0.f);
+    }
   }
 }
 
@@ -438,15 +501,17 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
 template <typename TO, int D>
 __global__ void __launch_bounds__(128) splitkv_reduce_kernel(const DecodeParams p) {
   constexpr int DL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t ih = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  const bool live = ih < static_cast<int64_t>(p.B) * p.H;
+  // The lengths are an input of both kernels, not a result of the first, so
+  // they are read before the wait.
+  int L = live ? __ldg(p.seq_lens + ih / p.H) : 0;
   // Launched as a programmatic dependent of the partition pass: its CTAs may be
   // resident before that pass ends; this waits until the pass has completed
   // and its partials are visible.
   grid_dependency_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t ih = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
-  if (ih >= static_cast<int64_t>(p.B) * p.H) return;
-  const int i = static_cast<int>(ih / p.H);
-  int L = __ldg(p.seq_lens + i);
+  if (!live) return;
   L = L < 0 ? 0 : (L > p.L_cap ? p.L_cap : L);
   const int nparts = (L + p.P - 1) / p.P;
   if (nparts <= 1) return;  // written by the partition pass
@@ -505,6 +570,35 @@ inline cudaError_t launch_splitkv_reduce(const DecodeParams& p, cudaStream_t str
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, splitkv_reduce_kernel<TO, D>, p);
+}
+
+// Launches the partition pass (grid NP x H x B) and the merge: `kern_cl` in
+// clusters of NP CTAs that merge among themselves (dynamic shared memory
+// smem_cl), or `kern` as a plain grid (smem) followed by the merge kernel.
+template <typename TO, int D, typename Kern>
+inline cudaError_t launch_partition_pass(Kern kern, Kern kern_cl, bool cluster,
+                                         const DecodeParams& p, int threads, int smem,
+                                         int smem_cl, cudaStream_t stream) {
+  const dim3 grid(p.NP, p.H, p.B);
+  if (cluster) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem_cl;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.NP;  // one cluster per (request, head)
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern_cl, p);
+  }
+  kern<<<grid, threads, smem, stream>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_splitkv_reduce<TO, D>(p, stream);
 }
 
 }  // namespace pa

@@ -95,6 +95,32 @@ __device__ __forceinline__ void grid_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Thread-block clusters. The cluster barrier is split: every thread of every
+// CTA of the cluster arrives, then waits until all have arrived (non-.aligned
+// forms, so a warp need not be converged). A relaxed arrival orders nothing;
+// a release arrival followed by an acquire wait makes the arriving threads'
+// earlier shared-memory stores (distributed ones included) visible to the
+// waiting threads.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+// The shared::cluster address of the same shared-memory offset in CTA `rank`
+// of this cluster, and a 32-bit store through such an address.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 // L2 policy for data read exactly once per step (the KV slabs).
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t pol;

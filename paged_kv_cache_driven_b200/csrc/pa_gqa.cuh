@@ -137,6 +137,19 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
 
+  // The producer's first table entries assume a whole partition (P / S
+  // blocks, clipped to the table's row), so they are requested together with
+  // the length; a request's last, partial partition loads them again.
+  const int t_beg = part * p.P;
+  const int blk0 = t_beg / S;
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(i) * p.MB;
+  int ids_a = -1, ids_b = -1;
+  auto load_ids = [&](int blk1) {
+    const int lim = min(blk1, p.MB);
+    ids_a = (blk0 + lane < lim) ? __ldg(trow + blk0 + lane) : -1;
+    ids_b = (blk0 + 32 + lane < lim) ? __ldg(trow + blk0 + 32 + lane) : -1;
+  };
+  if (w == NC) load_ids(blk0 + p.P / S);
   int L = __ldg(p.seq_lens + i);
   const bool len_ok = L >= 0 && L <= p.L_cap;
   if (!len_ok) {
@@ -163,10 +176,8 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   }
   __syncthreads();
 
-  const int t_beg = part * p.P;
   const int t_end = min(t_beg + p.P, L);
   const int nunits = t_end > t_beg ? (t_end - t_beg + ROWS - 1) / ROWS : 0;
-  const int32_t* trow = p.block_tables + static_cast<int64_t>(i) * p.MB;
   const int64_t block_stride = static_cast<int64_t>(p.Hkv) * SLAB;
   const uint8_t* kbase = static_cast<const uint8_t*>(p.k_cache) + static_cast<int64_t>(hk) * SLAB;
   const uint8_t* vbase = static_cast<const uint8_t*>(p.v_cache) + static_cast<int64_t>(hk) * SLAB;
@@ -174,11 +185,9 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   if (w == NC) {
     // ---- producer: one lane per box of a unit issues the loads ----
     const uint64_t policy = policy_evict_first();
-    const int blk0 = t_beg / S;
     const int blk1 = t_end > t_beg ? (t_end + S - 1) / S : blk0;
+    if (t_end < t_beg + p.P) load_ids(blk1);  // the last partition: its own run
     int base = 0;
-    int ids_a = (blk0 + lane < blk1) ? __ldg(trow + blk0 + lane) : -1;
-    int ids_b = (blk0 + 32 + lane < blk1) ? __ldg(trow + blk0 + 32 + lane) : -1;
     for (int u = 0; u < nunits; ++u) {
       const int s = u % NS;
       // every lane waits; the warp leaves together if any lane gave up
@@ -322,7 +331,8 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
 
   for (int k = w; k < nunits; k += NC) {
     const int s = k % NS;
-    if (!mbar_wait_bounded(&full[s], (k / NS) & 1)) {
+    // every lane waits; the warp leaves together if any lane gave up
+    if (!__all_sync(kFullMask, mbar_wait_bounded(&full[s], (k / NS) & 1))) {
       if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
       break;
     }

@@ -1,6 +1,8 @@
 // Kernels of pa_decode / pa_decode_append with one KV head per query head:
-// the partition pass (with its fused split-KV merge) for every cache dtype,
-// output dtype, head size and block size, and their launcher.
+// the partition pass (whose CTAs merge a split request among themselves in a
+// cluster launch, or leave partials for the merge kernel) and the merge kernel,
+// for every cache dtype, output dtype, head size and block size, and their
+// launcher.
 
 #include <type_traits>
 
@@ -13,21 +15,24 @@ namespace {
 
 // One CTA per (partition, head, request).
 template <typename T, typename TO, int D, int S, bool APPEND>
-pa_status launch(const DecodeParams& prm, cudaStream_t stream) {
+pa_status launch(const DecodeParams& prm, bool cluster, cudaStream_t stream) {
   using Tl = DecodeTiling<D, S>;
   auto kern = paged_decode_partition_kernel<T, TO, D, S, APPEND>;
-  static bool configured[kMaxDevices] = {};
-  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
-  const dim3 grid(prm.NP, prm.H, prm.B);
-  kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
-  if (launch_splitkv_reduce<TO, D>(prm, stream) != cudaSuccess) return PA_ERR_CUDA;
+  auto kern_cl = paged_decode_partition_kernel<T, TO, D, S, APPEND, T, true>;
+  static bool configured[kMaxDevices] = {}, configured_cl[kMaxDevices] = {};
+  if (!opt_in_smem(kern, Tl::SMEM, configured) ||
+      !opt_in_smem(kern_cl, Tl::SMEM_CL, configured_cl))
+    return PA_ERR_CUDA;
+  if (launch_partition_pass<TO, D>(kern, kern_cl, cluster, prm, Tl::NW * 32, Tl::SMEM,
+                                   Tl::SMEM_CL, stream) != cudaSuccess)
+    return PA_ERR_CUDA;
   return cuda_status();
 }
 
 template <typename T, typename TO, bool APPEND>
-pa_status by_shape(const DecodeParams& prm, int D, int S, cudaStream_t st) {
+pa_status by_shape(const DecodeParams& prm, int D, int S, bool cl, cudaStream_t st) {
 #define PA_CASE(DD, SS) \
-  if (D == DD && S == SS) return launch<T, TO, DD, SS, APPEND>(prm, st);
+  if (D == DD && S == SS) return launch<T, TO, DD, SS, APPEND>(prm, cl, st);
   PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
   PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
   PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
@@ -36,11 +41,12 @@ pa_status by_shape(const DecodeParams& prm, int D, int S, cudaStream_t st) {
 }
 
 template <typename T, bool APPEND>
-pa_status by_out(const DecodeParams& prm, pa_dtype out_dt, int D, int S, cudaStream_t st) {
+pa_status by_out(const DecodeParams& prm, pa_dtype out_dt, int D, int S, bool cl,
+                 cudaStream_t st) {
   switch (out_dt) {
-    case PA_F32: return by_shape<T, float, APPEND>(prm, D, S, st);
-    case PA_F16: return by_shape<T, __half, APPEND>(prm, D, S, st);
-    case PA_BF16: return by_shape<T, __nv_bfloat16, APPEND>(prm, D, S, st);
+    case PA_F32: return by_shape<T, float, APPEND>(prm, D, S, cl, st);
+    case PA_F16: return by_shape<T, __half, APPEND>(prm, D, S, cl, st);
+    case PA_BF16: return by_shape<T, __nv_bfloat16, APPEND>(prm, D, S, cl, st);
   }
   return PA_ERR_INVALID;
 }
@@ -48,12 +54,12 @@ pa_status by_out(const DecodeParams& prm, pa_dtype out_dt, int D, int S, cudaStr
 }  // namespace
 
 pa_status launch_decode16(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt, int D, int S,
-                          bool append, cudaStream_t stream) {
+                          bool append, bool cluster, cudaStream_t stream) {
   if (append)
-    return dt == PA_F16 ? by_out<__half, true>(prm, out_dt, D, S, stream)
-                        : by_out<__nv_bfloat16, true>(prm, out_dt, D, S, stream);
-  return dt == PA_F16 ? by_out<__half, false>(prm, out_dt, D, S, stream)
-                      : by_out<__nv_bfloat16, false>(prm, out_dt, D, S, stream);
+    return dt == PA_F16 ? by_out<__half, true>(prm, out_dt, D, S, cluster, stream)
+                        : by_out<__nv_bfloat16, true>(prm, out_dt, D, S, cluster, stream);
+  return dt == PA_F16 ? by_out<__half, false>(prm, out_dt, D, S, cluster, stream)
+                      : by_out<__nv_bfloat16, false>(prm, out_dt, D, S, cluster, stream);
 }
 
 bool take_error_decode16(unsigned int* bits) { return take_error_word(bits); }

@@ -13,21 +13,24 @@ namespace {
 
 // One CTA per (partition, head, request).
 template <typename T, typename TO, int D, int S>
-pa_status launch(const DecodeParams& prm, cudaStream_t stream) {
+pa_status launch(const DecodeParams& prm, bool cluster, cudaStream_t stream) {
   using Tl = DecodeTiling<D, S, 1>;
   auto kern = paged_decode_partition_kernel<T, TO, D, S, false, __nv_fp8_e4m3>;
-  static bool configured[kMaxDevices] = {};
-  if (!opt_in_smem(kern, Tl::SMEM, configured)) return PA_ERR_CUDA;
-  const dim3 grid(prm.NP, prm.H, prm.B);
-  kern<<<grid, Tl::NW * 32, Tl::SMEM, stream>>>(prm);
-  if (launch_splitkv_reduce<TO, D>(prm, stream) != cudaSuccess) return PA_ERR_CUDA;
+  auto kern_cl = paged_decode_partition_kernel<T, TO, D, S, false, __nv_fp8_e4m3, true>;
+  static bool configured[kMaxDevices] = {}, configured_cl[kMaxDevices] = {};
+  if (!opt_in_smem(kern, Tl::SMEM, configured) ||
+      !opt_in_smem(kern_cl, Tl::SMEM_CL, configured_cl))
+    return PA_ERR_CUDA;
+  if (launch_partition_pass<TO, D>(kern, kern_cl, cluster, prm, Tl::NW * 32, Tl::SMEM,
+                                   Tl::SMEM_CL, stream) != cudaSuccess)
+    return PA_ERR_CUDA;
   return cuda_status();
 }
 
 template <typename T, typename TO>
-pa_status by_shape(const DecodeParams& prm, int D, int S, cudaStream_t st) {
+pa_status by_shape(const DecodeParams& prm, int D, int S, bool cl, cudaStream_t st) {
 #define PA_CASE(DD, SS) \
-  if (D == DD && S == SS) return launch<T, TO, DD, SS>(prm, st);
+  if (D == DD && S == SS) return launch<T, TO, DD, SS>(prm, cl, st);
   PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
   PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
   PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
@@ -36,11 +39,12 @@ pa_status by_shape(const DecodeParams& prm, int D, int S, cudaStream_t st) {
 }
 
 template <typename T>
-pa_status by_out(const DecodeParams& prm, pa_dtype out_dt, int D, int S, cudaStream_t st) {
+pa_status by_out(const DecodeParams& prm, pa_dtype out_dt, int D, int S, bool cl,
+                 cudaStream_t st) {
   switch (out_dt) {
-    case PA_F32: return by_shape<T, float>(prm, D, S, st);
-    case PA_F16: return by_shape<T, __half>(prm, D, S, st);
-    case PA_BF16: return by_shape<T, __nv_bfloat16>(prm, D, S, st);
+    case PA_F32: return by_shape<T, float>(prm, D, S, cl, st);
+    case PA_F16: return by_shape<T, __half>(prm, D, S, cl, st);
+    case PA_BF16: return by_shape<T, __nv_bfloat16>(prm, D, S, cl, st);
   }
   return PA_ERR_INVALID;
 }
@@ -48,9 +52,9 @@ pa_status by_out(const DecodeParams& prm, pa_dtype out_dt, int D, int S, cudaStr
 }  // namespace
 
 pa_status launch_decode_fp8(const DecodeParams& prm, pa_dtype q_dt, pa_dtype out_dt, int D,
-                            int S, cudaStream_t stream) {
-  return q_dt == PA_F16 ? by_out<__half>(prm, out_dt, D, S, stream)
-                        : by_out<__nv_bfloat16>(prm, out_dt, D, S, stream);
+                            int S, bool cluster, cudaStream_t stream) {
+  return q_dt == PA_F16 ? by_out<__half>(prm, out_dt, D, S, cluster, stream)
+                        : by_out<__nv_bfloat16>(prm, out_dt, D, S, cluster, stream);
 }
 
 bool take_error_fp8(unsigned int* bits) { return take_error_word(bits); }

@@ -77,12 +77,14 @@ bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_ro
 bool query_map(CUtensorMap* out, const void* q, int64_t T, int H, int D, pa_dtype dt);
 
 // Launchers (asynchronous on `stream`; the arguments are already checked).
+// cluster: launch the partition pass in clusters of prm.NP CTAs (NP of 2, 4
+// or 8) that merge a split among themselves, instead of the merge kernel.
 pa_status launch_decode16(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt, int D, int S,
-                          bool append, cudaStream_t stream);            // pa_k_decode.cu
+                          bool append, bool cluster, cudaStream_t stream);  // pa_k_decode.cu
 pa_status launch_grouped(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt, int D, int S,
                          bool append, cudaStream_t stream);             // pa_k_gqa.cu
 pa_status launch_decode_fp8(const DecodeParams& prm, pa_dtype q_dt, pa_dtype out_dt, int D,
-                            int S, cudaStream_t stream);                // pa_k_fp8.cu
+                            int S, bool cluster, cudaStream_t stream);  // pa_k_fp8.cu
 pa_status launch_prefill(const PrefillParams& prm, const void* q, pa_dtype dt, pa_dtype out_dt,
                          int D, int S, cudaStream_t stream);            // pa_k_prefill.cu
 pa_status launch_kv_append(const void* k, const void* v, const int64_t* slots, void* k_cache,

@@ -79,8 +79,19 @@ def test_workspace_and_plan(lib):
     assert binding.pa_decode_plan(64, 40, 128, 16, 2048, partition=-1) == (0, 1)
     assert binding.pa_decode_plan(64, 40, 128, 16, 2048, partition=256) == (256, 8)
     # small grids: partitions halve while the grid has fewer CTAs than SMs (148
-    # without a device): one request of 1332 tokens on 32 heads -> 256 x 6
-    assert binding.pa_decode_plan(1, 32, 128, 16, 1332) == (256, 6)
+    # without a device); a count of 3, 5, 6 or 7 is then rounded to a power of
+    # two (the next, else the previous) if the grid stays within 2 CTAs per SM:
+    # one request of 1332 tokens on 32 heads -> 256 x 6 -> 176 x 8 (256 CTAs)
+    assert binding.pa_decode_plan(1, 32, 128, 16, 1332) == (176, 8)
+    # on 40 heads 8 partitions would be 320 CTAs: 4 of 336 tokens instead
+    assert binding.pa_decode_plan(1, 40, 128, 16, 1332) == (336, 4)
+    # 3 partitions of 64 -> 4 of 48 (S = 16)
+    assert binding.pa_decode_plan(1, 32, 128, 16, 150) == (48, 4)
+    assert binding.pa_decode_plan(2, 32, 128, 16, 280) == (80, 4)
+    # 270 tokens in blocks of 32: 8 partitions of 64 tokens, the last three empty
+    assert binding.pa_decode_plan(1, 1, 128, 32, 270) == (64, 8)
+    # 1332 tokens in blocks of 32 on 32 heads: 8 of 192 (the eighth empty)
+    assert binding.pa_decode_plan(1, 32, 128, 32, 1332) == (192, 8)
     assert binding.pa_decode_plan(1, 1, 128, 16, 8192) == (64, 128)
     assert binding.pa_decode_plan(1, 32, 128, 8, 100) == (64, 2)
     n = 64 * 40 * 4
