@@ -907,6 +907,116 @@ def prefill_cpu_baseline(target_seconds, cores, seed):
                                f"{total:.1f} s on {cores} threads")
 
 
+def prefill_trace_phases(buf):
+    """Per-phase medians (SM cycles) from the trace build's stamps
+    [CTA][slot][key tile] (slot meanings in pa_prefill.cuh), over the
+    steady-state key tiles of the traced CTAs: the first two and the last key
+    tile of each CTA are left out."""
+    agg = {}
+
+    def add(k, v):
+        if v > 0:
+            agg.setdefault(k, []).append(int(v))
+
+    for cta in range(buf.shape[0]):
+        if buf[cta, 31, 0] == 0:
+            continue
+        nk = int((buf[cta, 20, :] > 0).sum())
+        for j in range(2, nk - 1):
+            for t in range(2):
+                for hw in range(2):
+                    k = 2 * t + hw
+                    s0 = buf[cta, k, j]
+                    if s0 == 0 or buf[cta, 16 + k, j] == 0:
+                        continue
+                    add("softmax: scores from tensor memory and the row max",
+                        buf[cta, 4 + k, j] - s0)
+                    add("softmax: the max exchange between the two halves",
+                        buf[cta, 8 + k, j] - buf[cta, 4 + k, j])
+                    add("softmax: weights P (exp2, hi + lo packing, stores)",
+                        buf[cta, 12 + k, j] - buf[cta, 8 + k, j])
+                    add("softmax: output rescale and fences",
+                        buf[cta, 16 + k, j] - buf[cta, 12 + k, j])
+                    add("softmax of one query tile and key tile (per warpgroup)",
+                        buf[cta, 16 + k, j] - s0)
+                    if buf[cta, k, j + 1]:
+                        add("from a warpgroup's P-ready arrival to its next scores",
+                            buf[cta, k, j + 1] - buf[cta, 16 + k, j])
+            for t in range(2):
+                if buf[cta, 20 + t, j] and buf[cta, 22 + t, j]:
+                    add(f"MMA warp: P(j) of tile {t} seen to its P.V and next S issued",
+                        buf[cta, 22 + t, j] - buf[cta, 20 + t, j])
+            if buf[cta, 20, j + 1]:
+                add("one key tile for both query tiles (period)",
+                    buf[cta, 20, j + 1] - buf[cta, 20, j])
+    return {k: {"median": int(statistics.median(v)), "n": len(v)} for k, v in agg.items()}
+
+
+def run_prefill_trace(args):
+    """--workload prefill_trace: where the prefill kernel's time goes. The
+    profiling-size prompt case (4 prompts of 2048 tokens, 8 heads) runs on the
+    library proper and on the trace build (libpagedattn_trace.so, from
+    `python -m paged_kv_cache_driven_b200.build --trace`: the same kernel with
+    clock stamps at its hand-offs); the two outputs must be the same bits, and
+    the trace build's stamps of one launch are reduced to per-phase medians in
+    SM cycles (prefill_trace_phases)."""
+    import ctypes
+    import numpy as np
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    pc = workloads.prompt_prefill(seed=args.seed, device=device, n_req=4, lo=2048, hi=2048, H=8)
+    c = pc.cache
+    T, Hq, Dh = pc.q.shape
+
+    def run(out):
+        binding.pa_prefill(out, pc.q, c.k_cache, c.v_cache, c.block_tables, c.seq_lens,
+                           pc.q_start, c.scale, pc.max_q_len)
+
+    def timed(out):
+        for _ in range(args.warmup):
+            run(out)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        run(out)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    ref = torch.empty((T, Hq, Dh), dtype=DTYPE, device=device)
+    ms_plain = timed(ref)
+    if binding.pa_get_device_error():
+        raise SystemExit("device error word set")
+    path = os.path.join(ROOT, "paged_kv_cache_driven_b200", "libpagedattn_trace.so")
+    th = binding.open_library(path)
+    th.pa_prefill_trace_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
+    th.pa_prefill_trace_read.restype = ctypes.c_int
+    th.pa_prefill_trace_clear.restype = ctypes.c_int
+    prev = binding.use_library(th)
+    try:
+        got = torch.empty_like(ref)
+        for _ in range(args.warmup):
+            run(got)
+        torch.cuda.synchronize()
+        if th.pa_prefill_trace_clear() != 0:
+            raise SystemExit("pa_prefill_trace_clear failed")
+        ms_trace = timed(got)
+        buf = np.zeros((64, 32, 48), dtype=np.int64)
+        if th.pa_prefill_trace_read(ctypes.c_void_p(buf.ctypes.data), buf.nbytes) != 0:
+            raise SystemExit("pa_prefill_trace_read failed")
+        if binding.pa_get_device_error():
+            raise SystemExit("device error word set (trace build)")
+    finally:
+        binding.use_library(prev)
+    same = torch.equal(ref.view(torch.int16), got.view(torch.int16))
+    print(json.dumps({"workload": "prompt prefill, profiling size: 4 prompts of 2048 tokens, "
+                                  "8 heads, head_dim 128, block 16, bf16, causal",
+                      "launch_ms": round(ms_plain, 4), "launch_ms_trace_build": round(ms_trace, 4),
+                      "same_bits_as_library": same, "traced_ctas": int((buf[:, 31, 0] > 0).sum()),
+                      "cycles": prefill_trace_phases(buf)}), flush=True)
+    if not same:
+        raise SystemExit("the trace build's output differs from the library's")
+
+
 def run_prefill_workload(args):
     """--workload prompt_prefill: pa_prefill over the prompt prefill workload,
     TFLOP/s against the measured bf16 tensor peak, plus an end-to-end prefill
@@ -1054,12 +1164,15 @@ def main():
     ap.add_argument("--workload", default="llama13b",
                     choices=["llama13b", "long_context", "sweep", "llama70b", "llama13b_fp8",
                              "prompt_prefill", "prompt_prefill_small", "worked_example",
-                             "prefill_append", "prefill_append_small", "batching"],
+                             "prefill_append", "prefill_append_small", "batching",
+                             "prefill_trace"],
                     help="llama13b: the headline step (default); the others time decode-only "
                          "calls of the long-context, shape-sweep and LLaMA-2-70B-shaped "
                          "grouped-query configurations, paged prefill attention over "
                          "16 prompts (prompt_prefill), the pages' worked example, the "
-                         "prefill-scale append, or the continuous-batching loop")
+                         "prefill-scale append, or the continuous-batching loop; "
+                         "prefill_trace: per-phase clock stamps of the prefill kernel "
+                         "(needs `python -m paged_kv_cache_driven_b200.build --trace`)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
@@ -1071,7 +1184,8 @@ def main():
         run_prefill_workload(args)
         return
     extra = {"worked_example": run_worked_example, "prefill_append": run_append_workload,
-             "prefill_append_small": run_append_workload, "batching": run_batching_workload}
+             "prefill_append_small": run_append_workload, "batching": run_batching_workload,
+             "prefill_trace": run_prefill_trace}
     if args.workload in extra:
         binding.lib()
         extra[args.workload](args)

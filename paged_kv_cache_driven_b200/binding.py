@@ -83,19 +83,32 @@ class PagedAttnError(RuntimeError):
         self.code = code
 
 
+def open_library(path):
+    """Loads the library build at `path` with the C signatures declared here."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: run `python -m paged_kv_cache_driven_b200.build`")
+    handle = ctypes.CDLL(path)
+    for name, (args, res) in _SIGNATURES.items():
+        fn = getattr(handle, name)
+        fn.argtypes = args
+        fn.restype = res
+    return handle
+
+
 def lib():
     """The loaded library (loaded on first use; raises if it was never built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: run `python -m paged_kv_cache_driven_b200.build`")
-        handle = ctypes.CDLL(LIB_PATH)
-        for name, (args, res) in _SIGNATURES.items():
-            fn = getattr(handle, name)
-            fn.argtypes = args
-            fn.restype = res
-        _lib = handle
+        _lib = open_library(LIB_PATH)
     return _lib
+
+
+def use_library(handle):
+    """Makes `handle` (from open_library) the library the functions here call;
+    returns the one it replaces (None if none was loaded yet)."""
+    global _lib
+    old, _lib = _lib, handle
+    return old
 
 
 def _check(rc, where):

@@ -4,7 +4,12 @@ The kernels are split over several translation units (csrc/pa_k_*.cu) that
 compile in parallel into ``_build/``; a unit is recompiled when it or any
 header is newer than its object, then everything is linked into one library.
 
-Usage: python -m paged_kv_cache_driven_b200.build [--verbose] [--force]
+With --trace it also builds libpagedattn_trace.so: the same library with the
+prefill unit compiled with PA_PREFILL_TRACE, which adds clock stamps at the
+prefill kernel's hand-offs and exports pa_prefill_trace_read / _clear (for
+bench.py --workload prefill_trace; the library proper has none of it).
+
+Usage: python -m paged_kv_cache_driven_b200.build [--verbose] [--force] [--trace]
 """
 
 import concurrent.futures
@@ -18,6 +23,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libpagedattn.so")
+TRACE_LIB = os.path.join(PKG, "libpagedattn_trace.so")
+TRACE_SRC = os.path.join(CSRC, "pa_k_prefill.cu")
+TRACE_OBJ = os.path.join(OBJ, "pa_k_prefill.trace.o")
 SOURCES = sorted(glob.glob(os.path.join(CSRC, "*.cu"))) + \
     [os.path.join(CSRC, f) for f in ("pa_alloc.cpp", "pa_stepper.cpp")]
 HEADERS = sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))) + \
@@ -78,6 +86,28 @@ def build(force=False, verbose=False):
     return LIB
 
 
+def build_trace(force=False, verbose=False):
+    """libpagedattn_trace.so: the objects of build(), with the prefill unit
+    compiled with PA_PREFILL_TRACE instead."""
+    build(force=force, verbose=verbose)
+    fresh = os.path.exists(TRACE_OBJ) and all(
+        os.path.getmtime(f) <= os.path.getmtime(TRACE_OBJ) for f in [TRACE_SRC, *HEADERS])
+    if force or not fresh:
+        cmd = [NVCC, *FLAGS, "-DPA_PREFILL_TRACE", "-c", TRACE_SRC, "-o", TRACE_OBJ]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if verbose or r.returncode != 0:
+            sys.stderr.write(r.stdout + r.stderr)
+        if r.returncode != 0:
+            raise subprocess.CalledProcessError(r.returncode, "nvcc")
+    objs = [TRACE_OBJ if s == TRACE_SRC else _obj(s) for s in SOURCES]
+    subprocess.run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs,
+                    "-o", TRACE_LIB], check=True)
+    return TRACE_LIB
+
+
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
+    if "--trace" in sys.argv:
+        build_trace(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
+    else:
+        build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
     print(LIB)

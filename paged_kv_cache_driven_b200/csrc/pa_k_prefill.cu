@@ -62,3 +62,18 @@ bool take_error_prefill(unsigned int* bits) { return take_error_word(bits); }
 
 }  // namespace host
 }  // namespace pa
+
+#ifdef PA_PREFILL_TRACE
+// Trace build only: the stamp buffer g_prefill_trace ([64][32][48] int64, see
+// pa_prefill.cuh), copied to host memory `dst` of `bytes` (which must be its
+// size), or set to zero. Return 0 on success.
+extern "C" int pa_prefill_trace_read(void* dst, size_t bytes) {
+  if (!dst || bytes != sizeof(pa::g_prefill_trace)) return 1;
+  return cudaMemcpyFromSymbol(dst, pa::g_prefill_trace, bytes) == cudaSuccess ? 0 : 2;
+}
+extern "C" int pa_prefill_trace_clear(void) {
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, pa::g_prefill_trace) != cudaSuccess) return 2;
+  return cudaMemset(addr, 0, sizeof(pa::g_prefill_trace)) == cudaSuccess ? 0 : 2;
+}
+#endif

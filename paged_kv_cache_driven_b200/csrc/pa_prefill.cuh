@@ -46,6 +46,26 @@
 
 namespace pa {
 
+#ifdef PA_PREFILL_TRACE
+// Trace build only (libpagedattn_trace.so; the library proper compiles none of
+// this): clock64() stamps at the kernel's hand-offs, for the CTAs of query
+// head 0 with request < 8 and row block < 8, indexed [CTA][slot][key tile].
+// Slots: 31 start, 30 end; producer 25 K(j) issued, 26 V(j) issued; MMA warp
+// 24 V(j) landed, 20 + t P(j) of tile t seen, 22 + t its P.V and next S
+// issued; softmax half k = 2t + hw: 0 + k scores ready, 4 + k row max taken,
+// 8 + k max exchanged, 12 + k P stored, 16 + k output rescaled and fenced.
+constexpr int kTraceCtas = 64, kTraceSlots = 32, kTraceTiles = 48;
+__device__ long long g_prefill_trace[kTraceCtas][kTraceSlots][kTraceTiles];
+#define PA_TRACE(slot, j)                                                       \
+  do {                                                                          \
+    if (trc >= 0 && (j) < kTraceTiles) g_prefill_trace[trc][slot][j] = clock64(); \
+  } while (0)
+#else
+#define PA_TRACE(slot, j) \
+  do {                    \
+  } while (0)
+#endif
+
 
 template <int D, bool LO>
 struct PrefillTiling {
@@ -222,6 +242,10 @@ __global__ void __launch_bounds__(576, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#ifdef PA_PREFILL_TRACE
+  const int trc = (h == 0 && i < 8 && blockIdx.x < 8) ? i * 8 + blockIdx.x : -1;
+  if (threadIdx.x == 0) PA_TRACE(31, 0);
+#endif
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < Tl::KST; ++s) {
@@ -304,12 +328,14 @@ __global__ void __launch_bounds__(576, 1)
         if (kj >= Tl::KST && !(ok = wait_warp(&k_empty[st], ((kj / Tl::KST) - 1) & 1, abort_flag)))
           break;
         load_tile(&tmk, sK + st * Tl::KV_BYTES, &k_full[st], id_k);
+        if (lane == 0) PA_TRACE(25, kj);
         k_issued = kj + 1;
       }
       const int st = j % Tl::VST;
       if (j >= Tl::VST && !(ok = wait_warp(&v_empty[st], ((j / Tl::VST) - 1) & 1, abort_flag)))
         break;
       load_tile(&tmv, sV + st * Tl::KV_BYTES, &v_full[st], id_v);
+      if (lane == 0) PA_TRACE(26, j);
       v_issued = j + 1;
       id_v = id_k;
       if (j + 2 < NK) id_k = block_id(j + 2);
@@ -353,6 +379,7 @@ __global__ void __launch_bounds__(576, 1)
       const int st = j % Tl::VST;
       ok = wait_warp(&v_full[st], (j / Tl::VST) & 1, abort_flag);
       if (!ok) break;
+      if (lane == 0) PA_TRACE(24, j);
       const int kb = j * Tl::BN;
       if (j == NK - 1 && kb + Tl::BN > L) {
         // keys past the end of the request: P is 0 there, and 0 * NaN would not be
@@ -371,6 +398,7 @@ __global__ void __launch_bounds__(576, 1)
         if (j >= nk[t]) continue;
         ok = wait_warp(&p_full[t], j & 1, abort_flag);
         if (!ok) break;
+        if (lane == 0) PA_TRACE(20 + t, j);
         tc::fence_after_sync();
         if (lane == 0) {
           const uint32_t tS = tmem + t * 256, tO = tS + 128;
@@ -389,6 +417,7 @@ __global__ void __launch_bounds__(576, 1)
           tc::fence_after_sync();
           if (lane == 0) issue_s(t, j + 1);
         }
+        if (lane == 0) PA_TRACE(22 + t, j);
       }
       // V(j) and, if any tile read it, K(j + 1) are free once these products finish
       if (ok && lane == 0) {
@@ -422,6 +451,7 @@ __global__ void __launch_bounds__(576, 1)
     for (int j = 0; ok && j < nk[t]; ++j) {
       ok = wait_warp(&s_full[t], j & 1, abort_flag);
       if (!ok) break;
+      if (r == 0) PA_TRACE(0 + t * 2 + hw, j);
       tc::fence_after_sync();
       const int kb = j * Tl::BN + hw * HK;
       // keys past this row's last one count as -inf (scale > 0, so the order of
@@ -448,10 +478,12 @@ __global__ void __launch_bounds__(576, 1)
       // the row's max over both halves: post this half's, read the other's
       // (slots alternate with the key tile, so a half never overwrites a value
       // the other has not read yet)
+      if (r == 0) PA_TRACE(4 + t * 2 + hw, j);
       slot(j, hw)[r] = hmax;
       mbar_arrive(&xch_bar[t]);
       ok = wait_warp(&xch_bar[t], j & 1, abort_flag);
       if (!ok) break;
+      if (r == 0) PA_TRACE(8 + t * 2 + hw, j);
       const float tmax = fmaxf(hmax, slot(j, hw ^ 1)[r]) * p.scale_log2;
       // The reference max only moves when the tile max exceeds it by more than
       // 2^8 in weight; the weights stay <= 256, exact in the final ratio. Both
@@ -488,6 +520,7 @@ __global__ void __launch_bounds__(576, 1)
         tc::tmem_st4(tS + col, hi);
         if constexpr (LO) tc::tmem_st4(tS + col + 16, lo);
       }
+      if (r == 0) PA_TRACE(12 + t * 2 + hw, j);
       // The product of the previous key tile has completed (the commit that
       // released these scores covers it): rescale this half's output columns
       // of the rows whose max moved.
@@ -505,6 +538,7 @@ __global__ void __launch_bounds__(576, 1)
       l = l * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
       tc::tmem_wait_st();
       tc::fence_before_sync();
+      if (r == 0) PA_TRACE(16 + t * 2 + hw, j);
       mbar_arrive(&p_full[t]);
     }
     // epilogue: the row's sum over both halves, then O / l -> out (this half's columns)
@@ -532,6 +566,7 @@ __global__ void __launch_bounds__(576, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
+  if (threadIdx.x == 0) PA_TRACE(30, 0);
   if (warp == kIssuer) {
     __syncwarp();
     tc::fence_after_sync();
