@@ -516,7 +516,9 @@ def time_decode_case(case, iters, warmup, partition=0):
 def time_decode_fp8(seed, iters, warmup):
     """The LLaMA-2-13B decode shape over an E4M3 cache (filled by pa_kv_append_fp8
     from the bf16 case): median event-timed pa_decode_fp8 call with L2 flushed
-    before each; returns (ms, KV bytes, plan)."""
+    before each, and the same for pa_decode_append_fp8 (each request's new row
+    quantized into its last slot inside the launch); returns (ms, KV bytes,
+    plan, fused-append ms)."""
     device = torch.device("cuda", 0)
     case = workloads.llama13b_decode(seed=seed, device=device)
     B, Hc, Dc = case.q.shape
@@ -533,22 +535,34 @@ def time_decode_fp8(seed, iters, warmup):
     wsb = binding.pa_decode_workspace_bytes(B, Hc, Dc, Sc, maxlen, 0)
     ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device)
     flush = L2Flush(device)
-    times = []
-    for k in range(warmup + iters):
-        flush()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        binding.pa_decode_fp8(out, case.q, kc8, vc8, 0.05, 0.08, case.block_tables,
-                              case.seq_lens, case.scale, maxlen, partition=0, workspace=ws)
-        b.record()
-        torch.cuda.synchronize()
-        if k >= warmup:
-            times.append(a.elapsed_time(b))
-    if binding.pa_get_device_error():
-        raise SystemExit("device error word set")
+    g = torch.Generator(device=device).manual_seed(seed + 77)
+    k_new = torch.randn((B, Hc, Dc), generator=g, device=device).to(DTYPE)
+    v_new = torch.randn((B, Hc, Dc), generator=g, device=device).to(DTYPE)
+
+    def timed(call):
+        times = []
+        for k in range(warmup + iters):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            torch.cuda.synchronize()
+            if k >= warmup:
+                times.append(a.elapsed_time(b))
+        if binding.pa_get_device_error():
+            raise SystemExit("device error word set")
+        return statistics.median(times)
+
+    ms = timed(lambda: binding.pa_decode_fp8(out, case.q, kc8, vc8, 0.05, 0.08, case.block_tables,
+                                             case.seq_lens, case.scale, maxlen, partition=0,
+                                             workspace=ws))
+    ms_fused = timed(lambda: binding.pa_decode_append_fp8(
+        out, case.q, k_new, v_new, kc8, vc8, 0.05, 0.08, case.block_tables, case.seq_lens,
+        case.scale, maxlen, partition=0, workspace=ws))
     nbytes = sum(Hc * (2 * L * Dc + 2 * Dc * 2) + 4 * (-(-L // Sc)) for L in case.seq_lens_host) \
         + 4 * B
-    return statistics.median(times), nbytes, binding.pa_decode_plan(B, Hc, Dc, Sc, maxlen, 0)
+    return ms, nbytes, binding.pa_decode_plan(B, Hc, Dc, Sc, maxlen, 0), ms_fused
 
 
 def latency_floors(device, iters, warmup):
@@ -591,11 +605,12 @@ def run_shape_workloads(args):
         cases = [("long_context", lambda: workloads.long_context_decode(seed=args.seed,
                                                                         device=device))]
     elif args.workload == "llama13b_fp8":
-        ms, nbytes, plan = time_decode_fp8(args.seed, args.steps, args.warmup)
+        ms, nbytes, plan, ms_fused = time_decode_fp8(args.seed, args.steps, args.warmup)
         gbs = nbytes / (ms / 1e3) / 1e9
         print(json.dumps({"workload": "llama13b_fp8_e4m3_cache", "ms": round(ms, 4),
                           "gb_s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 3),
                           "kv_bytes": nbytes, "tok_s_layer": round(64 / (ms / 1e3), 1),
+                          "fused_append_ms": round(ms_fused, 4),
                           "partition": {"tokens": plan[0], "num": plan[1]},
                           "l2": L2_FLUSHED}), flush=True)
         return

@@ -177,12 +177,29 @@ pa_status pa_kv_append_fp8(const void* k, const void* v, pa_dtype in_dt,
  * out[i, h] = softmax_t(scale * q . K_t) V_t with K_t, V_t dequantized as above
  * (k_scale is folded into the scores, v_scale into the output). D, S,
  * partition, workspace (pa_decode_workspace_bytes) and errors as pa_decode; one
- * KV head per query head; no fused append (append with pa_kv_append_fp8). */
+ * KV head per query head. */
 pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
                         const void* k_cache, const void* v_cache, float k_scale, float v_scale,
                         const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
                         int B, int H, int D, int S, int NB, int partition, int max_seq_len,
                         void* workspace, size_t ws_bytes, void* stream);
+
+/* One decode step over E4M3 caches in one launch: pa_kv_append_fp8 of the new
+ * tokens' rows, then pa_decode_fp8 ([vllm] 7단계 "전체 흐름 요약": the new token's
+ * K/V is added to the cache, then attention reads the cache). For each request
+ * i with L = seq_lens[i] >= 1, k_new[i] and v_new[i] ([B, H, D], dtype q_dt,
+ * 16-byte aligned) are quantized with k_scale / v_scale as pa_kv_append_fp8
+ * does and written at token position L - 1 (block block_tables[i][(L-1)/S],
+ * offset (L-1)%S), and the attention over the request's L tokens sees them.
+ * The output and the cache bytes are those of pa_kv_append_fp8 followed by
+ * pa_decode_fp8, bit for bit. Other arguments, workspace and errors as
+ * pa_decode_fp8; a request whose length is out of range appends nothing. */
+pa_status pa_decode_append_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
+                               const void* k_new, const void* v_new, void* k_cache,
+                               void* v_cache, float k_scale, float v_scale,
+                               const int32_t* block_tables, int MB, const int32_t* seq_lens,
+                               float scale, int B, int H, int D, int S, int NB, int partition,
+                               int max_seq_len, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Paged prefill attention ("vLLM KV Cache and PagedAttention Explained", Step 6

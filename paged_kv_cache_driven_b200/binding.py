@@ -48,6 +48,9 @@ _SIGNATURES = {
     "pa_decode_fp8": ([_vp, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _i32,
                        _vp, ctypes.c_float, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz,
                        _vp], _i32),
+    "pa_decode_append_fp8": ([_vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, ctypes.c_float,
+                              ctypes.c_float, _vp, _i32, _vp, ctypes.c_float, _i32, _i32, _i32,
+                              _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     # out, out_dt, q, k_cache, v_cache, block_tables, MB, seq_lens, q_start, scale,
     # B, H, Hkv, D, S, NB, dt, T, max_q_len, stream
     "pa_prefill": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, ctypes.c_float, _i32, _i32,
@@ -318,6 +321,33 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_
                                MB, _ptr(seq_lens), float(scale), B, H, D, S, NB, int(partition),
                                int(max_seq_len), _ptr(workspace), ws_bytes, _stream(stream)),
            "pa_decode_fp8")
+
+
+def pa_decode_append_fp8(out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_tables,
+                         seq_lens, scale, max_seq_len, partition=0, workspace=None, stream=None):
+    """pa_kv_append_fp8 of k_new / v_new [B, H, D] at each request's last position,
+    then pa_decode_fp8, in one launch (same bits as the two calls)."""
+    for n, t in (("out", out), ("q", q), ("k_new", k_new), ("v_new", v_new),
+                 ("k_cache", k_cache), ("v_cache", v_cache), ("block_tables", block_tables),
+                 ("seq_lens", seq_lens)):
+        _cuda(t, n)
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise ValueError("E4M3 caches are uint8 tensors of codes")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    B, H, D = q.shape
+    NB, H2, S, _ = k_cache.shape
+    if H2 != H or tuple(k_new.shape) != (B, H, D) or tuple(v_new.shape) != (B, H, D):
+        raise ValueError("k_new / v_new must be [B, H, D] with one KV head per query head")
+    if k_new.dtype != q.dtype or v_new.dtype != q.dtype:
+        raise ValueError("k_new / v_new must have q's dtype")
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_decode_append_fp8(
+        _ptr(out), _DT[out.dtype], _ptr(q), _DT[q.dtype], _ptr(k_new), _ptr(v_new),
+        _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale), _ptr(block_tables), MB,
+        _ptr(seq_lens), float(scale), B, H, D, S, NB, int(partition), int(max_seq_len),
+        _ptr(workspace), ws_bytes, _stream(stream)), "pa_decode_append_fp8")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

@@ -462,11 +462,14 @@ pa_status pa_kv_append_fp8(const void* k, const void* v, pa_dtype in_dt,
                                         v_scale, T, H, D, S, NB, static_cast<cudaStream_t>(stream));
 }
 
-pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
-                        const void* k_cache, const void* v_cache, float k_scale, float v_scale,
-                        const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
-                        int B, int H, int D, int S, int NB, int partition, int max_seq_len,
-                        void* workspace, size_t ws_bytes, void* stream) {
+// pa_decode_fp8 and pa_decode_append_fp8: k_new / v_new null = plain decode.
+static pa_status decode_fp8_impl(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
+                                 const void* k_new, const void* v_new, const void* k_cache,
+                                 const void* v_cache, float k_scale, float v_scale,
+                                 const int32_t* block_tables, int MB, const int32_t* seq_lens,
+                                 float scale, int B, int H, int D, int S, int NB, int partition,
+                                 int max_seq_len, void* workspace, size_t ws_bytes,
+                                 void* stream) {
   if (B < 0 || H <= 0 || NB < 0 || MB < 0) return PA_ERR_INVALID;
   if (!cache_dtype_ok(q_dt) || !out_dtype_ok(out_dt) || !decode_shape_ok(D, S)) return PA_ERR_INVALID;
   if (!std::isfinite(scale)) return PA_ERR_INVALID;
@@ -505,9 +508,35 @@ pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt
     prm.NP = 1;
     prm.L_cap = static_cast<int>(L_max);
   }
+  const bool append = k_new != nullptr;
+  if (append && (!v_new || !aligned16(k_new) || !aligned16(v_new))) return PA_ERR_INVALID;
+  prm.k_new = k_new;
+  prm.v_new = v_new;
   const bool cluster = partition == 0 && cluster_merge(B, H, prm.NP);
-  return pa::host::launch_decode_fp8(prm, q_dt, out_dt, D, S, cluster,
+  return pa::host::launch_decode_fp8(prm, q_dt, out_dt, D, S, cluster, append, k_scale,
                                      static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
+                        const void* k_cache, const void* v_cache, float k_scale, float v_scale,
+                        const int32_t* block_tables, int MB, const int32_t* seq_lens, float scale,
+                        int B, int H, int D, int S, int NB, int partition, int max_seq_len,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  return decode_fp8_impl(out, out_dt, q, q_dt, nullptr, nullptr, k_cache, v_cache, k_scale,
+                         v_scale, block_tables, MB, seq_lens, scale, B, H, D, S, NB, partition,
+                         max_seq_len, workspace, ws_bytes, stream);
+}
+
+pa_status pa_decode_append_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
+                               const void* k_new, const void* v_new, void* k_cache,
+                               void* v_cache, float k_scale, float v_scale,
+                               const int32_t* block_tables, int MB, const int32_t* seq_lens,
+                               float scale, int B, int H, int D, int S, int NB, int partition,
+                               int max_seq_len, void* workspace, size_t ws_bytes, void* stream) {
+  if (B > 0 && (!k_new || !v_new)) return PA_ERR_INVALID;
+  return decode_fp8_impl(out, out_dt, q, q_dt, B > 0 ? k_new : nullptr, v_new, k_cache, v_cache,
+                         k_scale, v_scale, block_tables, MB, seq_lens, scale, B, H, D, S, NB,
+                         partition, max_seq_len, workspace, ws_bytes, stream);
 }
 
 pa_status pa_get_device_error(void* stream, uint32_t* flags) {

@@ -102,12 +102,31 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[NV], int lane) {
   return r;
 }
 
-// Raw 16-bit row fragment of 8 elements (16 bytes) for copying K/V rows bit for bit.
+// A 16-byte row fragment for copying K/V rows bit for bit (8 16-bit elements,
+// or 16 E4M3 codes).
 struct RawFrag {
   uint4 w;
   __device__ __forceinline__ void load(const void* src) { w = *reinterpret_cast<const uint4*>(src); }
   __device__ __forceinline__ void store(void* dst) const { *reinterpret_cast<uint4*>(dst) = w; }
 };
+
+// The E4M3 codes of EL consecutive 16-bit elements (EL = 2, 4 or 8, packed in
+// x), each the code of fp32(x / scale) (one correctly rounded division, round
+// to nearest even, saturated at 448): the rule of kv_append_fp8_kernel, so the
+// fused append stores the same bytes as pa_kv_append_fp8. Codes in element
+// order, the first in the lowest byte.
+template <typename T, int EL>
+__device__ __forceinline__ void quantize_e4m3(const uint32_t (&x)[EL / 2], float scale,
+                                              uint32_t (&codes)[(EL + 3) / 4]) {
+#pragma unroll
+  for (int j = 0; j < (EL + 3) / 4; ++j) codes[j] = 0;
+#pragma unroll
+  for (int e = 0; e < EL / 2; ++e) {
+    const float2 f = Elem<T>::pair(x[e]);
+    const uint32_t c = float2_to_e4m3x2(__fdiv_rn(f.x, scale), __fdiv_rn(f.y, scale));
+    codes[e / 2] |= c << (16 * (e & 1));
+  }
+}
 
 // One CTA per (partition, head, request); NW warps, each an independent
 // pipeline over the tokens of a contiguous run of the partition's blocks,
@@ -117,7 +136,8 @@ struct RawFrag {
 // new token (position L - 1) takes its K/V from k_new / v_new. The warp whose
 // run holds that token copies the row into its staged unit once the bulk copy
 // has landed (so the scores see it) and stores it to the cache, as
-// pa_kv_append would have before the decode.
+// pa_kv_append would have before the decode. Over an E4M3 cache (Prm =
+// DecodeParamsQ8) the row is first quantized as pa_kv_append_fp8 does.
 //
 // TC is the cache element type: T itself, or E4M3 codes with per-tensor
 // scales (K's folded into q_scale, V's applied to the accumulated output).
@@ -127,11 +147,12 @@ struct RawFrag {
 // workspace. (A template parameter, so that the plain form's code is not
 // touched by it.)
 template <typename T, typename TO, int D, int S, bool APPEND, typename TC = T,
-          bool CLUSTER = false>
+          bool CLUSTER = false, typename Prm = DecodeParams>
 __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
-    paged_decode_partition_kernel(const DecodeParams p) {
+    paged_decode_partition_kernel(const Prm p) {
   constexpr int EB = sizeof(TC);
-  static_assert(!APPEND || EB == 2, "the fused append copies 16-bit rows");
+  static_assert(!APPEND || EB == 2 || std::is_same<Prm, DecodeParamsQ8>::value,
+                "the fused append over an E4M3 cache needs K's scale");
   using Tl = DecodeTiling<D, S, EB>;
   constexpr int NW = Tl::NW, NS = Tl::NS, SLAB = Tl::SLAB, UNIT = Tl::UNIT, STAGE = Tl::STAGE;
   constexpr int EPL = Tl::EPL, LPR = Tl::LPR, RPW = Tl::RPW, CR = Tl::CR, NV = Tl::NV;
@@ -149,6 +170,16 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
   const int i = blockIdx.z;
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
+  if constexpr (APPEND && EB == 1) {
+    // the new rows (D 16-bit elements each), wanted by whichever warp turns out
+    // to own the new token: have L2 fetch them while the length is read
+    // (one KV head per query head here: the row of (i, h); D * 2 bytes, D / 64 lines)
+    if (threadIdx.x < D / 64) {
+      const int64_t row = ((static_cast<int64_t>(i) * p.H + h) * D) * 2 + threadIdx.x * 128;
+      prefetch_l2(static_cast<const uint8_t*>(p.k_new) + row);
+      prefetch_l2(static_cast<const uint8_t*>(p.v_new) + row);
+    }
+  }
   const int g = lane / LPR;   // row group
   const int pl = lane % LPR;  // position in the row: elements pl * EPL .. pl * EPL + EPL - 1
 
@@ -243,12 +274,60 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
   const bool appender = APPEND && len_ok && L >= 1 && t_new >= wt0 && t_new < wt1;
   RawFrag k_row, v_row;
   int id_new = -1;
-  if (appender && g == 0) {
+  // E4M3 cache: every lane of the appender warp takes EL = D / 32 elements of
+  // the new rows (16-bit), and quantizes and stores them itself
+  constexpr int EL = D / 32;
+  uint32_t k_raw[EB == 1 ? EL / 2 : 1], v_raw[EB == 1 ? EL / 2 : 1];
+  if constexpr (APPEND && EB == 1) {
+    if (appender) {
+      const int64_t off = ((static_cast<int64_t>(i) * p.Hkv + hk) * D + lane * EL) * 2;
+#pragma unroll
+      for (int e = 0; e < EL / 2; ++e) {
+        k_raw[e] = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.k_new) + off)[e];
+        v_raw[e] = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.v_new) + off)[e];
+      }
+      id_new = __ldg(trow + t_new / S);
+    }
+  } else if (appender && g == 0) {
+    // the new rows are 16-bit: EPL elements, EPL * 2 bytes, per lane
     const int64_t off = ((static_cast<int64_t>(i) * p.Hkv + hk) * D + pl * EPL) * 2;
     k_row.load(static_cast<const uint8_t*>(p.k_new) + off);
     v_row.load(static_cast<const uint8_t*>(p.v_new) + off);
     id_new = __ldg(trow + t_new / S);
   }
+  // E4M3 cache: the new token sits in the appender's last unit. Its codes go to
+  // the cache just before that unit's bulk copy is issued (after the warp's
+  // earlier copies, so the loads and the quantization overlap their flight),
+  // and the copy brings them; the proxy fence orders the generic-proxy stores
+  // before lane 0's async-proxy read. The pipeline loop then runs as without
+  // the append. (A block id out of range stores nothing; its unit is flagged
+  // when issued.)
+  const int k_new_unit = appender ? (t_new - wt0) / CR : -1;
+  auto store_new_rows = [&]() {
+    if constexpr (APPEND && EB == 1) {
+      uint32_t kc[(EL + 3) / 4], vc[(EL + 3) / 4];
+      quantize_e4m3<T, EL>(k_raw, p.k_scale, kc);
+      quantize_e4m3<T, EL>(v_raw, p.v_scale, vc);
+      if (static_cast<unsigned>(id_new) < static_cast<unsigned>(p.NB)) {
+        const int64_t goff = static_cast<int64_t>(id_new) * block_stride +
+                             static_cast<int64_t>(t_new % S) * D + lane * EL;
+        uint8_t* kd = const_cast<uint8_t*>(kbase) + goff;
+        uint8_t* vd = const_cast<uint8_t*>(vbase) + goff;
+        if constexpr (EL == 2) {
+          *reinterpret_cast<uint16_t*>(kd) = static_cast<uint16_t>(kc[0]);
+          *reinterpret_cast<uint16_t*>(vd) = static_cast<uint16_t>(vc[0]);
+        } else if constexpr (EL == 4) {
+          *reinterpret_cast<uint32_t*>(kd) = kc[0];
+          *reinterpret_cast<uint32_t*>(vd) = vc[0];
+        } else {
+          *reinterpret_cast<uint2*>(kd) = make_uint2(kc[0], kc[1]);
+          *reinterpret_cast<uint2*>(vd) = make_uint2(vc[0], vc[1]);
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
+      __syncwarp();
+    }
+  };
 
   // Block-id prefetch: ids_a holds the table entries of blocks wb + base .. +31,
   // ids_b the next 32.
@@ -288,7 +367,15 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
   };
 
 #pragma unroll
-  for (int k = 0; k < NS; ++k) issue_next();
+  for (int k = 0; k < NS; ++k) {
+    if constexpr (APPEND && EB == 1) {
+      if (issued == k_new_unit) store_new_rows();  // warp-uniform
+    }
+    issue_next();
+  }
+  if constexpr (APPEND && EB == 1) {
+    if (issued <= k_new_unit) store_new_rows();  // that unit is issued in the loop below
+  }
 
   float m = -INFINITY;  // running max (base-2 units), warp-uniform
   float lsum = 0.f;     // running sum of 2^(s - m); one lane per row counts it
@@ -310,15 +397,15 @@ __global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
       const int nvalid = min(CR, L - t0);
       uint8_t* ks = stage0 + s * STAGE;
       uint8_t* vs = ks + UNIT;
-      if (APPEND && appender && t_new >= t0 && t_new < t0 + CR) {
+      if (APPEND && EB == 2 && appender && t_new >= t0 && t_new < t0 + CR) {
         // the bulk copy brought the old bytes; put the new token's row in both
         // the staged unit and the cache
         if (g == 0) {
-          const int64_t row_off = (static_cast<int64_t>(t_new - t0) * D + pl * EPL) * 2;
+          const int64_t row_off = (static_cast<int64_t>(t_new - t0) * D + pl * EPL) * EB;
           k_row.store(ks + row_off);
           v_row.store(vs + row_off);
           const int64_t goff = static_cast<int64_t>(id_new) * block_stride +
-                               (static_cast<int64_t>(t_new % S) * D + pl * EPL) * 2;
+                               (static_cast<int64_t>(t_new % S) * D + pl * EPL) * EB;
           k_row.store(const_cast<uint8_t*>(kbase) + goff);
           v_row.store(const_cast<uint8_t*>(vbase) + goff);
           // these generic-proxy writes must be ordered before the next bulk
@@ -575,10 +662,10 @@ inline cudaError_t launch_splitkv_reduce(const DecodeParams& p, cudaStream_t str
 // Launches the partition pass (grid NP x H x B) and the merge: `kern_cl` in
 // clusters of NP CTAs that merge among themselves (dynamic shared memory
 // smem_cl), or `kern` as a plain grid (smem) followed by the merge kernel.
-template <typename TO, int D, typename Kern>
-inline cudaError_t launch_partition_pass(Kern kern, Kern kern_cl, bool cluster,
-                                         const DecodeParams& p, int threads, int smem,
-                                         int smem_cl, cudaStream_t stream) {
+template <typename TO, int D, typename Kern, typename Prm>
+inline cudaError_t launch_partition_pass(Kern kern, Kern kern_cl, bool cluster, const Prm& p,
+                                         int threads, int smem, int smem_cl,
+                                         cudaStream_t stream) {
   const dim3 grid(p.NP, p.H, p.B);
   if (cluster) {
     cudaLaunchConfig_t cfg = {};

@@ -95,6 +95,11 @@ __device__ __forceinline__ void grid_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Asks L2 to fetch the 128-byte line at p (no register result, no wait).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Thread-block clusters. The cluster barrier is split: every thread of every
 // CTA of the cluster arrives, then waits until all have arrived (non-.aligned
 // forms, so a warp need not be converged). A relaxed arrival orders nothing;

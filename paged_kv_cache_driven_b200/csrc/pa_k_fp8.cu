@@ -1,6 +1,7 @@
-// Kernels of pa_decode_fp8: the partition pass over E4M3 caches (one-byte
-// cache elements, per-tensor scales) and the split-KV merge, with their
-// launcher.
+// Kernels of pa_decode_fp8 and pa_decode_append_fp8: the partition pass over
+// E4M3 caches (one-byte cache elements, per-tensor scales; with or without the
+// quantized fused append, plain or in clusters) and the split-KV merge, with
+// their launcher.
 
 #include <type_traits>
 
@@ -11,12 +12,13 @@ namespace pa {
 namespace host {
 namespace {
 
-// One CTA per (partition, head, request).
-template <typename T, typename TO, int D, int S>
-pa_status launch(const DecodeParams& prm, bool cluster, cudaStream_t stream) {
+// One CTA per (partition, head, request). Prm: DecodeParams, or DecodeParamsQ8
+// for the fused append (APPEND).
+template <typename T, typename TO, int D, int S, bool APPEND, typename Prm>
+pa_status launch(const Prm& prm, bool cluster, cudaStream_t stream) {
   using Tl = DecodeTiling<D, S, 1>;
-  auto kern = paged_decode_partition_kernel<T, TO, D, S, false, __nv_fp8_e4m3>;
-  auto kern_cl = paged_decode_partition_kernel<T, TO, D, S, false, __nv_fp8_e4m3, true>;
+  auto kern = paged_decode_partition_kernel<T, TO, D, S, APPEND, __nv_fp8_e4m3, false, Prm>;
+  auto kern_cl = paged_decode_partition_kernel<T, TO, D, S, APPEND, __nv_fp8_e4m3, true, Prm>;
   static bool configured[kMaxDevices] = {}, configured_cl[kMaxDevices] = {};
   if (!opt_in_smem(kern, Tl::SMEM, configured) ||
       !opt_in_smem(kern_cl, Tl::SMEM_CL, configured_cl))
@@ -27,10 +29,10 @@ pa_status launch(const DecodeParams& prm, bool cluster, cudaStream_t stream) {
   return cuda_status();
 }
 
-template <typename T, typename TO>
-pa_status by_shape(const DecodeParams& prm, int D, int S, bool cl, cudaStream_t st) {
+template <typename T, typename TO, bool APPEND, typename Prm>
+pa_status by_shape(const Prm& prm, int D, int S, bool cl, cudaStream_t st) {
 #define PA_CASE(DD, SS) \
-  if (D == DD && S == SS) return launch<T, TO, DD, SS>(prm, cl, st);
+  if (D == DD && S == SS) return launch<T, TO, DD, SS, APPEND>(prm, cl, st);
   PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32)
   PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32)
   PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32)
@@ -38,23 +40,33 @@ pa_status by_shape(const DecodeParams& prm, int D, int S, bool cl, cudaStream_t 
   return PA_ERR_INVALID;
 }
 
-template <typename T>
-pa_status by_out(const DecodeParams& prm, pa_dtype out_dt, int D, int S, bool cl,
-                 cudaStream_t st) {
+template <typename T, bool APPEND, typename Prm>
+pa_status by_out(const Prm& prm, pa_dtype out_dt, int D, int S, bool cl, cudaStream_t st) {
   switch (out_dt) {
-    case PA_F32: return by_shape<T, float>(prm, D, S, cl, st);
-    case PA_F16: return by_shape<T, __half>(prm, D, S, cl, st);
-    case PA_BF16: return by_shape<T, __nv_bfloat16>(prm, D, S, cl, st);
+    case PA_F32: return by_shape<T, float, APPEND>(prm, D, S, cl, st);
+    case PA_F16: return by_shape<T, __half, APPEND>(prm, D, S, cl, st);
+    case PA_BF16: return by_shape<T, __nv_bfloat16, APPEND>(prm, D, S, cl, st);
   }
   return PA_ERR_INVALID;
+}
+
+template <bool APPEND, typename Prm>
+pa_status by_q(const Prm& prm, pa_dtype q_dt, pa_dtype out_dt, int D, int S, bool cl,
+               cudaStream_t st) {
+  return q_dt == PA_F16 ? by_out<__half, APPEND>(prm, out_dt, D, S, cl, st)
+                        : by_out<__nv_bfloat16, APPEND>(prm, out_dt, D, S, cl, st);
 }
 
 }  // namespace
 
 pa_status launch_decode_fp8(const DecodeParams& prm, pa_dtype q_dt, pa_dtype out_dt, int D,
-                            int S, bool cluster, cudaStream_t stream) {
-  return q_dt == PA_F16 ? by_out<__half>(prm, out_dt, D, S, cluster, stream)
-                        : by_out<__nv_bfloat16>(prm, out_dt, D, S, cluster, stream);
+                            int S, bool cluster, bool append, float k_scale,
+                            cudaStream_t stream) {
+  if (!append) return by_q<false>(prm, q_dt, out_dt, D, S, cluster, stream);
+  DecodeParamsQ8 q8;
+  static_cast<DecodeParams&>(q8) = prm;
+  q8.k_scale = k_scale;
+  return by_q<true>(q8, q_dt, out_dt, D, S, cluster, stream);
 }
 
 bool take_error_fp8(unsigned int* bits) { return take_error_word(bits); }

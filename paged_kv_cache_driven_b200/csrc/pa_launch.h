@@ -36,6 +36,14 @@ struct DecodeParams {
   float v_scale;  // V = v_scale * stored value (1 for 16-bit caches; E4M3 caches)
 };
 
+// The parameters of the FP8 fused append (pa_decode_append_fp8): K's
+// per-tensor scale, which the quantizer divides by (q_scale holds it folded
+// with the softmax scale). A type of its own, so that the other kernels'
+// parameter block stays as it is.
+struct DecodeParamsQ8 : DecodeParams {
+  float k_scale;
+};
+
 struct PrefillParams {
   void* out;                    // [T, H, D] TO
   const void* k_cache;          // [NB, Hkv, S, D] T
@@ -83,8 +91,11 @@ pa_status launch_decode16(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt,
                           bool append, bool cluster, cudaStream_t stream);  // pa_k_decode.cu
 pa_status launch_grouped(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt, int D, int S,
                          bool append, cudaStream_t stream);             // pa_k_gqa.cu
+// append: the new tokens' rows (prm.k_new / v_new, dtype q_dt) are quantized
+// with k_scale and prm.v_scale and written into the caches inside the launch.
 pa_status launch_decode_fp8(const DecodeParams& prm, pa_dtype q_dt, pa_dtype out_dt, int D,
-                            int S, bool cluster, cudaStream_t stream);  // pa_k_fp8.cu
+                            int S, bool cluster, bool append, float k_scale,
+                            cudaStream_t stream);                       // pa_k_fp8.cu
 pa_status launch_prefill(const PrefillParams& prm, const void* q, pa_dtype dt, pa_dtype out_dt,
                          int D, int S, cudaStream_t stream);            // pa_k_prefill.cu
 pa_status launch_kv_append(const void* k, const void* v, const int64_t* slots, void* k_cache,

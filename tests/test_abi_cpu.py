@@ -146,7 +146,7 @@ def prefill_args(**kw):
     dict(D=96), dict(D=256), dict(S=4), dict(S=256), dict(dt=binding.PA_F32), dict(out_dt=9),
     dict(scale=0.0), dict(scale=-1.0), dict(scale=float("nan")), dict(Hkv=3), dict(Hkv=0),
     dict(q=NULL), dict(qs=NULL), dict(bt=NULL), dict(out=ctypes.c_void_p(16 * 1024 + 4)),
-    dict(NB=0), dict(NB=1 << 28), dict(T=-1), dict(max_q_len=-1), dict(B=-1),
+    dict(NB=0), dict(NB=1 << 28), dict(T=-1), dict(max_q_len=-1), dict(B=-1), dict(B=65536),
 ])
 def test_prefill_rejects_bad_arguments_on_host(lib, bad):
     assert lib.pa_prefill(*prefill_args(**bad)) == binding.PA_ERR_INVALID
@@ -178,6 +178,25 @@ def test_decode_fp8_rejects_bad_arguments_on_host(lib, bad):
 
 def test_decode_fp8_zero_batch_is_noop(lib):
     assert lib.pa_decode_fp8(*fp8_decode_args(B=0, q=NULL, out=NULL)) == binding.PA_OK
+
+
+def fp8_decode_append_args(kn=P, vn=P, **kw):
+    a = fp8_decode_args(**kw)
+    return a[:4] + [kn, vn] + a[4:]  # k_new, v_new after q_dt
+
+
+@pytest.mark.parametrize("bad", [
+    dict(kn=NULL), dict(vn=NULL), dict(kn=ctypes.c_void_p(16 * 1024 + 8)),
+    dict(vn=ctypes.c_void_p(16 * 1024 + 2)), dict(ks=0.0), dict(D=96), dict(k=NULL),
+    dict(q_dt=binding.PA_F32), dict(max_seq_len=100, partition=16),
+])
+def test_decode_append_fp8_rejects_bad_arguments_on_host(lib, bad):
+    assert lib.pa_decode_append_fp8(*fp8_decode_append_args(**bad)) == binding.PA_ERR_INVALID
+
+
+def test_decode_append_fp8_zero_batch_is_noop(lib):
+    args = fp8_decode_append_args(kn=NULL, vn=NULL, B=0, q=NULL, out=NULL)
+    assert lib.pa_decode_append_fp8(*args) == binding.PA_OK
 
 
 def fp8_append_args(**kw):

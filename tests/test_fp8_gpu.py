@@ -170,3 +170,53 @@ def test_decode_fp8_bad_block_id_is_skipped_and_flagged():
     assert binding.pa_get_device_error() & binding.PA_DEVERR_BLOCK_ID
     assert_parity(out[1:].cpu().numpy(), want[1:], "fp8 neighbour of a bad id")
     assert bool(torch.isfinite(out[0]).all())
+
+
+@pytest.mark.parametrize("lens,H,D,S,in_dt,out_dt,partition", [
+    ([0, 1, 17, 300, 1000], 3, 128, 16, torch.bfloat16, torch.float32, 0),
+    ([0, 1, 17, 300, 1000], 3, 128, 16, torch.bfloat16, torch.float32, -1),
+    ([5, 64, 333], 2, 64, 8, torch.float16, torch.bfloat16, 32),
+    ([7, 129, 700], 2, 256, 32, torch.bfloat16, torch.float16, 64),
+    ([1332], 32, 128, 16, torch.bfloat16, torch.float32, 0),  # a cluster plan: 8 x 176 tokens
+])
+def test_decode_append_fp8_equals_two_calls(lens, H, D, S, in_dt, out_dt, partition):
+    """pa_decode_append_fp8 quantizes each request's new row into its last slot
+    inside the decode launch: the same cache bytes as pa_kv_append_fp8 (and as
+    the oracle's quantizer), the same output bits as pa_kv_append_fp8 followed
+    by pa_decode_fp8, and the oracle's decode of those codes."""
+    case, kc8, vc8 = fp8_case(lens, H=H, D=D, S=S, in_dt=in_dt, seed=sum(lens) + D)
+    B = len(lens)
+    g = torch.Generator(device=DEV).manual_seed(D + S)
+    k_new = (torch.randn((B, H, D), generator=g, device=DEV) * 4).to(in_dt)
+    v_new = (torch.randn((B, H, D), generator=g, device=DEV) * 4).to(in_dt)
+    k_new[-1, 0, :3] = torch.tensor([1e4, -1e4, 0.0], device=DEV).to(in_dt)  # saturation
+    slots = torch.tensor([case.tables_host[i][(L - 1) // S] * S + (L - 1) % S if L > 0 else -1
+                          for i, L in enumerate(lens)], dtype=torch.int64, device=DEV)
+    kc_a, vc_a = kc8.clone(), vc8.clone()
+    binding.pa_kv_append_fp8(k_new, v_new, slots, kc_a, vc_a, 0.05, 0.08)
+    out_a = run_fp8(case, kc_a, vc_a, out_dt=out_dt, partition=partition)
+    kc_b, vc_b = kc8.clone(), vc8.clone()
+    maxlen = max(lens)
+    out_b = torch.empty((B, H, D), dtype=out_dt, device=DEV)
+    wsb = binding.pa_decode_workspace_bytes(B, H, D, S, maxlen, partition)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=DEV)
+    binding.pa_decode_append_fp8(out_b, case.q, k_new, v_new, kc_b, vc_b, 0.05, 0.08,
+                                 case.block_tables, case.seq_lens, case.scale, maxlen,
+                                 partition=partition, workspace=ws)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    assert torch.equal(kc_a, kc_b) and torch.equal(vc_a, vc_b), "cache bytes differ"
+    bits = torch.int32 if out_dt == torch.float32 else torch.int16
+    assert torch.equal(out_a.view(bits), out_b.view(bits)), "output bits differ"
+    # the appended codes are the oracle quantizer's
+    kq = ofp8.quantize(k_new.float().cpu().numpy(), 0.05)
+    vq = ofp8.quantize(v_new.float().cpu().numpy(), 0.08)
+    kcb, vcb = kc_b.cpu().numpy(), vc_b.cpu().numpy()
+    for i, s in enumerate(slots.tolist()):
+        if s >= 0:
+            assert np.array_equal(kcb[s // S, :, s % S, :], kq[i])
+            assert np.array_equal(vcb[s // S, :, s % S, :], vq[i])
+    if out_dt == torch.float32:
+        want = ofp8.paged_decode_fp8(case.q.cpu(), kc_b.cpu(), vc_b.cpu(), 0.05, 0.08,
+                                     case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
+        assert_parity(out_b.cpu().numpy(), want, f"fused fp8 append {lens} D={D}")
