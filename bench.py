@@ -565,6 +565,45 @@ def time_decode_fp8(seed, iters, warmup):
     return ms, nbytes, binding.pa_decode_plan(B, Hc, Dc, Sc, maxlen, 0), ms_fused
 
 
+def time_decode_gqa_fp8(seed, iters, warmup):
+    """The LLaMA-2-70B decode shape (64 query heads on 8 KV heads) over an E4M3
+    cache filled by pa_kv_append_fp8 from the bf16 case: median event-timed
+    pa_decode_gqa_fp8 call with L2 flushed before each; returns (ms, KV bytes,
+    plan)."""
+    device = torch.device("cuda", 0)
+    case = workloads.llama70b_decode(seed=seed, device=device)
+    B, Hq, Dc = case.q.shape
+    NB, Hkv, Sc, _ = case.k_cache.shape
+    kc8 = torch.empty((NB, Hkv, Sc, Dc), dtype=torch.uint8, device=device)
+    vc8 = torch.empty_like(kc8)
+    slots = torch.arange(NB * Sc, dtype=torch.int64, device=device)
+    binding.pa_kv_append_fp8(case.k_cache.permute(0, 2, 1, 3).reshape(-1, Hkv, Dc).contiguous(),
+                             case.v_cache.permute(0, 2, 1, 3).reshape(-1, Hkv, Dc).contiguous(),
+                             slots, kc8, vc8, 0.05, 0.08)
+    del case.k_cache, case.v_cache
+    maxlen = max(case.seq_lens_host)
+    out = torch.empty((B, Hq, Dc), dtype=DTYPE, device=device)
+    wsb = binding.pa_decode_workspace_bytes(B, Hq, Dc, Sc, maxlen, 0)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
+    times = []
+    for k in range(warmup + iters):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        binding.pa_decode_gqa_fp8(out, case.q, kc8, vc8, 0.05, 0.08, case.block_tables,
+                                  case.seq_lens, case.scale, maxlen, partition=0, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        if k >= warmup:
+            times.append(a.elapsed_time(b))
+    if binding.pa_get_device_error():
+        raise SystemExit("device error word set")
+    nbytes = sum(Hkv * 2 * L * Dc + Hq * 2 * Dc * 2 + 4 * (-(-L // Sc))
+                 for L in case.seq_lens_host) + 4 * B
+    return statistics.median(times), nbytes, binding.pa_decode_plan(B, Hq, Dc, Sc, maxlen, 0)
+
+
 def latency_floors(device, iters, warmup):
     """The small-batch floor, timed like the sweep's calls (L2 flushed, events
     around the call): a launch of a one-element fill (a kernel that does
@@ -617,6 +656,15 @@ def run_shape_workloads(args):
     elif args.workload == "llama70b":
         cases = [("llama70b_gqa_64q_8kv", lambda: workloads.llama70b_decode(seed=args.seed,
                                                                             device=device))]
+    elif args.workload == "llama70b_fp8":
+        ms, nbytes, plan = time_decode_gqa_fp8(args.seed, args.steps, args.warmup)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        print(json.dumps({"workload": "llama70b_gqa_64q_8kv_fp8_e4m3_cache", "ms": round(ms, 4),
+                          "gb_s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 3),
+                          "kv_bytes": nbytes, "tok_s_layer": round(64 / (ms / 1e3), 1),
+                          "partition": {"tokens": plan[0], "num": plan[1]},
+                          "l2": L2_FLUSHED}), flush=True)
+        return
     else:
         cases = []
         for Sx in (8, 16, 32):
@@ -1177,7 +1225,8 @@ def main():
     ap.add_argument("--case", default=None,
                     help="with --workload sweep: time only this case (e.g. S16_D128_B1_bf16)")
     ap.add_argument("--workload", default="llama13b",
-                    choices=["llama13b", "long_context", "sweep", "llama70b", "llama13b_fp8",
+                    choices=["llama13b", "long_context", "sweep", "llama70b", "llama70b_fp8",
+                             "llama13b_fp8",
                              "prompt_prefill", "prompt_prefill_small", "worked_example",
                              "prefill_append", "prefill_append_small", "batching",
                              "prefill_trace"],

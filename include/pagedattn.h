@@ -201,6 +201,21 @@ pa_status pa_decode_append_fp8(void* out, pa_dtype out_dt, const void* q, pa_dty
                                float scale, int B, int H, int D, int S, int NB, int partition,
                                int max_seq_len, void* workspace, size_t ws_bytes, void* stream);
 
+/* pa_decode_fp8 with grouped-query heads: H query heads share Hkv KV heads
+ * (H % Hkv == 0), query head h reading KV head h / (H / Hkv) of the E4M3 caches
+ * [NB, Hkv, S, D]. The products run on the tensor cores in f16 (E4M3 values
+ * are f16 values; each query head is held in f16 after an exact power-of-two
+ * scaling that keeps its largest element below 2^15, undone on its scores),
+ * with fp32 accumulation; the softmax weights enter P.V as f16. Hkv == H is
+ * pa_decode_fp8. Other arguments, workspace (pa_decode_workspace_bytes with H
+ * the query heads) and errors as pa_decode_fp8; no fused append. */
+pa_status pa_decode_gqa_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
+                            const void* k_cache, const void* v_cache, float k_scale,
+                            float v_scale, const int32_t* block_tables, int MB,
+                            const int32_t* seq_lens, float scale, int B, int H, int Hkv, int D,
+                            int S, int NB, int partition, int max_seq_len, void* workspace,
+                            size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Paged prefill attention ("vLLM KV Cache and PagedAttention Explained", Step 6
  * "Prefill and Decode": every prompt token is processed at once, and each one

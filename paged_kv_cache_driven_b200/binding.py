@@ -48,6 +48,9 @@ _SIGNATURES = {
     "pa_decode_fp8": ([_vp, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _i32,
                        _vp, ctypes.c_float, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz,
                        _vp], _i32),
+    "pa_decode_gqa_fp8": ([_vp, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp,
+                           _i32, _vp, ctypes.c_float, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                           _i32, _vp, _sz, _vp], _i32),
     "pa_decode_append_fp8": ([_vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, ctypes.c_float,
                               ctypes.c_float, _vp, _i32, _vp, ctypes.c_float, _i32, _i32, _i32,
                               _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
@@ -321,6 +324,28 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_
                                MB, _ptr(seq_lens), float(scale), B, H, D, S, NB, int(partition),
                                int(max_seq_len), _ptr(workspace), ws_bytes, _stream(stream)),
            "pa_decode_fp8")
+
+
+def pa_decode_gqa_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_lens, scale,
+                      max_seq_len, partition=0, workspace=None, stream=None):
+    """Decode over uint8 E4M3 caches [NB, Hkv, S, D] for q [B, H, D] with H a
+    multiple of Hkv (query head h reads KV head h // (H // Hkv))."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                 ("block_tables", block_tables), ("seq_lens", seq_lens)):
+        _cuda(t, n)
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise ValueError("E4M3 caches are uint8 tensors of codes")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    B, H, D = q.shape
+    NB, Hkv, S, _ = k_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_decode_gqa_fp8(_ptr(out), _DT[out.dtype], _ptr(q), _DT[q.dtype],
+                                   _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale),
+                                   _ptr(block_tables), MB, _ptr(seq_lens), float(scale), B, H, Hkv,
+                                   D, S, NB, int(partition), int(max_seq_len), _ptr(workspace),
+                                   ws_bytes, _stream(stream)), "pa_decode_gqa_fp8")
 
 
 def pa_decode_append_fp8(out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_tables,

@@ -173,8 +173,9 @@ struct RowMapKey {
 namespace pa {
 namespace host {
 
-// kind: 0 = f16, 1 = bf16; boxes of 64 elements, so every box row is 128 bytes,
-// the 128-byte swizzle's width.
+// kind: 0 = f16, 1 = bf16: boxes of 64 elements, so every box row is 128 bytes,
+// the 128-byte swizzle's width; 2 = one-byte E4M3 codes: a box spans the whole
+// D-byte row, unswizzled (the consumer converts it to 16-bit tiles itself).
 static bool row_map_kind(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows,
                          int kind) {
   static std::mutex mu;
@@ -190,16 +191,20 @@ static bool row_map_kind(CUtensorMap* out, const void* base, int64_t rows, int D
     }
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t esize = 2;
+  const bool codes = kind == 2;
+  const cuuint64_t esize = codes ? 1 : 2;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * esize};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(codes ? D : 128 / esize),
+                             static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType type =
-      kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+      codes ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+            : (kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   CUtensorMap map;
   if (fn(&map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_INTERLEAVE_NONE,
+         codes ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   const int slot = used < 16 ? used++ : next;
@@ -212,6 +217,10 @@ static bool row_map_kind(CUtensorMap* out, const void* base, int64_t rows, int D
 
 bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows, pa_dtype dt) {
   return row_map_kind(out, base, rows, D, box_rows, dt == PA_BF16 ? 1 : 0);
+}
+
+bool row_map_codes(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows) {
+  return row_map_kind(out, base, rows, D, box_rows, 2);
 }
 
 // ---- paged prefill -------------------------------------------------------------
@@ -463,14 +472,16 @@ pa_status pa_kv_append_fp8(const void* k, const void* v, pa_dtype in_dt,
 }
 
 // pa_decode_fp8 and pa_decode_append_fp8: k_new / v_new null = plain decode.
+// pa_decode_gqa_fp8: Hkv < H (grouped-query heads; no fused append).
 static pa_status decode_fp8_impl(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
                                  const void* k_new, const void* v_new, const void* k_cache,
                                  const void* v_cache, float k_scale, float v_scale,
                                  const int32_t* block_tables, int MB, const int32_t* seq_lens,
-                                 float scale, int B, int H, int D, int S, int NB, int partition,
-                                 int max_seq_len, void* workspace, size_t ws_bytes,
-                                 void* stream) {
+                                 float scale, int B, int H, int Hkv, int D, int S, int NB,
+                                 int partition, int max_seq_len, void* workspace,
+                                 size_t ws_bytes, void* stream) {
   if (B < 0 || H <= 0 || NB < 0 || MB < 0) return PA_ERR_INVALID;
+  if (Hkv <= 0 || H % Hkv != 0 || (k_new && Hkv != H)) return PA_ERR_INVALID;
   if (!cache_dtype_ok(q_dt) || !out_dtype_ok(out_dt) || !decode_shape_ok(D, S)) return PA_ERR_INVALID;
   if (!std::isfinite(scale)) return PA_ERR_INVALID;
   if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
@@ -499,7 +510,7 @@ static pa_status decode_fp8_impl(void* out, pa_dtype out_dt, const void* q, pa_d
   prm.MB = MB;
   prm.B = B;
   prm.H = H;
-  prm.Hkv = H;
+  prm.Hkv = Hkv;
   prm.NB = NB;
   if (NP > 1) {
     set_split(prm, workspace, B, H, P, NP, L_max);
@@ -508,6 +519,9 @@ static pa_status decode_fp8_impl(void* out, pa_dtype out_dt, const void* q, pa_d
     prm.NP = 1;
     prm.L_cap = static_cast<int>(L_max);
   }
+  if (Hkv != H)  // grouped-query heads: the tensor-core kernel
+    return pa::host::launch_grouped_fp8(prm, q_dt, out_dt, D, S,
+                                        static_cast<cudaStream_t>(stream));
   const bool append = k_new != nullptr;
   if (append && (!v_new || !aligned16(k_new) || !aligned16(v_new))) return PA_ERR_INVALID;
   prm.k_new = k_new;
@@ -523,8 +537,19 @@ pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt
                         int B, int H, int D, int S, int NB, int partition, int max_seq_len,
                         void* workspace, size_t ws_bytes, void* stream) {
   return decode_fp8_impl(out, out_dt, q, q_dt, nullptr, nullptr, k_cache, v_cache, k_scale,
-                         v_scale, block_tables, MB, seq_lens, scale, B, H, D, S, NB, partition,
-                         max_seq_len, workspace, ws_bytes, stream);
+                         v_scale, block_tables, MB, seq_lens, scale, B, H, H, D, S, NB,
+                         partition, max_seq_len, workspace, ws_bytes, stream);
+}
+
+pa_status pa_decode_gqa_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
+                            const void* k_cache, const void* v_cache, float k_scale,
+                            float v_scale, const int32_t* block_tables, int MB,
+                            const int32_t* seq_lens, float scale, int B, int H, int Hkv, int D,
+                            int S, int NB, int partition, int max_seq_len, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  return decode_fp8_impl(out, out_dt, q, q_dt, nullptr, nullptr, k_cache, v_cache, k_scale,
+                         v_scale, block_tables, MB, seq_lens, scale, B, H, Hkv, D, S, NB,
+                         partition, max_seq_len, workspace, ws_bytes, stream);
 }
 
 pa_status pa_decode_append_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,
@@ -535,7 +560,7 @@ pa_status pa_decode_append_fp8(void* out, pa_dtype out_dt, const void* q, pa_dty
                                int max_seq_len, void* workspace, size_t ws_bytes, void* stream) {
   if (B > 0 && (!k_new || !v_new)) return PA_ERR_INVALID;
   return decode_fp8_impl(out, out_dt, q, q_dt, B > 0 ? k_new : nullptr, v_new, k_cache, v_cache,
-                         k_scale, v_scale, block_tables, MB, seq_lens, scale, B, H, D, S, NB,
+                         k_scale, v_scale, block_tables, MB, seq_lens, scale, B, H, H, D, S, NB,
                          partition, max_seq_len, workspace, ws_bytes, stream);
 }
 

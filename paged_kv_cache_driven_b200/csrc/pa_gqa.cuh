@@ -28,11 +28,13 @@
 
 namespace pa {
 
-template <int D>
+template <int D, int EB = 2>
 struct GqaTiling {
   static constexpr int ROWS = 16;               // tokens per unit = one MMA k-step of P V
   static constexpr int BOX = 16 * 128;          // one swizzled box: 16 rows x 64 elements
-  static constexpr int TILE = (D / 64) * BOX;   // one K (or V) unit
+  static constexpr int TILE16 = (D / 64) * BOX; // one K (or V) unit of 16-bit elements
+  // as staged: 16-bit tiles as above; E4M3 tiles as 16 unswizzled D-byte rows
+  static constexpr int TILE = EB == 2 ? TILE16 : ROWS * D;
   static constexpr int STAGE = 2 * TILE;
   static constexpr int NC = 4;                  // consumer warps; unit u goes to warp u % NC
   static constexpr int NS = 2 * NC;             // two stages per consumer
@@ -42,11 +44,26 @@ struct GqaTiling {
   static_assert(NS % NC == 0, "stages must be a multiple of the consumer count");
   static constexpr int SMEM_MERGE = NC * ROWS * (D + 2) * 4;  // reuses the stages at the end
   static constexpr int SMEM_STAGES = NS * STAGE > SMEM_MERGE ? NS * STAGE : SMEM_MERGE;
+  // E4M3: each consumer's unit converted to 16-bit K and V tiles (swizzled as
+  // TMA would have written them, so the MMA path reads them unchanged)
+  static constexpr int SMEM_CONV = EB == 1 ? NC * 2 * TILE16 : 0;
   // + 1024: the stages start on a 1024-byte boundary (the swizzle period)
   static constexpr int QPITCH = (D + 8) * 2;    // the Q tile (when Q is not kept in registers)
   static constexpr int SMEM_Q = ROWS * QPITCH;
-  static constexpr int SMEM = 1024 + SMEM_STAGES + SMEM_Q + 2 * NS * 8 + NS * 4;
+  static constexpr int SMEM = 1024 + SMEM_STAGES + SMEM_CONV + SMEM_Q + 2 * NS * 8 + NS * 4;
+  static_assert(SMEM_STAGES % 128 == 0, "the converted tiles start on a 128-byte boundary");
 };
+
+// The power-of-two exponent qe that brings a query row whose largest magnitude
+// is mx below 2^15 (mx * 2^qe < 2^15, clamped to [-100, 100]; 0 for a zero or
+// non-finite row): the row times 2^qe then fits f16, exactly up to f16's
+// rounding, and the score is divided by 2^qe again.
+__device__ __forceinline__ int q_exponent(float mx) {
+  int e = 0;
+  if (!(mx > 0.f && mx < INFINITY)) return 0;
+  frexpf(mx, &e);  // mx = f * 2^e, f in [0.5, 1)
+  return max(-100, min(100, 15 - e));
+}
 
 // Byte offset of 16-byte chunk cc (0 .. D/8 - 1) of row r (0 .. 15) in a unit tile
 // of D/64 boxes, each 16 rows x 128 bytes with the 128-byte swizzle (chunk c of
@@ -115,15 +132,22 @@ __device__ __forceinline__ float2 unpack2(uint32_t x) {
   return Elem<T>::pair(x);
 }
 
-template <typename T, typename TO, int D, int S, bool APPEND, int NHT>
-__global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
+// TC: the cache element type, T or E4M3 codes (per-tensor scales: K's folded
+// into q_scale, V's applied to the output). Over E4M3 the consumers convert
+// each staged unit to f16 tiles and the products run in f16 (E4M3 values are
+// f16 values), with q held in f16 after an exact power-of-two scaling per head.
+template <typename T, typename TO, int D, int S, bool APPEND, int NHT, typename TC = T>
+__global__ void __launch_bounds__((GqaTiling<D, sizeof(TC)>::NC + 1) * 32)
     paged_decode_gqa_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv) {
-  using Tg = GqaTiling<D>;
+  constexpr int EB = sizeof(TC);
+  static_assert(!APPEND || EB == 2, "no fused append over E4M3 caches here");
+  using TM = typename std::conditional<EB == 1, __half, T>::type;  // the MMA operand type
+  using Tg = GqaTiling<D, EB>;
   constexpr int ROWS = Tg::ROWS, TILE = Tg::TILE, STAGE = Tg::STAGE;
   constexpr int NS = Tg::NS, NC = Tg::NC;
   constexpr int BR = S < 16 ? S : 16;  // rows per box
-  constexpr int SLAB = S * D * 2;
+  constexpr int SLAB = S * D * EB;
   constexpr int KS = D / 16;  // k-steps of S
 
   grid_dependents_launch();  // the merge of split requests may be scheduled early
@@ -162,7 +186,8 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* stages = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* qtile = stages + Tg::SMEM_STAGES;
+  uint8_t* conv = stages + Tg::SMEM_STAGES;  // E4M3: [NC][K, V] 16-bit tiles
+  uint8_t* qtile = conv + Tg::SMEM_CONV;
   uint64_t* full = reinterpret_cast<uint64_t*>(qtile + Tg::SMEM_Q);
   uint64_t* empty = full + NS;
   uint32_t* rowmask = reinterpret_cast<uint32_t*>(empty + NS);  // per stage: rows copied
@@ -226,19 +251,30 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
         rows_y[hh] = (id * p.Hkv + hk) * S + th % S;
         const int nrow = min(BR, t_end - th);
         okmask |= ((1u << nrow) - 1u) << (hh * BR);
-        bytes += 2u * (D / 64) * BR * 128u;
+        bytes += 2u * BR * D * EB;
       }
       if (lane == 0) {
         rowmask[s] = okmask;
         mbar_arrive_expect_tx(&full[s], bytes);
       }
       __syncwarp();
-      constexpr int NBOX = NH * (D / 64) * 2;  // (row group, column block, K or V)
-      if (lane < NBOX) {
-        const int hh = lane / ((D / 64) * 2), c = (lane >> 1) % (D / 64), kv = lane & 1;
-        if (issue[hh]) {
-          uint8_t* dst = stages + s * STAGE + c * Tg::BOX + hh * BR * 128 + kv * TILE;
-          tma_load_2d(dst, kv ? &tmv : &tmk, c * 64, rows_y[hh], &full[s], policy);
+      if constexpr (EB == 1) {
+        // E4M3: one box per (row group, K or V), the rows' whole D bytes
+        if (lane < NH * 2) {
+          const int hh = lane >> 1, kv = lane & 1;
+          if (issue[hh]) {
+            uint8_t* dst = stages + s * STAGE + hh * BR * D + kv * TILE;
+            tma_load_2d(dst, kv ? &tmv : &tmk, 0, rows_y[hh], &full[s], policy);
+          }
+        }
+      } else {
+        constexpr int NBOX = NH * (D / 64) * 2;  // (row group, column block, K or V)
+        if (lane < NBOX) {
+          const int hh = lane / ((D / 64) * 2), c = (lane >> 1) % (D / 64), kv = lane & 1;
+          if (issue[hh]) {
+            uint8_t* dst = stages + s * STAGE + c * Tg::BOX + hh * BR * 128 + kv * TILE;
+            tma_load_2d(dst, kv ? &tmv : &tmk, c * 64, rows_y[hh], &full[s], policy);
+          }
         }
       }
       __syncwarp();
@@ -259,6 +295,9 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   // (rows = heads, zero past gc) read with ldmatrix at every k-step.
   constexpr bool QREG = NHT * KS <= 8;
   uint32_t qb[QREG ? NHT : 1][QREG ? KS : 1][2];
+  float qdown[NHT];  // E4M3, Q in registers: 2^-qe of head 8 nt + g
+#pragma unroll
+  for (int nt = 0; nt < NHT; ++nt) qdown[nt] = 1.f;
   if constexpr (QREG) {
 #pragma unroll
     for (int nt = 0; nt < NHT; ++nt) {
@@ -272,7 +311,74 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
         qb[nt][kk][0] = row < gc ? __ldg(qrow + kk * 8 + t) : 0u;
         qb[nt][kk][1] = row < gc ? __ldg(qrow + kk * 8 + 4 + t) : 0u;
       }
+      if constexpr (EB == 1) {
+        // f16 operands: head row's q times 2^qe, its largest element below 2^15
+        // (the four lanes t of head g hold the row between them)
+        float mx = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float2 f = unpack2<T>(qb[nt][kk][j]);
+            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
+        const int qe = q_exponent(mx);
+        const float up = ldexpf(1.f, qe);
+        qdown[nt] = ldexpf(1.f, -qe);
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float2 f = unpack2<T>(qb[nt][kk][j]);
+            qb[nt][kk][j] = pack2<__half>(f.x * up, f.y * up);
+          }
+      }
     }
+  } else if constexpr (EB == 1) {
+    // the Q tile in f16: 8 threads per head row, each with D / 64 chunks; the
+    // row's scale exponent over the 8 (one warp's 8 consecutive lanes), its
+    // 2^-qe kept in the row's padding
+    const int row = threadIdx.x >> 3, sub = threadIdx.x & 7;
+    constexpr int QC = D / 64;
+    uint4 val[QC];
+    float mx = 0.f;
+#pragma unroll
+    for (int c = 0; c < QC; ++c) {
+      val[c] = make_uint4(0, 0, 0, 0);
+      if (row < gc) {
+        const int64_t hq = static_cast<int64_t>(hk) * G + c0 + row;
+        val[c] = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
+                                                 ((static_cast<int64_t>(i) * p.H + hq) * D +
+                                                  (sub + 8 * c) * 8) * 2);
+      }
+      const uint32_t wv[4] = {val[c].x, val[c].y, val[c].z, val[c].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack2<T>(wv[j]);
+        mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
+    const int qe = q_exponent(mx);
+    const float up = ldexpf(1.f, qe);
+#pragma unroll
+    for (int c = 0; c < QC; ++c) {
+      const uint32_t wv[4] = {val[c].x, val[c].y, val[c].z, val[c].w};
+      uint32_t hv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack2<T>(wv[j]);
+        hv[j] = pack2<__half>(f.x * up, f.y * up);
+      }
+      *reinterpret_cast<uint4*>(qtile + row * Tg::QPITCH + (sub + 8 * c) * 16) =
+          make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    }
+    if (sub == 0) *reinterpret_cast<float*>(qtile + row * Tg::QPITCH + D * 2) = ldexpf(1.f, -qe);
+    // consumers only: the Q tile is complete before anyone reads it
+    asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
   } else {
     for (int idx = threadIdx.x; idx < ROWS * (D / 8); idx += NC * 32) {
       const int row = idx / (D / 8), ch = idx % (D / 8);
@@ -329,6 +435,22 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
   const int k_tok = lane & 15, k_c8 = (lane >> 4) * 8;
   const int v_tok = (lane & 7) + 8 * (lane >> 4), v_c8 = ((lane >> 3) & 1) * 8;
 
+  // E4M3: the score multiplier of head 8 nt + 2t + c (q_scale and 2^-qe)
+  float qs[NHT][2];
+#pragma unroll
+  for (int nt = 0; nt < NHT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      float down = 1.f;
+      if constexpr (EB == 1) {
+        if constexpr (QREG)
+          down = __shfl_sync(kFullMask, qdown[nt], 4 * (2 * t + c));
+        else
+          down = *reinterpret_cast<const float*>(qtile + (8 * nt + 2 * t + c) * Tg::QPITCH + D * 2);
+      }
+      qs[nt][c] = p.q_scale * down;
+    }
+
   for (int k = w; k < nunits; k += NC) {
     const int s = k % NS;
     // every lane waits; the warp leaves together if any lane gave up
@@ -340,6 +462,27 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
     uint8_t* vtile = ktile + TILE;
     const int t0 = t_beg + k * ROWS;
     uint32_t valid = rowmask[s];
+    if constexpr (EB == 1) {
+      // E4M3: this consumer converts the unit to f16 tiles of its own (16 codes
+      // per chunk, two 16-byte chunks of f16 each), then frees the stage
+      uint8_t* kc = conv + w * 2 * Tg::TILE16;
+      uint8_t* vc = kc + Tg::TILE16;
+#pragma unroll 1
+      for (int idx = lane; idx < ROWS * D / 16; idx += 32) {
+        const int r = idx / (D / 16), j = idx % (D / 16);
+        uint32_t hk2[8], hv2[8];
+        e4m3x16_to_h2(ktile + r * D + j * 16, hk2);
+        e4m3x16_to_h2(vtile + r * D + j * 16, hv2);
+        *reinterpret_cast<uint4*>(kc + swz(r, 2 * j)) = make_uint4(hk2[0], hk2[1], hk2[2], hk2[3]);
+        *reinterpret_cast<uint4*>(kc + swz(r, 2 * j + 1)) = make_uint4(hk2[4], hk2[5], hk2[6], hk2[7]);
+        *reinterpret_cast<uint4*>(vc + swz(r, 2 * j)) = make_uint4(hv2[0], hv2[1], hv2[2], hv2[3]);
+        *reinterpret_cast<uint4*>(vc + swz(r, 2 * j + 1)) = make_uint4(hv2[4], hv2[5], hv2[6], hv2[7]);
+      }
+      __syncwarp();  // the tiles are written (and the staged codes read) by every lane
+      if (lane == 0) mbar_arrive(&empty[s]);
+      ktile = kc;
+      vtile = vc;
+    }
     if (has_new && t_new >= t0 && t_new < t0 + ROWS) {
       const int rnew = t_new - t0;
       if (chunk_lane) {
@@ -363,13 +506,13 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
       if constexpr (QREG) {
 #pragma unroll
         for (int nt = 0; nt < NHT; ++nt)
-          mma16816<T>((kk & 1) ? sodd[nt] : sacc[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+          mma16816<TM>((kk & 1) ? sodd[nt] : sacc[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
       } else {
         uint32_t b[4];
         ldsm_x4(b, qtile + q_row * Tg::QPITCH + (kk * 16 + q_c8) * 2);
 #pragma unroll
         for (int nt = 0; nt < NHT; ++nt)
-          mma16816<T>((kk & 1) ? sodd[nt] : sacc[nt], a, b[2 * nt], b[2 * nt + 1]);
+          mma16816<TM>((kk & 1) ? sodd[nt] : sacc[nt], a, b[2 * nt], b[2 * nt + 1]);
       }
     }
     // scores (base 2), masked by selection: element e is token g + 8 (e >> 1),
@@ -384,7 +527,10 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const bool ok = (e >> 1) ? tok_hi : tok_lo;
-        sc[e] = ok ? (sacc[nt][e] + sodd[nt][e]) * p.q_scale : -INFINITY;
+        if constexpr (EB == 1)
+          sc[e] = ok ? (sacc[nt][e] + sodd[nt][e]) * qs[nt][e & 1] : -INFINITY;
+        else
+          sc[e] = ok ? (sacc[nt][e] + sodd[nt][e]) * p.q_scale : -INFINITY;
       }
       float pr[4];
 #pragma unroll
@@ -405,13 +551,13 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
       // head g, by transposing the accumulator-layout pairs. bf16 keeps 8 bits,
       // so P goes in as a hi + lo pair (its rounding drops from 2^-9 to 2^-17);
       // fp16 keeps 11, within the tolerance on its own.
-      const uint32_t h0 = pack2<T>(pr[0], pr[1]), h1 = pack2<T>(pr[2], pr[3]);
+      const uint32_t h0 = pack2<TM>(pr[0], pr[1]), h1 = pack2<TM>(pr[2], pr[3]);
       bhi[nt][0] = movmatrix_trans(h0);
       bhi[nt][1] = movmatrix_trans(h1);
-      if (std::is_same<T, __nv_bfloat16>::value) {
-        const float2 f0 = unpack2<T>(h0), f1 = unpack2<T>(h1);
-        blo[nt][0] = movmatrix_trans(pack2<T>(pr[0] - f0.x, pr[1] - f0.y));
-        blo[nt][1] = movmatrix_trans(pack2<T>(pr[2] - f1.x, pr[3] - f1.y));
+      if (std::is_same<TM, __nv_bfloat16>::value) {
+        const float2 f0 = unpack2<TM>(h0), f1 = unpack2<TM>(h1);
+        blo[nt][0] = movmatrix_trans(pack2<TM>(pr[0] - f0.x, pr[1] - f0.y));
+        blo[nt][1] = movmatrix_trans(pack2<TM>(pr[2] - f1.x, pr[3] - f1.y));
       }
     }
     // once the running max settles most units move no head's max
@@ -445,13 +591,15 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
       }
 #pragma unroll
       for (int nt = 0; nt < NHT; ++nt) {
-        mma16816<T>(o[mt][nt], a, bhi[nt][0], bhi[nt][1]);
-        if (std::is_same<T, __nv_bfloat16>::value)
-          mma16816<T>(o[mt][nt], a, blo[nt][0], blo[nt][1]);
+        mma16816<TM>(o[mt][nt], a, bhi[nt][0], bhi[nt][1]);
+        if (std::is_same<TM, __nv_bfloat16>::value)
+          mma16816<TM>(o[mt][nt], a, blo[nt][0], blo[nt][1]);
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    if constexpr (EB == 2) {
+      if (lane == 0) mbar_arrive(&empty[s]);  // (E4M3 freed its stage after converting)
+    }
   }
 
   // head sums over the 8 lanes that share t
@@ -504,6 +652,7 @@ __global__ void __launch_bounds__((GqaTiling<D>::NC + 1) * 32)
       float a = 0.f;
 #pragma unroll
       for (int c = 0; c < NC; ++c) a = fmaf(wt[c], mg[(c * ROWS + row) * (D + 2) + 2 + d], a);
+      if constexpr (EB == 1) a *= p.v_scale;
       if (direct) {
         static_cast<TO*>(p.out)[ih * D + d] = to_out<TO>(lsum > 0.f ? a / lsum : 0.f);
       } else {

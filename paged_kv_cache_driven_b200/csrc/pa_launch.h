@@ -82,6 +82,9 @@ bool opt_in_smem(K kern, int bytes, bool (&configured)[kMaxDevices]) {
 // box_rows rows, 128-byte swizzle (the last few maps are cached). query_map: the
 // packed queries [T, H, D] as (D, H, T), boxes of 64 elements x 1 head x 128 rows.
 bool row_map(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows, pa_dtype dt);
+// row_map_codes: the same view of a cache of one-byte E4M3 codes; a box is one
+// whole D-byte row x box_rows rows, unswizzled.
+bool row_map_codes(CUtensorMap* out, const void* base, int64_t rows, int D, int box_rows);
 bool query_map(CUtensorMap* out, const void* q, int64_t T, int H, int D, pa_dtype dt);
 
 // Launchers (asynchronous on `stream`; the arguments are already checked).
@@ -91,6 +94,9 @@ pa_status launch_decode16(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt,
                           bool append, bool cluster, cudaStream_t stream);  // pa_k_decode.cu
 pa_status launch_grouped(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt, int D, int S,
                          bool append, cudaStream_t stream);             // pa_k_gqa.cu
+// grouped-query heads over E4M3 caches (q_dt: the queries' 16-bit type)
+pa_status launch_grouped_fp8(const DecodeParams& prm, pa_dtype q_dt, pa_dtype out_dt, int D,
+                             int S, cudaStream_t stream);               // pa_k_gqa.cu
 // append: the new tokens' rows (prm.k_new / v_new, dtype q_dt) are quantized
 // with k_scale and prm.v_scale and written into the caches inside the launch.
 pa_status launch_decode_fp8(const DecodeParams& prm, pa_dtype q_dt, pa_dtype out_dt, int D,

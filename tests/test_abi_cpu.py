@@ -180,6 +180,23 @@ def test_decode_fp8_zero_batch_is_noop(lib):
     assert lib.pa_decode_fp8(*fp8_decode_args(B=0, q=NULL, out=NULL)) == binding.PA_OK
 
 
+def fp8_gqa_args(Hkv=2, **kw):
+    a = fp8_decode_args(**kw)
+    return a[:14] + [Hkv] + a[14:]  # Hkv after H
+
+
+@pytest.mark.parametrize("bad", [
+    dict(Hkv=3), dict(Hkv=0), dict(Hkv=8), dict(ks=0.0), dict(D=96), dict(k=NULL),
+    dict(q_dt=binding.PA_F32), dict(max_seq_len=100, partition=16),
+])
+def test_decode_gqa_fp8_rejects_bad_arguments_on_host(lib, bad):
+    assert lib.pa_decode_gqa_fp8(*fp8_gqa_args(**bad)) == binding.PA_ERR_INVALID
+
+
+def test_decode_gqa_fp8_zero_batch_is_noop(lib):
+    assert lib.pa_decode_gqa_fp8(*fp8_gqa_args(B=0, q=NULL, out=NULL)) == binding.PA_OK
+
+
 def fp8_decode_append_args(kn=P, vn=P, **kw):
     a = fp8_decode_args(**kw)
     return a[:4] + [kn, vn] + a[4:]  # k_new, v_new after q_dt

@@ -220,3 +220,128 @@ def test_decode_append_fp8_equals_two_calls(lens, H, D, S, in_dt, out_dt, partit
         want = ofp8.paged_decode_fp8(case.q.cpu(), kc_b.cpu(), vc_b.cpu(), 0.05, 0.08,
                                      case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
         assert_parity(out_b.cpu().numpy(), want, f"fused fp8 append {lens} D={D}")
+
+
+def fp8_gqa_case(lens, H, Hkv, D, S, in_dt, seed, k_scale=0.05, v_scale=0.08):
+    """fp8_case with Hkv KV heads in the caches ([NB, Hkv, S, D]) and H query heads."""
+    case = workloads.decode_case(lens, H=H, D=D, S=S, dtype=in_dt, seed=seed, device=DEV,
+                                 poison=False, Hkv=Hkv)
+    NB = case.k_cache.shape[0]
+    kc8 = torch.full((NB, Hkv, S, D), NAN_CODE, dtype=torch.uint8, device=DEV)
+    vc8 = torch.full_like(kc8, NAN_CODE)
+    for i, L in enumerate(case.seq_lens_host):
+        if L == 0:
+            continue
+        blocks = torch.tensor(case.tables_host[i], device=DEV)
+        k = case.k_cache[blocks].permute(0, 2, 1, 3).reshape(-1, Hkv, D)[:L].contiguous()
+        v = case.v_cache[blocks].permute(0, 2, 1, 3).reshape(-1, Hkv, D)[:L].contiguous()
+        slots = (blocks.repeat_interleave(S) * S + torch.arange(S, device=DEV).repeat(len(blocks)))[:L]
+        binding.pa_kv_append_fp8(k, v, slots.to(torch.int64), kc8, vc8, k_scale, v_scale)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    return case, kc8, vc8
+
+
+def run_gqa_fp8(case, kc8, vc8, out_dt=torch.float32, partition=0):
+    B, H, D = case.q.shape
+    S = kc8.shape[2]
+    maxlen = max(case.seq_lens_host + [0])
+    out = torch.empty((B, H, D), dtype=out_dt, device=DEV)
+    wsb = binding.pa_decode_workspace_bytes(B, H, D, S, maxlen, partition)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=DEV)
+    binding.pa_decode_gqa_fp8(out, case.q, kc8, vc8, 0.05, 0.08, case.block_tables,
+                              case.seq_lens, case.scale, maxlen, partition=partition, workspace=ws)
+    torch.cuda.synchronize()
+    assert binding.pa_get_device_error() == 0
+    return out
+
+
+@pytest.mark.parametrize("G,D,S,in_dt,partition", [
+    (8, 128, 16, torch.bfloat16, 0), (8, 128, 16, torch.bfloat16, 64),
+    (2, 64, 8, torch.float16, -1), (4, 256, 32, torch.bfloat16, 64),
+    (16, 128, 16, torch.float16, 0), (3, 128, 8, torch.bfloat16, 32),
+    (8, 64, 32, torch.bfloat16, 0), (12, 256, 16, torch.float16, 0),
+])
+def test_decode_gqa_fp8(G, D, S, in_dt, partition):
+    """Grouped-query heads over E4M3 caches (tensor cores, f16 products) against
+    the oracle's decode over the same codes, every output element."""
+    lens = [0, 1, S - 1, 16, 17, 300, 1000]
+    Hkv = 2
+    case, kc8, vc8 = fp8_gqa_case(lens, H=G * Hkv, Hkv=Hkv, D=D, S=S, in_dt=in_dt, seed=G + D + S)
+    out = run_gqa_fp8(case, kc8, vc8, partition=partition)
+    want = ofp8.paged_decode_fp8(case.q.cpu(), kc8.cpu(), vc8.cpu(), 0.05, 0.08,
+                                 case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
+    assert_parity(out.cpu().numpy(), want, f"fp8 gqa G={G} D={D} S={S} p={partition}")
+    assert np.all(out[0].cpu().numpy() == 0)  # L = 0
+
+
+@pytest.mark.parametrize("q_mag", [1e-3, 3e3])
+def test_decode_gqa_fp8_query_magnitude(q_mag):
+    """Each query head is scaled into f16 by its own power of two: tiny and large
+    queries (and heads of different magnitudes in one group) match the oracle."""
+    case, kc8, vc8 = fp8_gqa_case([5, 40, 333], H=16, Hkv=2, D=128, S=16,
+                                  in_dt=torch.bfloat16, seed=11)
+    case.q.mul_(q_mag)
+    case.q[:, 1::2].mul_(64.0)  # neighbouring heads four orders of magnitude apart
+    for out_dt in (torch.float32, torch.bfloat16):
+        out = run_gqa_fp8(case, kc8, vc8, out_dt=out_dt)
+        want = ofp8.paged_decode_fp8(case.q.cpu(), kc8.cpu(), vc8.cpu(), 0.05, 0.08,
+                                     case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
+        got = out.float().cpu().numpy()
+        if out_dt == torch.float32:
+            assert_parity(got, want, f"fp8 gqa |q|~{q_mag}")
+        else:
+            assert np.abs(got - want).max() <= MAX_ABS + 2.0 ** -8 * np.abs(want).max()
+
+
+def test_decode_gqa_fp8_one_group_is_decode_fp8():
+    """Hkv == H goes to pa_decode_fp8: the same bits."""
+    case, kc8, vc8 = fp8_case([7, 300, 999], H=4, D=128, S=16, in_dt=torch.bfloat16, seed=5)
+    a = run_fp8(case, kc8, vc8)
+    b = run_gqa_fp8(case, kc8, vc8)
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+def test_decode_gqa_fp8_llama70b_shape_sampled():
+    """64 query heads on 8 KV heads, head_dim 128, block 16, batch 64, L ~ U[1, 2048]
+    over an E4M3 cache, in the automatic plan, on sampled (request, head) pairs."""
+    lens = workloads.uniform_lengths(64, 1, 2048, 0)
+    case, kc8, vc8 = fp8_gqa_case(lens, H=64, Hkv=8, D=128, S=16, in_dt=torch.bfloat16, seed=0)
+    out = run_gqa_fp8(case, kc8, vc8)
+    pairs = sample_pairs(case, 24)
+    G = 8
+    qs, ks, vs, tabs, Ls = [], [], [], [], []
+    off = 0
+    for i, h in pairs:
+        blocks = torch.tensor(case.tables_host[i], device=DEV)
+        ks.append(kc8[blocks, h // G].unsqueeze(1).cpu())
+        vs.append(vc8[blocks, h // G].unsqueeze(1).cpu())
+        qs.append(case.q[i, h].view(1, 1, -1).cpu())
+        tabs.append(list(range(off, off + len(blocks))))
+        Ls.append(case.seq_lens_host[i])
+        off += len(blocks)
+    MB = max(len(t) for t in tabs)
+    bt = torch.full((len(pairs), MB), -1, dtype=torch.int32)
+    for r, t in enumerate(tabs):
+        bt[r, :len(t)] = torch.tensor(t, dtype=torch.int32)
+    want = ofp8.paged_decode_fp8(torch.cat(qs), torch.cat(ks), torch.cat(vs), 0.05, 0.08, bt,
+                                 torch.tensor(Ls, dtype=torch.int32), case.scale)[:, 0]
+    got = torch.stack([out[i, h] for i, h in pairs]).cpu().numpy()
+    assert_parity(got, want, "fp8 70B shape")
+    assert bool(torch.isfinite(out).all())
+
+
+def test_decode_gqa_fp8_bad_block_id_is_skipped_and_flagged():
+    case, kc8, vc8 = fp8_gqa_case([64, 48], H=8, Hkv=2, D=128, S=16, in_dt=torch.bfloat16,
+                                  seed=9)
+    want = ofp8.paged_decode_fp8(case.q.cpu(), kc8.cpu(), vc8.cpu(), 0.05, 0.08,
+                                 case.block_tables.cpu(), case.seq_lens.cpu(), case.scale)
+    bt = case.block_tables.clone()
+    bt[0, 1] = kc8.shape[0] + 7
+    B, H, D = case.q.shape
+    out = torch.empty((B, H, D), dtype=torch.float32, device=DEV)
+    binding.pa_decode_gqa_fp8(out, case.q, kc8, vc8, 0.05, 0.08, bt, case.seq_lens, case.scale,
+                              64, partition=-1)
+    assert binding.pa_get_device_error() & binding.PA_DEVERR_BLOCK_ID
+    assert_parity(out[1:].cpu().numpy(), want[1:], "fp8 gqa neighbour of a bad id")
+    assert bool(torch.isfinite(out[0]).all())
