@@ -124,7 +124,9 @@ size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, in
  * (partition = 0) depends on B * H and the device's SM count: call this and
  * pa_decode_workspace_bytes with the device current that pa_decode will run on.
  * Automatic: 512-token partitions, halved (down to 64 tokens) while the grid
- * has fewer CTAs than the device has SMs; a resulting count of 3, 5, 6 or 7 is
+ * has fewer CTAs than the device has SMs, or for contexts of 32K tokens and
+ * more doubled (up to 2048) while the grid keeps 8 CTAs per SM; a resulting
+ * count of 3, 5, 6 or 7 is
  * then re-cut to the next (else the previous) power of two when that grid fits
  * within two CTAs per SM, so that the split merges inside clusters. */
 pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partition,

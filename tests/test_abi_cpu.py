@@ -93,6 +93,10 @@ def test_workspace_and_plan(lib):
     # 1332 tokens in blocks of 32 on 32 heads: 8 of 192 (the eighth empty)
     assert binding.pa_decode_plan(1, 32, 128, 32, 1332) == (192, 8)
     assert binding.pa_decode_plan(1, 1, 128, 16, 8192) == (64, 128)
+    # long contexts: up to 2048-token partitions while >= 8 CTAs per SM remain
+    assert binding.pa_decode_plan(8, 32, 128, 16, 131072) == (2048, 64)
+    assert binding.pa_decode_plan(2, 4, 128, 16, 40000) == (512, 79)  # too few CTAs to grow
+    assert binding.pa_decode_plan(64, 40, 128, 16, 8192) == (512, 16)  # below 32K: 512
     assert binding.pa_decode_plan(1, 32, 128, 8, 100) == (64, 2)
     n = 64 * 40 * 4
     want = ((n * 8 + 255) // 256) * 256 + n * 128 * 4
