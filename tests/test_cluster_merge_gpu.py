@@ -117,3 +117,33 @@ def test_cluster_merge_fp8():
     assert same_bits(outs[0], outs[1])
     assert torch.isfinite(outs[0]).all()
     assert binding.pa_get_device_error() == 0
+
+
+def test_cluster_merge_in_a_cuda_graph():
+    """A cluster launch captured in a CUDA graph replays to the eager bits."""
+    lens = [1332, 17]
+    H, D, S = 16, 128, 16
+    case = workloads.decode_case(lens, H=H, D=D, S=S, dtype=torch.bfloat16, seed=21, device=DEV)
+    cluster_plan(len(lens), H, D, S, max(lens))
+    eager, _ = run_decode(case, partition=0)
+    out = torch.empty_like(eager)
+    wsb = binding.pa_decode_workspace_bytes(len(lens), H, D, S, max(lens), 0)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up outside the capture (attribute set-up)
+        binding.pa_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables,
+                          case.seq_lens, case.scale, max(lens), partition=0, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    out.zero_()
+    with torch.cuda.graph(g):
+        binding.pa_decode(out, case.q, case.k_cache, case.v_cache, case.block_tables,
+                          case.seq_lens, case.scale, max(lens), partition=0, workspace=ws)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert same_bits(out, eager)
+    del g
+    assert binding.pa_get_device_error() == 0
