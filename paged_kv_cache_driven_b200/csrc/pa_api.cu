@@ -435,7 +435,7 @@ pa_status pa_prefill(void* out, pa_dtype out_dt, const void* q, const void* k_ca
   if (B < 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || T < 0 || max_q_len < 0 || MB < 0 || NB < 0)
     return PA_ERR_INVALID;
   if (!cache_dtype_ok(dt) || !out_dtype_ok(out_dt)) return PA_ERR_INVALID;
-  if (!(D == 64 || D == 128) || !(S == 8 || S == 16 || S == 32 || S == 64 || S == 128))
+  if (!(D == 64 || D == 128 || D == 256) || !(S == 8 || S == 16 || S == 32 || S == 64 || S == 128))
     return PA_ERR_INVALID;
   if (!std::isfinite(scale) || !(scale > 0.f)) return PA_ERR_INVALID;
   if (B == 0 || T == 0 || max_q_len == 0) return PA_OK;

@@ -1,6 +1,6 @@
 // Kernels of pa_prefill: causal paged prefill attention on the fifth-generation
-// tensor cores, for both 16-bit cache dtypes, every output dtype, head size 64
-// and 128 and block sizes 8 .. 128, and their launcher.
+// tensor cores, for both 16-bit cache dtypes, every output dtype, head size 64,
+// 128 and 256 and block sizes 8 .. 128, and their launcher.
 
 #include <type_traits>
 
@@ -35,6 +35,7 @@ pa_status by_shape(const PrefillParams& prm, const void* q, int D, int S, cudaSt
   if (D == DD && S == SS) return launch<T, TO, DD, SS>(prm, q, st);
   PA_CASE(64, 8) PA_CASE(64, 16) PA_CASE(64, 32) PA_CASE(64, 64) PA_CASE(64, 128)
   PA_CASE(128, 8) PA_CASE(128, 16) PA_CASE(128, 32) PA_CASE(128, 64) PA_CASE(128, 128)
+  PA_CASE(256, 8) PA_CASE(256, 16) PA_CASE(256, 32) PA_CASE(256, 64) PA_CASE(256, 128)
 #undef PA_CASE
   return PA_ERR_INVALID;
 }

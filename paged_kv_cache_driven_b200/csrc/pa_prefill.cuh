@@ -70,12 +70,16 @@ __device__ long long g_prefill_trace[kTraceCtas][kTraceSlots][kTraceTiles];
 template <int D, bool LO>
 struct PrefillTiling {
   static constexpr int BM = 128;              // query rows per tile (MMA M)
-  static constexpr int NQT = 2;               // query tiles per CTA
+  // query tiles per CTA: two that ping-pong; head_dim 256 holds one (its S and
+  // O take 384 of the 512 tensor-memory columns, and a second 64 KB query tile
+  // would not fit beside the K and V tiles)
+  static constexpr int NQT = D == 256 ? 1 : 2;
   static constexpr int BN = 128;              // keys per tile
   // separate K and V rings: S needs K(j + 1) right after P(j) is ready,
-  // V(j + 1) only after the next softmax
-  static constexpr int KST = D == 128 ? 2 : 4;  // K stages
-  static constexpr int VST = D == 128 ? 2 : 4;  // V stages
+  // V(j + 1) only after the next softmax (one stage each at head_dim 256:
+  // 64 KB tiles)
+  static constexpr int KST = D == 256 ? 1 : (D == 128 ? 2 : 4);  // K stages
+  static constexpr int VST = D == 256 ? 1 : (D == 128 ? 2 : 4);  // V stages
   static constexpr int COLB = D / 64;         // 64-element (128-byte) column blocks
   static constexpr int CB_BYTES = 128 * 128;  // one column block of 128 rows
   static constexpr int Q_BYTES = BM * D * 2;  // one query tile
@@ -89,8 +93,10 @@ struct PrefillTiling {
   // SM (it allocates all 512 tensor-memory columns)
   static constexpr int SMEM = 1024 + OFF_BAR + 256 > 120 * 1024 ? 1024 + OFF_BAR + 256 : 120 * 1024;
   static constexpr int THREADS = NQT * 256 + 64;  // two softmax warpgroups per tile
-  static constexpr uint32_t TMEM_COLS = 512;  // per tile: S/P 128 columns, O 128
-  static_assert(D == 64 || D == 128, "head size 64 or 128");
+  static constexpr uint32_t TMEM_COLS = 512;  // per tile: S/P 128 columns, O D columns
+  static_assert(D == 64 || D == 128 || D == 256, "head size 64, 128 or 256");
+  // tiles sit 256 columns apart: S (128 columns) then O (D columns)
+  static_assert(NQT == 1 ? 128 + D <= 512 : 128 + D <= 256, "tensor-memory columns");
   static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
@@ -216,8 +222,12 @@ __global__ void __launch_bounds__(576, 1)
     const int first = row0 + t * Tl::BM;
     nk[t] = first >= n ? 0 : (ctx + min(n, first + Tl::BM) - 1) / Tl::BN + 1;
   }
-  const int NK = max(nk[0], nk[1]);
-  const int nq = nk[1] > 0 ? 2 : 1;
+  int NK = nk[0], nq = 1;  // key tiles of the CTA; query tiles holding rows
+#pragma unroll
+  for (int t = 1; t < Tl::NQT; ++t) {
+    NK = max(NK, nk[t]);
+    if (nk[t] > 0) nq = t + 1;
+  }
   const int hk = h / (p.H / p.Hkv);
 
   extern __shared__ uint8_t smem_raw[];

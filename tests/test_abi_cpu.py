@@ -147,7 +147,7 @@ def prefill_args(**kw):
 
 
 @pytest.mark.parametrize("bad", [
-    dict(D=96), dict(D=256), dict(S=4), dict(S=256), dict(dt=binding.PA_F32), dict(out_dt=9),
+    dict(D=96), dict(D=512), dict(S=4), dict(S=256), dict(dt=binding.PA_F32), dict(out_dt=9),
     dict(scale=0.0), dict(scale=-1.0), dict(scale=float("nan")), dict(Hkv=3), dict(Hkv=0),
     dict(q=NULL), dict(qs=NULL), dict(bt=NULL), dict(out=ctypes.c_void_p(16 * 1024 + 4)),
     dict(NB=0), dict(NB=1 << 28), dict(T=-1), dict(max_q_len=-1), dict(B=-1), dict(B=65536),

@@ -58,6 +58,24 @@ def test_head_dim_64(dt, S):
     check(pc, what=f"D=64 S={S} {dt}")
 
 
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("S", [8, 16, 64, 128])
+def test_head_dim_256(dt, S):
+    """head_dim 256: one 128-row query tile per CTA; prompts and chunks that
+    span several query and key tiles with ragged tails, with context."""
+    pc = workloads.prefill_case([0, 37, 200, 0], [1, 129, 300, 256], H=2, D=256, S=S, dtype=dt,
+                                seed=S + 256, device=DEV)
+    check(pc, what=f"D=256 S={S} {dt}")
+
+
+def test_head_dim_256_grouped_and_outputs():
+    """head_dim 256 with grouped query heads (6 on 2) and 16-bit outputs."""
+    pc = workloads.prefill_case([5, 0], [140, 260], H=6, D=256, S=16, dtype=torch.bfloat16,
+                                seed=9, device=DEV, Hkv=2)
+    check(pc, what="D=256 gqa")
+    check(pc, out_dtype=torch.bfloat16, what="D=256 bf16 out")
+
+
 @pytest.mark.parametrize("odt", [torch.bfloat16, torch.float16])
 def test_output_dtypes(odt):
     pc = workloads.prefill_case([0, 40], [150, 90], H=2, D=128, S=16, dtype=torch.bfloat16,
