@@ -1090,6 +1090,8 @@ def run_prefill_workload(args):
     if args.workload == "prompt_prefill_small":  # a profiling-sized case of the same kernel
         pc = workloads.prompt_prefill(seed=args.seed, device=device, n_req=4, lo=2048, hi=2048,
                                       H=8)
+    elif args.workload == "prompt_prefill_d256":  # the same prompts at head_dim 256
+        pc = workloads.prompt_prefill(seed=args.seed, device=device, D=256)
     else:
         pc = workloads.prompt_prefill(seed=args.seed, device=device)
     c = pc.cache
@@ -1189,11 +1191,14 @@ def run_prefill_workload(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": PREFILL_WORKLOAD if args.workload == "prompt_prefill" else
-                   "prompt prefill, profiling size: 4 prompts of 2048 tokens, 8 heads",
+        "config": {"workload": {"prompt_prefill": PREFILL_WORKLOAD,
+                                "prompt_prefill_d256": PREFILL_WORKLOAD.replace("head_dim 128",
+                                                                                "head_dim 256")}.get(
+                       args.workload,
+                       "prompt prefill, profiling size: 4 prompts of 2048 tokens, 8 heads"),
                    "prompt_tokens": T, "heads": Hq,
                    "head_dim": Dh, "block_size": c.k_cache.shape[2], "flops_per_step": flops,
-                   "l2": "inputs larger than L2 (0.9 GB of q and K/V vs 126 MB L2)",
+                   "l2": "inputs larger than L2 (0.9 GB or more of q and K/V vs 126 MB L2)",
                    "parallelism": "dp1"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
@@ -1227,7 +1232,8 @@ def main():
     ap.add_argument("--workload", default="llama13b",
                     choices=["llama13b", "long_context", "sweep", "llama70b", "llama70b_fp8",
                              "llama13b_fp8",
-                             "prompt_prefill", "prompt_prefill_small", "worked_example",
+                             "prompt_prefill", "prompt_prefill_small", "prompt_prefill_d256",
+                             "worked_example",
                              "prefill_append", "prefill_append_small", "batching",
                              "prefill_trace"],
                     help="llama13b: the headline step (default); the others time decode-only "
