@@ -36,7 +36,7 @@ struct GqaTiling {
   // as staged: 16-bit tiles as above; E4M3 tiles as 16 unswizzled D-byte rows
   static constexpr int TILE = EB == 2 ? TILE16 : ROWS * D;
   static constexpr int STAGE = 2 * TILE;
-  static constexpr int NC = 4;                  // consumer warps; unit u goes to warp u % NC
+  static constexpr int NC = 3;                  // consumer warps; unit u goes to warp u % NC
   static constexpr int NS = 2 * NC;             // two stages per consumer
   // Consumer w takes units w, w + NC, ...; a stage is reused every NS units, so
   // with NS a multiple of NC each stage's units belong to one consumer and it
@@ -339,44 +339,48 @@ __global__ void __launch_bounds__((GqaTiling<D, sizeof(TC)>::NC + 1) * 32)
   } else if constexpr (EB == 1) {
     // the Q tile in f16: 8 threads per head row, each with D / 64 chunks; the
     // row's scale exponent over the 8 (one warp's 8 consecutive lanes), its
-    // 2^-qe kept in the row's padding
-    const int row = threadIdx.x >> 3, sub = threadIdx.x & 7;
+    // 2^-qe kept in the row's padding. A warp's four rows of a pass are all in
+    // the tile or all past it, so the shuffles see whole warps.
+    static_assert(ROWS % 4 == 0, "four head rows per warp and pass");
+    const int sub = threadIdx.x & 7;
     constexpr int QC = D / 64;
-    uint4 val[QC];
-    float mx = 0.f;
+    for (int row = threadIdx.x >> 3; row < ROWS; row += NC * 4) {
+      uint4 val[QC];
+      float mx = 0.f;
 #pragma unroll
-    for (int c = 0; c < QC; ++c) {
-      val[c] = make_uint4(0, 0, 0, 0);
-      if (row < gc) {
-        const int64_t hq = static_cast<int64_t>(hk) * G + c0 + row;
-        val[c] = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
-                                                 ((static_cast<int64_t>(i) * p.H + hq) * D +
-                                                  (sub + 8 * c) * 8) * 2);
-      }
-      const uint32_t wv[4] = {val[c].x, val[c].y, val[c].z, val[c].w};
+      for (int c = 0; c < QC; ++c) {
+        val[c] = make_uint4(0, 0, 0, 0);
+        if (row < gc) {
+          const int64_t hq = static_cast<int64_t>(hk) * G + c0 + row;
+          val[c] = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
+                                                   ((static_cast<int64_t>(i) * p.H + hq) * D +
+                                                    (sub + 8 * c) * 8) * 2);
+        }
+        const uint32_t wv[4] = {val[c].x, val[c].y, val[c].z, val[c].w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack2<T>(wv[j]);
-        mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack2<T>(wv[j]);
+          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
       }
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
+      const int qe = q_exponent(mx);
+      const float up = ldexpf(1.f, qe);
+#pragma unroll
+      for (int c = 0; c < QC; ++c) {
+        const uint32_t wv[4] = {val[c].x, val[c].y, val[c].z, val[c].w};
+        uint32_t hv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack2<T>(wv[j]);
+          hv[j] = pack2<__half>(f.x * up, f.y * up);
+        }
+        *reinterpret_cast<uint4*>(qtile + row * Tg::QPITCH + (sub + 8 * c) * 16) =
+            make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      }
+      if (sub == 0) *reinterpret_cast<float*>(qtile + row * Tg::QPITCH + D * 2) = ldexpf(1.f, -qe);
     }
-#pragma unroll
-    for (int off = 1; off < 8; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
-    const int qe = q_exponent(mx);
-    const float up = ldexpf(1.f, qe);
-#pragma unroll
-    for (int c = 0; c < QC; ++c) {
-      const uint32_t wv[4] = {val[c].x, val[c].y, val[c].z, val[c].w};
-      uint32_t hv[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack2<T>(wv[j]);
-        hv[j] = pack2<__half>(f.x * up, f.y * up);
-      }
-      *reinterpret_cast<uint4*>(qtile + row * Tg::QPITCH + (sub + 8 * c) * 16) =
-          make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    }
-    if (sub == 0) *reinterpret_cast<float*>(qtile + row * Tg::QPITCH + D * 2) = ldexpf(1.f, -qe);
     // consumers only: the Q tile is complete before anyone reads it
     asm volatile("bar.sync 1, %0;" ::"n"(NC * 32) : "memory");
   } else {
