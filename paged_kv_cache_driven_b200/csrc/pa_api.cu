@@ -112,6 +112,12 @@ bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* 
   return true;
 }
 
+// Whether a partition pass of B x H x NP CTAs holds at most two CTAs per SM
+// (a small grid: the kernels then take their wide CTA shapes).
+bool small_grid(int B, int H, int NP) {
+  return static_cast<int64_t>(B) * H * NP <= 2 * static_cast<int64_t>(sm_count());
+}
+
 // Whether an automatic split of NP partitions over B x H (request, head) pairs
 // merges inside clusters instead of through the workspace and the merge
 // kernel: NP is a portable cluster size (2, 4 or 8; the cluster spans the
@@ -121,7 +127,7 @@ bool plan(int B, int H, int S, int max_seq_len, int partition, int* P_out, int* 
 // merge kernel, which overlaps their last wave.
 bool cluster_merge(int B, int H, int NP) {
   if (NP != 2 && NP != 4 && NP != 8) return false;
-  return static_cast<int64_t>(B) * H * NP <= 2 * static_cast<int64_t>(sm_count());
+  return small_grid(B, H, NP);
 }
 
 // Split-KV workspace: m and l [B, H, NP], then (256-byte aligned) acc [B, H, NP, D].
@@ -385,7 +391,8 @@ pa_status decode_impl(void* out, pa_dtype out_dt, const void* q, const void* k_n
   if (H != Hkv)  // (the grouped-query kernel always merges through the workspace)
     return pa::host::launch_grouped(prm, dt, out_dt, D, S, k_new != nullptr, st);
   const bool cluster = partition == 0 && cluster_merge(B, H, prm.NP);
-  return pa::host::launch_decode16(prm, dt, out_dt, D, S, k_new != nullptr, cluster, st);
+  return pa::host::launch_decode16(prm, dt, out_dt, D, S, k_new != nullptr, cluster,
+                                   small_grid(B, H, prm.NP), st);
 }
 
 }  // namespace
@@ -535,8 +542,8 @@ static pa_status decode_fp8_impl(void* out, pa_dtype out_dt, const void* q, pa_d
   prm.k_new = k_new;
   prm.v_new = v_new;
   const bool cluster = partition == 0 && cluster_merge(B, H, prm.NP);
-  return pa::host::launch_decode_fp8(prm, q_dt, out_dt, D, S, cluster, append, k_scale,
-                                     static_cast<cudaStream_t>(stream));
+  return pa::host::launch_decode_fp8(prm, q_dt, out_dt, D, S, cluster, small_grid(B, H, prm.NP),
+                                     append, k_scale, static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_decode_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype q_dt,

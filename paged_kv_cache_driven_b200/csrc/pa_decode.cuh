@@ -49,8 +49,17 @@ namespace pa {
 //   CR       rows per pipeline unit: CR x D of K and of V (up to 4 KB each) is one
 //            stage, so the stage size no longer grows with S; a block of S rows
 //            is S / CR units
-//   NS, NW   stages per warp and warps per CTA: about 64 KB of stages per CTA
-template <int D, int S, int EB = 2>
+//   NS, NW   stages per warp and warps per CTA: about 64 KB of stages per CTA.
+//            Grids of more than two CTAs per SM (WIDE = false) with units of
+//            2 KB or less take 32 KB: half the warps, each walking twice the
+//            blocks of a partition, so that pipeline fill and drain weigh half
+//            as much and twice the CTAs share an SM (head_dim 64 at blocks 8
+//            and 16: 5-12 % faster from batch 32 up; the 13B-shaped E4M3
+//            decode 124 -> 108 us). Smaller grids (WIDE = true, cluster
+//            launches among them) keep the wider CTAs, which spread their few
+//            CTAs' work over more warps (batch 1, head_dim 128, block 8: 14.4
+//            against 17.4 us).
+template <int D, int S, int EB = 2, bool WIDE = false>
 struct DecodeTiling {
   static constexpr int EPL = 16 / EB;
   static constexpr int LPR = D / EPL;
@@ -64,7 +73,7 @@ struct DecodeTiling {
   // E4M3 units carry twice the elements per byte, so more warps (two stages
   // each) keep the same bytes in flight with twice the threads to convert them
   static constexpr int NS = (STAGE <= 4096 && EB == 2) ? 4 : 2;
-  static constexpr int NW_RAW = 65536 / (NS * STAGE);
+  static constexpr int NW_RAW = ((UNIT <= 2048 && !WIDE) ? 32768 : 65536) / (NS * STAGE);
   static constexpr int NW = NW_RAW < 1 ? 1 : (NW_RAW > 8 ? 8 : NW_RAW);
   static constexpr int SMEM_PIPE = NW * NS * STAGE;
   static constexpr int SMEM_BARS = NW * NS * 8;
@@ -147,13 +156,14 @@ __device__ __forceinline__ void quantize_e4m3(const uint32_t (&x)[EL / 2], float
 // workspace. (A template parameter, so that the plain form's code is not
 // touched by it.)
 template <typename T, typename TO, int D, int S, bool APPEND, typename TC = T,
-          bool CLUSTER = false, typename Prm = DecodeParams>
-__global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC)>::NW * 32)
+          bool CLUSTER = false, typename Prm = DecodeParams, bool WIDE = CLUSTER>
+__global__ void __launch_bounds__(DecodeTiling<D, S, sizeof(TC), WIDE>::NW * 32)
     paged_decode_partition_kernel(const Prm p) {
   constexpr int EB = sizeof(TC);
   static_assert(!APPEND || EB == 2 || std::is_same<Prm, DecodeParamsQ8>::value,
                 "the fused append over an E4M3 cache needs K's scale");
-  using Tl = DecodeTiling<D, S, EB>;
+  static_assert(WIDE || !CLUSTER, "cluster launches take the wide shapes");
+  using Tl = DecodeTiling<D, S, EB, WIDE>;
   constexpr int NW = Tl::NW, NS = Tl::NS, SLAB = Tl::SLAB, UNIT = Tl::UNIT, STAGE = Tl::STAGE;
   constexpr int EPL = Tl::EPL, LPR = Tl::LPR, RPW = Tl::RPW, CR = Tl::CR, NV = Tl::NV;
   constexpr int DUP = LPR / NV;  // lanes of a group holding the same row's score
@@ -660,17 +670,18 @@ inline cudaError_t launch_splitkv_reduce(const DecodeParams& p, cudaStream_t str
 }
 
 // Launches the partition pass (grid NP x H x B) and the merge: `kern_cl` in
-// clusters of NP CTAs that merge among themselves (dynamic shared memory
-// smem_cl), or `kern` as a plain grid (smem) followed by the merge kernel.
+// clusters of NP CTAs that merge among themselves (threads_cl threads, dynamic
+// shared memory smem_cl), or `kern` as a plain grid (threads, smem) followed
+// by the merge kernel.
 template <typename TO, int D, typename Kern, typename Prm>
 inline cudaError_t launch_partition_pass(Kern kern, Kern kern_cl, bool cluster, const Prm& p,
-                                         int threads, int smem, int smem_cl,
+                                         int threads, int smem, int threads_cl, int smem_cl,
                                          cudaStream_t stream) {
   const dim3 grid(p.NP, p.H, p.B);
   if (cluster) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads);
+    cfg.blockDim = dim3(threads_cl);
     cfg.dynamicSmemBytes = smem_cl;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

@@ -90,8 +90,11 @@ bool query_map(CUtensorMap* out, const void* q, int64_t T, int H, int D, pa_dtyp
 // Launchers (asynchronous on `stream`; the arguments are already checked).
 // cluster: launch the partition pass in clusters of prm.NP CTAs (NP of 2, 4
 // or 8) that merge a split among themselves, instead of the merge kernel.
+// wide: the grid (B * H * NP CTAs) holds at most two CTAs per SM, so the
+// partition pass takes its wide CTA shapes (DecodeTiling, WIDE).
 pa_status launch_decode16(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt, int D, int S,
-                          bool append, bool cluster, cudaStream_t stream);  // pa_k_decode.cu
+                          bool append, bool cluster, bool wide,
+                          cudaStream_t stream);                        // pa_k_decode.cu
 pa_status launch_grouped(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt, int D, int S,
                          bool append, cudaStream_t stream);             // pa_k_gqa.cu
 // grouped-query heads over E4M3 caches (q_dt: the queries' 16-bit type)
@@ -100,7 +103,7 @@ pa_status launch_grouped_fp8(const DecodeParams& prm, pa_dtype q_dt, pa_dtype ou
 // append: the new tokens' rows (prm.k_new / v_new, dtype q_dt) are quantized
 // with k_scale and prm.v_scale and written into the caches inside the launch.
 pa_status launch_decode_fp8(const DecodeParams& prm, pa_dtype q_dt, pa_dtype out_dt, int D,
-                            int S, bool cluster, bool append, float k_scale,
+                            int S, bool cluster, bool wide, bool append, float k_scale,
                             cudaStream_t stream);                       // pa_k_fp8.cu
 pa_status launch_prefill(const PrefillParams& prm, const void* q, pa_dtype dt, pa_dtype out_dt,
                          int D, int S, cudaStream_t stream);            // pa_k_prefill.cu
