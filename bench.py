@@ -248,7 +248,15 @@ class Workload:
                                   self.max_len, out_dtype=DTYPE, fused=True)
 
     def launches_per_step(self, fused=True):
-        return 1 if fused else 2
+        """Kernels one step launches: the partition pass, the split-KV merge
+        kernel when the plan splits and does not merge inside clusters (a
+        cluster merge needs 2, 4 or 8 partitions and a grid of at most two CTAs
+        per SM), and for the unfused step the append."""
+        _, NP = binding.pa_decode_plan(BATCH, H, D, S, self.max_seq, 0)
+        sms = torch.cuda.get_device_properties(self.device).multi_processor_count
+        cluster = NP in (2, 4, 8) and BATCH * H * NP <= 2 * sms
+        merge = 1 if NP > 1 and not cluster else 0
+        return 1 + merge + (0 if fused else 1)
 
     def device_step(self, ev_decode=None, fused=True):
         """One step on device-resident inputs. Fused: pa_decode_append (the new
