@@ -238,7 +238,8 @@ pa_status pa_decode_gqa_fp8(void* out, pa_dtype out_dt, const void* q, pa_dtype 
  * block_tables [B, MB] int32 device; seq_lens [B] int32 device.
  * q_start    [B + 1] int32 device: q_start[0] = 0, non-decreasing, q_start[B] = T.
  * T          rows of q and out (host copy of q_start[B]).
- * max_q_len  host bound on q_start[i+1] - q_start[i]; sets the launch grid.
+ * max_q_len  host bound on q_start[i+1] - q_start[i]; sets the launch grid
+ *            (at most 65535 * 128 = 8,388,480)
  * D          64, 128 or 256 (256: one 128-row query tile per CTA instead of two);
  *            S one of 8, 16, 32, 64, 128; NB * Hkv * S <= 2^31 - 1.
  * scale      finite and > 0 (the usual 1 / sqrt(D)).

@@ -451,7 +451,8 @@ pa_status pa_prefill(void* out, pa_dtype out_dt, const void* q, const void* k_ca
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
   if (NB == 0 || static_cast<int64_t>(NB) * Hkv * S > INT_MAX) return PA_ERR_INVALID;
-  if (ceil_div(max_q_len, 128) > INT_MAX / 2 || H > 65535 || B > 65535) return PA_ERR_INVALID;
+  // grid (H, row blocks of up to 256 rows, B): the y and z extents are 16-bit
+  if (ceil_div(max_q_len, 128) > 65535 || B > 65535) return PA_ERR_INVALID;
   pa::PrefillParams prm;
   prm.out = out;
   prm.k_cache = k_cache;

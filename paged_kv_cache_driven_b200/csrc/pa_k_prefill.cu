@@ -11,7 +11,11 @@ namespace pa {
 namespace host {
 namespace {
 
-// One CTA per (256 query rows, query head, request).
+// One CTA per (256 query rows, query head, request). The grid runs the heads
+// fastest, then a request's row blocks from the last (the longest, with the
+// most keys) to the first, then the requests: a request's longest CTAs of
+// every head start first, and its K/V stays in L2 while its heads run (one
+// 4096-token prompt on 32 heads: 0.278 -> 0.231 ms against row blocks fastest).
 template <typename T, typename TO, int D, int S>
 pa_status launch(const PrefillParams& prm, const void* q, cudaStream_t stream) {
   using Tl = PrefillTiling<D, std::is_same<T, __nv_bfloat16>::value>;
@@ -24,7 +28,7 @@ pa_status launch(const PrefillParams& prm, const void* q, cudaStream_t stream) {
   if (!query_map(&tmq, q, prm.T, prm.H, D, dt) || !row_map(&tmk, prm.k_cache, rows, D, S, dt) ||
       !row_map(&tmv, prm.v_cache, rows, D, S, dt))
     return PA_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>(ceil_div(prm.max_q_len, Tl::NQT * Tl::BM)), prm.H, prm.B);
+  const dim3 grid(prm.H, static_cast<unsigned>(ceil_div(prm.max_q_len, Tl::NQT * Tl::BM)), prm.B);
   kern<<<grid, Tl::THREADS, Tl::SMEM, stream>>>(prm, tmq, tmk, tmv);
   return cuda_status();
 }

@@ -200,18 +200,18 @@ __global__ void __launch_bounds__(576, 1)
   constexpr int BPT = Tl::BN / S;  // cache blocks per key tile
   static_assert(S >= 8 && S <= 128 && Tl::BN % S == 0, "block size 8 .. 128, dividing 128");
 
-  const int i = blockIdx.z, h = blockIdx.y;
+  const int i = blockIdx.z, h = blockIdx.x;
   const int L = p.seq_lens[i];
   const int q0 = p.q_start[i], q1 = p.q_start[i + 1];
   const int n = q1 - q0;
   if (L < 0 || L > static_cast<int64_t>(p.MB) * S || n < 0 || n > L || q0 < 0 || q1 > p.T ||
       n > p.max_q_len) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) raise_error(PA_DEVERR_SEQ_LEN);
+    if (threadIdx.x == 0 && blockIdx.y == 0 && h == 0) raise_error(PA_DEVERR_SEQ_LEN);
     return;
   }
   constexpr int ROWS = Tl::NQT * Tl::BM;
   const int ncta = (n + ROWS - 1) / ROWS;
-  const int ct = ncta - 1 - static_cast<int>(blockIdx.x);  // longest first
+  const int ct = ncta - 1 - static_cast<int>(blockIdx.y);  // longest first (grid: heads fastest)
   if (ct < 0) return;
   const int row0 = ct * ROWS;
   const int ctx = L - n;  // tokens cached before the first new one
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(576, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #ifdef PA_PREFILL_TRACE
-  const int trc = (h == 0 && i < 8 && blockIdx.x < 8) ? i * 8 + blockIdx.x : -1;
+  const int trc = (h == 0 && i < 8 && blockIdx.y < 8) ? i * 8 + blockIdx.y : -1;
   if (threadIdx.x == 0) PA_TRACE(31, 0);
 #endif
   if (threadIdx.x == 0) {

@@ -151,6 +151,7 @@ def prefill_args(**kw):
     dict(scale=0.0), dict(scale=-1.0), dict(scale=float("nan")), dict(Hkv=3), dict(Hkv=0),
     dict(q=NULL), dict(qs=NULL), dict(bt=NULL), dict(out=ctypes.c_void_p(16 * 1024 + 4)),
     dict(NB=0), dict(NB=1 << 28), dict(T=-1), dict(max_q_len=-1), dict(B=-1), dict(B=65536),
+    dict(max_q_len=65535 * 128 + 1),
 ])
 def test_prefill_rejects_bad_arguments_on_host(lib, bad):
     assert lib.pa_prefill(*prefill_args(**bad)) == binding.PA_ERR_INVALID
