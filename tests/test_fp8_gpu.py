@@ -178,6 +178,9 @@ def test_decode_fp8_bad_block_id_is_skipped_and_flagged():
     ([5, 64, 333], 2, 64, 8, torch.float16, torch.bfloat16, 32),
     ([7, 129, 700], 2, 256, 32, torch.bfloat16, torch.float16, 64),
     ([1332], 32, 128, 16, torch.bfloat16, torch.float32, 0),  # a cluster plan: 8 x 176 tokens
+    # large grids (more than two CTAs per SM): the half-width CTAs of small units
+    ([(37 * i) % 600 + 1 for i in range(24)], 8, 128, 16, torch.bfloat16, torch.float32, 64),
+    ([(53 * i) % 500 + 1 for i in range(24)], 4, 64, 8, torch.float16, torch.float32, 32),
 ])
 def test_decode_append_fp8_equals_two_calls(lens, H, D, S, in_dt, out_dt, partition):
     """pa_decode_append_fp8 quantizes each request's new row into its last slot
