@@ -518,7 +518,9 @@ def time_decode_case(case, iters, warmup, partition=0):
             times.append(a.elapsed_time(b))
     if binding.pa_get_device_error():
         raise SystemExit("device error word set")
-    return statistics.median(times), binding.pa_decode_plan(B, Hc, Dc, Sc, maxlen, partition)
+    Hkv = case.k_cache.shape[1]
+    return statistics.median(times), binding.pa_decode_plan_grouped(B, Hc, Hkv, Dc, Sc, maxlen,
+                                                                      partition)
 
 
 def time_decode_fp8(seed, iters, warmup):
@@ -609,7 +611,8 @@ def time_decode_gqa_fp8(seed, iters, warmup):
         raise SystemExit("device error word set")
     nbytes = sum(Hkv * 2 * L * Dc + Hq * 2 * Dc * 2 + 4 * (-(-L // Sc))
                  for L in case.seq_lens_host) + 4 * B
-    return statistics.median(times), nbytes, binding.pa_decode_plan(B, Hq, Dc, Sc, maxlen, 0)
+    return statistics.median(times), nbytes, binding.pa_decode_plan_grouped(B, Hq, Hkv, Dc, Sc,
+                                                                             maxlen, 0)
 
 
 def latency_floors(device, iters, warmup):

@@ -115,6 +115,10 @@ pa_status pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping
  * results in the workspace (layout below) for a merge kernel. Both merges do
  * the same arithmetic in the same order: the output bits do not depend on
  * which one ran.
+ * pa_decode_workspace_bytes: the workspace any decode entry point needs for
+ * these arguments (H the query heads), the grouped-query plans of every Hkv
+ * included (pa_decode_plan_grouped); 0 when nothing splits or the arguments
+ * are bad.
  * ------------------------------------------------------------------------- */
 size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, int partition);
 
@@ -131,6 +135,16 @@ size_t pa_decode_workspace_bytes(int B, int H, int D, int S, int max_seq_len, in
  * within two CTAs per SM, so that the split merges inside clusters. */
 pa_status pa_decode_plan(int B, int H, int D, int S, int max_seq_len, int partition,
                          int* partition_tokens, int* num_partitions);
+
+/* The plan of pa_decode_gqa / pa_decode_gqa_fp8 with Hkv KV heads (H a multiple
+ * of Hkv; Hkv == H gives pa_decode_plan). Their partition pass has
+ * B * Hkv * ceil(H / Hkv / 16) CTAs per partition, so an automatic plan whose
+ * 512-token grid holds at most two CTAs per SM halves the partitions (down to
+ * 128 tokens, multiples of S) while the grid stays within that bound; other
+ * grids take pa_decode_plan's choice. pa_decode_workspace_bytes(B, H, ...)
+ * covers this plan for every Hkv. PA_ERR_INVALID for bad arguments. */
+pa_status pa_decode_plan_grouped(int B, int H, int Hkv, int D, int S, int max_seq_len,
+                                 int partition, int* partition_tokens, int* num_partitions);
 
 pa_status pa_decode(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
                     const void* v_cache, const int32_t* block_tables, int MB,
@@ -272,7 +286,8 @@ pa_status pa_prefill(void* out, pa_dtype out_dt, const void* q, const void* k_ca
  * appended at position seq_lens[i] - 1 first, exactly as pa_decode_append.
  * Everything else (dtypes, D, S, partition, workspace sized by
  * pa_decode_workspace_bytes(B, H, ...) with H the query heads, errors) is as
- * pa_decode. H == Hkv gives pa_decode / pa_decode_append bit for bit.
+ * pa_decode, except that the automatic plan is pa_decode_plan_grouped's.
+ * H == Hkv gives pa_decode / pa_decode_append bit for bit.
  * ------------------------------------------------------------------------- */
 pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k_new,
                         const void* v_new, void* k_cache, void* v_cache,

@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     PA_ERR_CUDA, PA_ERR_INVALID, PA_ERR_OOM, PA_ERR_OUT_OF_RANGE, PA_F16, PA_F32, PA_OK,
     BlockAllocator, PagedAttnError, lib, pa_decode, pa_decode_append, pa_decode_append_fp8,
     pa_decode_fp8, pa_decode_gqa_fp8,
-    pa_decode_gqa, pa_decode_noalloc, pa_decode_plan, pa_decode_workspace_bytes,
+    pa_decode_gqa, pa_decode_noalloc, pa_decode_plan, pa_decode_plan_grouped,
+    pa_decode_workspace_bytes,
     pa_copy_blocks, pa_get_device_error, pa_kv_append, pa_kv_append_fp8, pa_prefill,
 )

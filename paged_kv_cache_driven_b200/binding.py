@@ -29,6 +29,7 @@ _SIGNATURES = {
     "pa_kv_append": ([_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "pa_decode_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32, _i32], _sz),
     "pa_decode_plan": ([_i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
+    "pa_decode_plan_grouped": ([_i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp], _i32),
     "pa_decode": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, ctypes.c_float, _i32, _i32, _i32,
                    _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp], _i32),
     "pa_get_device_error": ([_vp, _vp], _i32),
@@ -170,6 +171,16 @@ def pa_decode_plan(B, H, D, S, max_seq_len, partition=0):
     P, NP = ctypes.c_int(), ctypes.c_int()
     _check(lib().pa_decode_plan(B, H, D, S, max_seq_len, partition, ctypes.byref(P),
                                 ctypes.byref(NP)), "pa_decode_plan")
+    return P.value, NP.value
+
+
+def pa_decode_plan_grouped(B, H, Hkv, D, S, max_seq_len, partition=0):
+    """The plan of pa_decode_gqa / pa_decode_gqa_fp8: (partition_tokens,
+    num_partitions); (0, 1) = single pass."""
+    P, NP = ctypes.c_int(), ctypes.c_int()
+    _check(lib().pa_decode_plan_grouped(B, H, Hkv, D, S, max_seq_len, partition,
+                                        ctypes.byref(P), ctypes.byref(NP)),
+           "pa_decode_plan_grouped")
     return P.value, NP.value
 
 

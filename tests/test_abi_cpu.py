@@ -105,6 +105,33 @@ def test_workspace_and_plan(lib):
         binding.pa_decode_plan(1, 1, 128, 16, 100, partition=20)
 
 
+def test_grouped_plan(lib):
+    """Grouped-query heads: the partition pass has B * Hkv * ceil(G / 16) CTAs
+    per partition; a grid within 2 CTAs per SM (296 without a device) at 512
+    tokens halves its partitions (down to 128) while it stays within that."""
+    # 64 query heads on 8 KV heads: 8 CTAs per partition for one request
+    assert binding.pa_decode_plan_grouped(1, 64, 8, 128, 16, 1332) == (128, 11)
+    assert binding.pa_decode_plan_grouped(1, 64, 8, 128, 16, 4096) == (128, 32)
+    assert binding.pa_decode_plan_grouped(4, 64, 8, 128, 16, 2048) == (256, 8)  # 512 CTAs at 128
+    assert binding.pa_decode_plan_grouped(1, 64, 8, 128, 16, 100) == (0, 1)
+    # blocks of 32 still halve to 128; 8 KV heads x 2 chunks (G = 32)
+    assert binding.pa_decode_plan_grouped(1, 256, 8, 128, 32, 1332) == (128, 11)
+    # larger grids, explicit partitions and Hkv == H take pa_decode_plan's choice
+    assert binding.pa_decode_plan_grouped(64, 64, 8, 128, 16, 2048) == (512, 4)
+    assert binding.pa_decode_plan_grouped(1, 64, 8, 128, 16, 1332, partition=64) == (64, 21)
+    assert binding.pa_decode_plan_grouped(1, 32, 32, 128, 16, 1332) == \
+        binding.pa_decode_plan(1, 32, 128, 16, 1332)
+    for bad in ((1, 64, 0), (1, 64, 7), (1, 0, 1)):
+        with pytest.raises(binding.PagedAttnError):
+            binding.pa_decode_plan_grouped(*bad, 128, 16, 1332)
+    # the workspace covers the grouped plan of every Hkv (H = 64: at most 11
+    # partitions of 1332 tokens; the one-head-per-KV-head plan has 4)
+    assert binding.pa_decode_plan(1, 64, 128, 16, 1332)[1] == 4
+    n = 1 * 64 * 11
+    want = ((n * 8 + 255) // 256) * 256 + n * 128 * 4
+    assert binding.pa_decode_workspace_bytes(1, 64, 128, 16, 1332) == want
+
+
 def append_args(**kw):
     a = dict(k=P, v=P, slots=P, kc=P, vc=P, T=4, H=2, D=64, S=16, NB=8, dt=binding.PA_F16,
              stream=NULL)
