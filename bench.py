@@ -996,6 +996,12 @@ def prefill_trace_phases(buf):
         if buf[cta, 31, 0] == 0:
             continue
         nk = int((buf[cta, 20, :] > 0).sum())
+        # the CTA's start to its first scores (tile 0, first half), and its
+        # whole run
+        if buf[cta, 0, 0]:
+            add("CTA start to its first scores ready (prologue)", buf[cta, 0, 0] - buf[cta, 31, 0])
+        if buf[cta, 30, 0]:
+            add("CTA start to end", buf[cta, 30, 0] - buf[cta, 31, 0])
         for j in range(2, nk - 1):
             for t in range(2):
                 for hw in range(2):
