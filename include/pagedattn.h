@@ -334,7 +334,7 @@ pa_status pa_decode_gqa(void* out, pa_dtype out_dt, const void* q, const void* k
  * ------------------------------------------------------------------------- */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
 
-/* The size of that array in this build of the library (PA_NOALLOC_SCRATCH_BYTES). */
+/* The size of that array as compiled into the library (PA_NOALLOC_SCRATCH_BYTES). */
 size_t pa_noalloc_scratch_bytes(void);
 
 pa_status pa_decode_noalloc(void* out, pa_dtype out_dt, const void* q, const void* k_cache,
