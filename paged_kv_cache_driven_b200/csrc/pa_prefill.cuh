@@ -20,11 +20,13 @@
 //              sum in fp32, writes the weights P back over the scores as 16-bit
 //              pairs (bf16 as hi + lo halves, so the weights keep ~16 bits), and
 //              rescales its output columns when the reference max moves;
-//   warp 16    producer: TMA loads of the two Q tiles and of 128-key K / V
-//              tiles, one box per (cache block, 64-column block); K and V run
-//              two tiles ahead (four for head size 64); lane b reads the table
-//              entry of block b of a tile and issues its boxes, so a tile's
-//              boxes go out in parallel;
+//   warp 16    producer: initialises the barriers, then TMA loads of the two
+//              Q tiles and of 128-key K / V tiles, one box per (cache block,
+//              64-column block); Q and the first K tile go out before the
+//              CTA-wide sync, overlapping the tensor-memory allocation; K and V
+//              run two tiles ahead (four for head size 64); lane b reads the
+//              table entry of block b of a tile and issues its boxes, so a
+//              tile's boxes go out in parallel;
 //   warp 17    MMA issuer (lane 0) and tensor-memory owner, also zeroing V rows
 //              past the end of the request in the last key tile:
 //              S_t = Q_t K^T (both operands K-major in shared memory) and
@@ -256,27 +258,73 @@ __global__ void __launch_bounds__(576, 1)
   const int trc = (h == 0 && i < 8 && blockIdx.y < 8) ? i * 8 + blockIdx.y : -1;
   if (threadIdx.x == 0) PA_TRACE(31, 0);
 #endif
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < Tl::KST; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-    }
-    for (int s = 0; s < Tl::VST; ++s) {
-      mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
-    }
-    for (int t = 0; t < Tl::NQT; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 256);
-      mbar_init(&o_done[t], 1);
-      mbar_init(&xch_bar[t], 256);
-    }
-    mbar_init(mma_done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
   constexpr int kProducer = 4 * Tl::NQT * 2, kIssuer = kProducer + 1;  // warps 16, 17
+  const int nblk = (L + S - 1) / S;
+  const int32_t* table = p.block_tables + static_cast<int64_t>(i) * p.MB;
+  // this lane's block id in key tile j (-1: none or invalid)
+  auto block_id = [&](int j) {
+    const int lb = j * BPT + lane;
+    int id = -1;
+    if (lane < BPT && lb < nblk) {
+      id = table[lb];
+      if (id < 0 || id >= p.NB) {
+        raise_error(PA_DEVERR_BLOCK_ID);
+        id = -1;
+      }
+    }
+    return id;
+  };
+  // one K or V tile: every lane issues the boxes of its block
+  auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full, int id) {
+    const int nvalid = __popc(__ballot_sync(kFullMask, id >= 0));
+    if (lane == 0)
+      mbar_arrive_expect_tx(full, static_cast<uint32_t>(nvalid) * S * 128 * Tl::COLB);
+    __syncwarp();
+    if (id >= 0) {
+      const int y = (id * p.Hkv + hk) * S;
+#pragma unroll
+      for (int c = 0; c < Tl::COLB; ++c)
+        tma_load_2d_nohint(dst + c * Tl::CB_BYTES + lane * S * 128, map, c * 64, y, full);
+    }
+  };
+  // The producer initialises the barriers and issues Q and the first K tile
+  // before the CTA-wide sync, so that their latency overlaps the tensor-memory
+  // allocation and the sync.
+  int id_v = -1, id_k = -1;
+  if (warp == kProducer) {
+    if (lane == 0) {
+      mbar_init(q_full, 1);
+      for (int s = 0; s < Tl::KST; ++s) {
+        mbar_init(&k_full[s], 1);
+        mbar_init(&k_empty[s], 1);
+      }
+      for (int s = 0; s < Tl::VST; ++s) {
+        mbar_init(&v_full[s], 1);
+        mbar_init(&v_empty[s], 1);
+      }
+      for (int t = 0; t < Tl::NQT; ++t) {
+        mbar_init(&s_full[t], 1);
+        mbar_init(&p_full[t], 256);
+        mbar_init(&o_done[t], 1);
+        mbar_init(&xch_bar[t], 256);
+      }
+      mbar_init(mma_done, 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, nq * Tl::Q_BYTES);
+      for (int t = 0; t < nq; ++t)
+#pragma unroll
+        for (int c = 0; c < Tl::COLB; ++c)
+          tc::tma_load_3d(sQ + t * Tl::Q_BYTES + c * Tl::CB_BYTES, &tmq, c * 64, h,
+                          q0 + row0 + t * Tl::BM, q_full);
+    }
+    id_v = block_id(0);
+    id_k = id_v;
+    load_tile(&tmk, sK, &k_full[0], id_k);
+  }
   if (warp == kIssuer) {
     __syncwarp();
     tc::tmem_alloc(tmem_slot, Tl::TMEM_COLS);
@@ -286,51 +334,11 @@ __global__ void __launch_bounds__(576, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-
   if (warp == kProducer) {
     // ---------------- producer: lane b loads cache block b of each key tile ----------------
-    if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, nq * Tl::Q_BYTES);
-      for (int t = 0; t < nq; ++t)
-#pragma unroll
-        for (int c = 0; c < Tl::COLB; ++c)
-          tc::tma_load_3d(sQ + t * Tl::Q_BYTES + c * Tl::CB_BYTES, &tmq, c * 64, h,
-                          q0 + row0 + t * Tl::BM, q_full);
-    }
-    const int nblk = (L + S - 1) / S;
-    const int32_t* table = p.block_tables + static_cast<int64_t>(i) * p.MB;
-    // this lane's block id in key tile j (-1: none or invalid)
-    auto block_id = [&](int j) {
-      const int lb = j * BPT + lane;
-      int id = -1;
-      if (lane < BPT && lb < nblk) {
-        id = table[lb];
-        if (id < 0 || id >= p.NB) {
-          raise_error(PA_DEVERR_BLOCK_ID);
-          id = -1;
-        }
-      }
-      return id;
-    };
-    // one K or V tile: every lane issues the boxes of its block
-    auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full, int id) {
-      const int nvalid = __popc(__ballot_sync(kFullMask, id >= 0));
-      if (lane == 0)
-        mbar_arrive_expect_tx(full, static_cast<uint32_t>(nvalid) * S * 128 * Tl::COLB);
-      __syncwarp();
-      if (id >= 0) {
-        const int y = (id * p.Hkv + hk) * S;
-#pragma unroll
-        for (int c = 0; c < Tl::COLB; ++c)
-          tma_load_2d_nohint(dst + c * Tl::CB_BYTES + lane * S * 128, map, c * 64, y, full);
-      }
-    };
     // K(j + 1) goes out before V(j); block ids are read one tile ahead
-    int id_v = block_id(0), id_k = id_v;
-    int k_issued = 0, v_issued = 0;
+    int k_issued = 1, v_issued = 0;
     bool ok = true;
-    load_tile(&tmk, sK, &k_full[0], id_k);
-    k_issued = 1;
     if (NK > 1) id_k = block_id(1);
     for (int j = 0; j < NK; ++j) {
       if (j + 1 < NK) {
