@@ -309,3 +309,30 @@ def test_noalloc_size_check_and_exported_limit(lib):
     assert need > limit
     assert lib.pa_decode_noalloc(*noalloc_args(**big)) == binding.PA_ERR_OOM
     assert lib.pa_decode_noalloc(*noalloc_args(B=0, q=NULL, out=NULL)) == binding.PA_OK
+
+
+def test_grouped_plan_invariants(lib):
+    """For a seeded spread of batch sizes, head groupings, block sizes and
+    lengths: every plan covers the length in whole blocks, and the workspace
+    pa_decode_workspace_bytes reports holds the partials of the grouped plan of
+    any KV-head count (the entry points refuse a smaller one)."""
+    import random
+    rng = random.Random(7)
+    D = 128
+    for _ in range(400):
+        B = rng.choice([1, 2, 3, 4, 8, 16, 33, 64, 200])
+        H = rng.choice([1, 2, 8, 32, 40, 64, 128])
+        divisors = [k for k in range(1, H + 1) if H % k == 0]
+        Hkv = rng.choice(divisors)
+        S = rng.choice([8, 16, 32])
+        L = rng.choice([0, 1, 15, 100, 513, 1332, 2048, 4096, 40000, 131072])
+        P, NP = binding.pa_decode_plan_grouped(B, H, Hkv, D, S, L)
+        if NP == 1:
+            assert P == 0
+        else:
+            # whole blocks, the length covered; a re-cut into a power of two
+            # may leave the last one or two partitions without a token
+            assert P % S == 0 and P >= 48 and P * NP >= L and NP - -(-L // P) <= 2
+        n = B * H * NP
+        need = 0 if NP == 1 else ((n * 8 + 255) // 256) * 256 + n * D * 4
+        assert binding.pa_decode_workspace_bytes(B, H, D, S, L) >= need, (B, H, Hkv, S, L)
