@@ -50,15 +50,17 @@ namespace pa {
 //            stage, so the stage size no longer grows with S; a block of S rows
 //            is S / CR units
 //   NS, NW   stages per warp and warps per CTA: about 64 KB of stages per CTA.
-//            Grids of more than two CTAs per SM (WIDE = false) with units of
-//            2 KB or less take 32 KB: half the warps, each walking twice the
-//            blocks of a partition, so that pipeline fill and drain weigh half
-//            as much and twice the CTAs share an SM (head_dim 64 at blocks 8
-//            and 16: 5-12 % faster from batch 32 up; the 13B-shaped E4M3
-//            decode 124 -> 108 us). Smaller grids (WIDE = true, cluster
-//            launches among them) keep the wider CTAs, which spread their few
-//            CTAs' work over more warps (batch 1, head_dim 128, block 8: 14.4
-//            against 17.4 us).
+//            Grids of more than four CTAs per SM (WIDE = false) with units of
+//            2 KB or less at head_dim 64 or over E4M3 caches take 32 KB: half
+//            the warps, each walking twice the blocks of a partition, so that
+//            pipeline fill and drain weigh half as much and twice the CTAs
+//            share an SM (head_dim 64 at blocks 8 and 16: 5-12 % faster from
+//            batch 32 up; the 13B-shaped E4M3 decode 124 -> 108 us). Smaller
+//            grids (WIDE = true, cluster launches among them) keep the wider
+//            CTAs, which spread their few CTAs' work over more warps (batch
+//            1, head_dim 128, block 8: 14.4 against 17.4 us), and so does
+//            16-bit head_dim 128 at block 8 (narrow CTAs: 99 against 89 us at
+//            batch 8, 2.441 against 2.476 ms at batch 256).
 template <int D, int S, int EB = 2, bool WIDE = false>
 struct DecodeTiling {
   static constexpr int EPL = 16 / EB;
@@ -73,7 +75,8 @@ struct DecodeTiling {
   // E4M3 units carry twice the elements per byte, so more warps (two stages
   // each) keep the same bytes in flight with twice the threads to convert them
   static constexpr int NS = (STAGE <= 4096 && EB == 2) ? 4 : 2;
-  static constexpr int NW_RAW = ((UNIT <= 2048 && !WIDE) ? 32768 : 65536) / (NS * STAGE);
+  static constexpr bool NARROW = !WIDE && UNIT <= 2048 && (EB == 1 || D <= 64);
+  static constexpr int NW_RAW = (NARROW ? 32768 : 65536) / (NS * STAGE);
   static constexpr int NW = NW_RAW < 1 ? 1 : (NW_RAW > 8 ? 8 : NW_RAW);
   static constexpr int SMEM_PIPE = NW * NS * STAGE;
   static constexpr int SMEM_BARS = NW * NS * 8;

@@ -90,8 +90,9 @@ bool query_map(CUtensorMap* out, const void* q, int64_t T, int H, int D, pa_dtyp
 // Launchers (asynchronous on `stream`; the arguments are already checked).
 // cluster: launch the partition pass in clusters of prm.NP CTAs (NP of 2, 4
 // or 8) that merge a split among themselves, instead of the merge kernel.
-// wide: the grid (B * H * NP CTAs) holds at most two CTAs per SM, so the
-// partition pass takes its wide CTA shapes (DecodeTiling, WIDE).
+// wide: the grid (B * H * NP CTAs) holds at most four CTAs per SM, so the
+// partition pass takes its wide CTA shapes (DecodeTiling, WIDE); a cluster
+// launch (at most two CTAs per SM) always does.
 pa_status launch_decode16(const DecodeParams& prm, pa_dtype dt, pa_dtype out_dt, int D, int S,
                           bool append, bool cluster, bool wide,
                           cudaStream_t stream);                        // pa_k_decode.cu
